@@ -1,0 +1,599 @@
+// gemm_tc.cu -- grouped GEMM on the 5th-generation tensor cores (tcgen05, accumulators in
+// tensor memory) for the expert FFN and the router logits (sm_100a).
+//
+// Expert FFN ("Expert Networks > Worked Example: Expert Specialization", token-0 trace: h = W1 x
+// + b1, a = SiLU(h), y = W2 a + b2; closing paragraph: each expert processes its kept tokens as
+// one batch):
+//   GEMM1: H[r, :] = SiLU(x[rowtok[r]] . W1[e]^T + b1[e])   rows r of expert e, gather folded
+//          into the A-operand load (the fused-MoE dataflow diagram's "GEMM 1 reads row p //
+//          top_k" idea, here indexed by expert-sorted row rather than pair order);
+//   GEMM2: Y[r, :] = H[r] . W2[e]^T + b2[e].
+// Router logits: L = x . [Wr_hi | Wr_mid | Wr_lo] with Wr split exactly into three bf16 terms;
+// the epilogue adds the three fp32 partial products and the router bias.
+//
+// One persistent CTA per SM walks a static list of (expert, 128-row m-tile, BN-column n-tile)
+// tiles, n-tile fastest.  Warp roles (320 threads):
+//   warp 0      TMA producer for B (weights, K-major, 128-byte swizzle)
+//   warp 1      TMEM allocator and the single thread that issues tcgen05.mma
+//   warps 2-5   epilogue: tcgen05.ld from TMEM, bias + activation, bf16/fp32 stores
+//   warps 6-9   A producers: 16-byte cp.async of the 128 rows of the m-tile (gathered through
+//               rowtok for GEMM1) into the 128-byte-swizzled K-major layout
+// Pipeline: STAGES shared-memory stages (full/empty mbarriers) and two TMEM accumulators
+// (tmem_full/tmem_empty) so the epilogue of tile i overlaps the main loop of tile i+1.
+// Every wait is bounded (about 2 s) and reports MOE_DEV_TIMEOUT instead of hanging.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kBM = 128;            // rows per tile (tcgen05 M)
+constexpr int kBK = 64;             // K per stage: one 128-byte swizzle atom of bf16
+constexpr int kThreads = 320;
+constexpr int kTmemCols = 512;      // two accumulators at column 0 and 256
+constexpr int kMaxGroups = 1024;
+
+enum Epi { kEpiSiLU = 0, kEpiBias = 1, kEpiRouter = 2 };
+
+struct GemmArgs {
+    const __nv_bfloat16* A;   // [*, lda] row-major
+    long long lda;            // elements
+    const int32_t* a_rows;    // nullable: A row of tile row r is a_rows[r] (gather)
+    int a_row_limit;          // rows of A (bound for gathered indices)
+    const int32_t* offsets;   // [E+1] row ranges of the groups; null = one group of rows0 rows
+    int rows0;
+    int E;                    // groups
+    int K;                    // reduction length, multiple of 64
+    int n_tiles;              // column tiles per group
+    int b_rows_per_group;     // row stride between groups in B's tensor map
+    int Nout;                 // valid output columns per group
+    const float* bias;        // [E, Nout] (FFN) or [router_E] (router); nullable
+    void* D;                  // output
+    long long ldd;            // elements
+    int router_E;             // router epilogue: number of experts (columns of D)
+    DeviceStatus* st;
+};
+
+template <int BN>
+struct Cfg {
+    static constexpr int kABytes = kBM * kBK * 2;           // 16 KB
+    static constexpr int kBBytes = BN * kBK * 2;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStages = (200 * 1024) / kStageBytes > 8 ? 8 : (200 * 1024) / kStageBytes;
+    static constexpr int kBarOff = kStages * kStageBytes;
+    static constexpr int kTableOff = kBarOff + 256;
+    static constexpr int kSmemBytes = 1024 + kTableOff + (kMaxGroups + 1) * 4;
+    static_assert(kStages >= 2, "at least two stages");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 N for M=128");
+    static_assert(kBBytes % 1024 == 0, "B stage must stay 1024-byte aligned");
+};
+
+__device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+    asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
+
+// 16 consecutive fp32 columns of this thread's TMEM lane, waited for inside the same asm
+// statement so that no use of the registers can be scheduled before the load has landed.
+__device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, float* v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 32 consecutive fp32 columns, load and wait in one statement.
+__device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, float* v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+        "%28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Tile t -> (group, first row, valid rows, column tile).  s_mt[e] = m-tiles before group e.
+struct TileCoord {
+    int e, row0, rows, nt;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(int tile, const int* s_mt, int E, int n_tiles,
+                                                const GemmArgs& a) {
+    TileCoord c;
+    const int mt = tile / n_tiles;
+    c.nt = tile - mt * n_tiles;
+    int lo = 0, hi = E - 1;                 // largest e with s_mt[e] <= mt
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_mt[mid] <= mt) lo = mid; else hi = mid - 1;
+    }
+    c.e = lo;
+    const int g0 = a.offsets ? __ldg(a.offsets + lo) : 0;
+    const int g1 = a.offsets ? __ldg(a.offsets + lo + 1) : a.rows0;
+    c.row0 = g0 + (mt - s_mt[lo]) * kBM;
+    c.rows = min(kBM, g1 - c.row0);
+    return c;
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+    using C = Cfg<BN>;
+    constexpr int S = C::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* base_ptr = smem_raw + (base - raw);
+    const uint32_t bar0 = base + C::kBarOff;
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+    auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * S + b); };
+    auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * S + 2 + b); };
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base_ptr + C::kBarOff + 8 * (2 * S + 4));
+    int* s_mt = reinterpret_cast<int*>(base_ptr + C::kTableOff);
+    auto sA = [&](int s) { return base + (uint32_t)s * C::kABytes; };
+    auto sB = [&](int s) { return base + (uint32_t)S * C::kABytes + (uint32_t)s * C::kBBytes; };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = args.E;
+    DeviceStatus* st = args.st;
+
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full_bar(s), 1 + 128);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull_bar(b), 1);
+            mbar_init(tempty_bar(b), 128);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
+    }
+    if (warp == 1) {
+        __syncwarp();
+        tmem_alloc(smem_u32(s_tmem), kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 2) {
+        // m-tile prefix over groups: lane l sums groups [l*per, (l+1)*per).
+        const int per = (E + 31) / 32;
+        int loc = 0;
+        for (int q = 0; q < per; ++q) {
+            const int e = lane * per + q;
+            if (e < E) {
+                const int n = args.offsets ? __ldg(args.offsets + e + 1) - __ldg(args.offsets + e)
+                                           : args.rows0;
+                loc += (max(n, 0) + kBM - 1) / kBM;
+            }
+        }
+        int inc = loc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        int run = inc - loc;
+        for (int q = 0; q < per; ++q) {
+            const int e = lane * per + q;
+            if (e < E) {
+                s_mt[e] = run;
+                const int n = args.offsets ? __ldg(args.offsets + e + 1) - __ldg(args.offsets + e)
+                                           : args.rows0;
+                run += (max(n, 0) + kBM - 1) / kBM;
+            }
+        }
+        if (lane == 31) s_mt[E] = inc;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *s_tmem;
+    const int n_tiles = args.n_tiles;
+    const int total = s_mt[E] * n_tiles;
+    const int nkb = args.K / kBK;
+    constexpr uint32_t kIdesc = idesc_bf16_m128(BN);
+
+    if (warp == 0) {
+        // ---------------- B producer (TMA) ----------------
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+                const TileCoord tc = tile_coord(tile, s_mt, E, n_tiles, args);
+                const int brow = tc.e * args.b_rows_per_group + tc.nt * BN;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1u;
+                    if (!mbar_wait(empty_bar(s), ph ^ 1u, st, 1)) { ok = false; break; }
+                    mbar_arrive_expect_tx(full_bar(s), C::kBBytes);
+                    tma_load_2d(sB(s), &tmB, full_bar(s), kb * kBK, brow);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            uint32_t it = 0, lt = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++lt) {
+                const uint32_t b = lt & 1u, use = lt >> 1;
+                if (!mbar_wait(tempty_bar(b), (use & 1u) ^ 1u, st, 2)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + b * 256u;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1u;
+                    if (!mbar_wait(full_bar(s), ph, st, 3)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t da = smem_desc_sw128(sA(s));
+                    const uint64_t db = smem_desc_sw128(sB(s));
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        tc_mma_bf16(d_tmem, da + 2u * kk, db + 2u * kk, kIdesc,
+                                    (kb | kk) != 0 ? 1u : 0u);
+                    tc_commit(empty_bar(s));
+                }
+                if (!ok) break;
+                tc_commit(tfull_bar(b));
+            }
+        }
+    } else if (warp < 6) {
+        // ---------------- epilogue ----------------
+        const int q = warp & 3;                       // TMEM lane quadrant of this warp
+        const int r = q * 32 + lane;                  // tile row of this thread
+        uint32_t lt = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++lt) {
+            const TileCoord tc = tile_coord(tile, s_mt, E, n_tiles, args);
+            const uint32_t b = lt & 1u, use = lt >> 1;
+            if (!mbar_wait(tfull_bar(b), use & 1u, st, 4)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + b * 256u;
+            const bool row_ok = r < tc.rows;
+            const long long orow = (long long)tc.row0 + r;
+            if (EPI == kEpiRouter) {
+                constexpr int Eg = BN / 3;
+#pragma unroll 1
+                for (int c0 = 0; c0 < Eg; c0 += 16) {
+                    float hi[16], mi[16], lo[16];
+                    __syncwarp();
+                    tmem_ld16_wait(taddr + c0, hi);
+                    tmem_ld16_wait(taddr + Eg + c0, mi);
+                    tmem_ld16_wait(taddr + 2 * Eg + c0, lo);
+                    const int e0 = tc.nt * Eg + c0;
+                    if (row_ok) {
+                        float* out = reinterpret_cast<float*>(args.D) + orow * args.ldd;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int e = e0 + i;
+                            if (e < args.router_E) {
+                                float v = __fadd_rn(hi[i], __fadd_rn(mi[i], lo[i]));
+                                if (args.bias) v = __fadd_rn(v, __ldg(args.bias + e));
+                                out[e] = v;
+                            }
+                        }
+                    }
+                }
+            } else {
+                const int n0 = tc.nt * BN;
+                const float* bias = args.bias ? args.bias + (size_t)tc.e * args.Nout + n0 : nullptr;
+#pragma unroll 1
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    float v[32];
+                    const int ncol = (BN - c0) >= 32 ? 32 : 16;
+                    __syncwarp();
+                    if (ncol == 32) tmem_ld32_wait(taddr + c0, v);
+                    else tmem_ld16_wait(taddr + c0, v);
+                    if (!row_ok || n0 + c0 >= args.Nout) continue;
+                    const int nc = min(ncol, args.Nout - (n0 + c0));     // 16 or 32
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        if (i >= nc) break;
+                        float a0 = v[i], a1 = v[i + 1];
+                        if (bias) {
+                            a0 = __fadd_rn(a0, __ldg(bias + c0 + i));
+                            a1 = __fadd_rn(a1, __ldg(bias + c0 + i + 1));
+                        }
+                        if (EPI == kEpiSiLU) {
+                            a0 = __fdividef(a0, 1.0f + __expf(-a0));
+                            a1 = __fdividef(a1, 1.0f + __expf(-a1));
+                        }
+                        pk[i >> 1] = pack_bf16x2(a0, a1);
+                    }
+                    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(args.D) +
+                                         orow * args.ldd + n0 + c0;
+                    st_global_v4(out, pk[0], pk[1], pk[2], pk[3]);
+                    st_global_v4(out + 8, pk[4], pk[5], pk[6], pk[7]);
+                    if (nc == 32) {
+                        st_global_v4(out + 16, pk[8], pk[9], pk[10], pk[11]);
+                        st_global_v4(out + 24, pk[12], pk[13], pk[14], pk[15]);
+                    }
+                }
+            }
+            __syncwarp();
+            tc_fence_before();
+            mbar_arrive(tempty_bar(b));
+        }
+    } else {
+        // ---------------- A producers (cp.async, gathered rows) ----------------
+        const int at = threadIdx.x - 192;             // 0..127
+        const int chunk = at & 7;                     // 16-byte chunk of the 128-byte row
+        const int rbase = at >> 3;                    // rows rbase + 16 i
+        uint32_t it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+            const TileCoord tc = tile_coord(tile, s_mt, E, n_tiles, args);
+            const __nv_bfloat16* src[8];
+            uint32_t dst_off[8];
+            bool valid[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int r = rbase + 16 * i;
+                valid[i] = r < tc.rows;
+                long long ar = tc.row0 + r;
+                if (valid[i] && args.a_rows) {
+                    const int g = __ldg(args.a_rows + tc.row0 + r);
+                    if ((unsigned)g >= (unsigned)args.a_row_limit) {
+                        report(st, MOE_DEV_BAD_INDEX, 501);
+                        valid[i] = false;
+                    }
+                    ar = g;
+                }
+                src[i] = args.A + ar * args.lda + chunk * 8;
+                dst_off[i] = (uint32_t)r * 128u + (uint32_t)((chunk ^ (r & 7)) << 4);
+            }
+            for (int kb = 0; kb < nkb; ++kb, ++it) {
+                const int s = it % S;
+                const uint32_t ph = (it / S) & 1u;
+                if (!mbar_wait(empty_bar(s), ph ^ 1u, st, 5)) { ok = false; break; }
+                const uint32_t dA = sA(s);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    if (valid[i]) cp_async_16(dA + dst_off[i], src[i] + kb * kBK);
+                cp_async_commit();
+                if (it > 0) {
+                    cp_async_wait<1>();
+                    fence_proxy_async_smem();
+                    mbar_arrive(full_bar((it - 1) % S));
+                }
+            }
+        }
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        if (ok && it > 0) mbar_arrive(full_bar((it - 1) % S));
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// Wr [d, E] fp32 -> B rows for the router GEMM: for column tile nt, rows
+// nt*3Eg + {0, Eg, 2Eg} + c hold the hi/mid/lo bf16 terms of Wr[:, nt*Eg + c] (zero past E).
+__global__ void router_split_kernel(const float* __restrict__ Wr, int d, int E, int Eg, int ntl,
+                                    __nv_bfloat16* __restrict__ B) {
+    const long long total = (long long)ntl * 3 * Eg * d;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int col = (int)(i % d);
+        const int row = (int)(i / d);
+        const int nt = row / (3 * Eg), part = (row / Eg) % 3, c = row % Eg;
+        const int e = nt * Eg + c;
+        float v = 0.0f;
+        if (e < E) {
+            const float w = Wr[(size_t)col * E + e];
+            const float hi = __bfloat162float(__float2bfloat16_rn(w));
+            const float r1 = __fsub_rn(w, hi);
+            const float mid = __bfloat162float(__float2bfloat16_rn(r1));
+            const float r2 = __fsub_rn(r1, mid);
+            v = part == 0 ? hi : (part == 1 ? mid : r2);
+        }
+        B[i] = __float2bfloat16_rn(v);
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool encode_fn_ready() {
+    std::call_once(g_encode_once, []() {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode != nullptr;
+}
+
+// 2-D bf16 tensor map over rows x K (K contiguous), box 64 x box_rows, 128-byte swizzle.
+bool make_tmap(CUtensorMap* tm, const void* ptr, long long rows, int K, int box_rows) {
+    if (!encode_fn_ready()) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int g_num_sms = 0;
+
+int num_sms() {
+    if (g_num_sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (g_num_sms <= 0) g_num_sms = 148;
+    }
+    return g_num_sms;
+}
+
+template <int BN, int EPI>
+cudaError_t launch_gemm_t(const CUtensorMap& tm, const GemmArgs& a, int grid, cudaStream_t s) {
+    using C = Cfg<BN>;
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<BN, EPI>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_done = true;
+    }
+    grouped_gemm_kernel<BN, EPI><<<grid, kThreads, C::kSmemBytes, s>>>(tm, a);
+    return cudaGetLastError();
+}
+
+template <int EPI>
+cudaError_t launch_gemm_bn(int BN, const CUtensorMap& tm, const GemmArgs& a, int grid,
+                           cudaStream_t s) {
+    switch (BN) {
+        case 256: return launch_gemm_t<256, EPI>(tm, a, grid, s);
+        case 192: return launch_gemm_t<192, EPI>(tm, a, grid, s);
+        case 176: return launch_gemm_t<176, EPI>(tm, a, grid, s);
+        case 128: return launch_gemm_t<128, EPI>(tm, a, grid, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_router_bn(int BN, const CUtensorMap& tm, const GemmArgs& a, int grid,
+                             cudaStream_t s) {
+    switch (BN) {
+        case 192: return launch_gemm_t<192, kEpiRouter>(tm, a, grid, s);
+        case 96: return launch_gemm_t<96, kEpiRouter>(tm, a, grid, s);
+        case 48: return launch_gemm_t<48, kEpiRouter>(tm, a, grid, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+// Column tile for an output width: least padded work, then the wider tile.
+int pick_bn(int nout) {
+    const int cands[] = {256, 192, 176, 128};
+    int best = 256;
+    long long best_pad = -1;
+    for (int bn : cands) {
+        const long long pad = (long long)((nout + bn - 1) / bn) * bn;
+        if (best_pad < 0 || pad < best_pad) { best = bn; best_pad = pad; }
+    }
+    return best;
+}
+
+int router_group(int E) { return E <= 16 ? 16 : (E <= 32 ? 32 : 64); }
+
+cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const int32_t* a_rows,
+                               int a_row_limit, const int32_t* offsets, int E, int K, int Nout,
+                               const void* W, const float* bias, void* D, long long ldd,
+                               long long max_rows, DeviceStatus* st, cudaStream_t s,
+                               int* launches) {
+    const int BN = pick_bn(Nout);
+    CUtensorMap tm;
+    if (!make_tmap(&tm, W, (long long)E * Nout, K, BN)) return cudaErrorInvalidValue;
+    GemmArgs a{};
+    a.A = reinterpret_cast<const __nv_bfloat16*>(A);
+    a.lda = lda;
+    a.a_rows = a_rows;
+    a.a_row_limit = a_row_limit;
+    a.offsets = offsets;
+    a.rows0 = 0;
+    a.E = E;
+    a.K = K;
+    a.n_tiles = (Nout + BN - 1) / BN;
+    a.b_rows_per_group = Nout;
+    a.Nout = Nout;
+    a.bias = bias;
+    a.D = D;
+    a.ldd = ldd;
+    a.router_E = 0;
+    a.st = st;
+    const long long max_tiles = ((max_rows + kBM - 1) / kBM + E) * a.n_tiles;
+    const int grid = (int)std::min<long long>(num_sms(), std::max<long long>(max_tiles, 1));
+    cudaError_t e = which == 0 ? launch_gemm_bn<kEpiSiLU>(BN, tm, a, grid, s)
+                               : launch_gemm_bn<kEpiBias>(BN, tm, a, grid, s);
+    if (e == cudaSuccess) *launches += 1;
+    return e;
+}
+
+size_t router_split_bytes(int d, int E) {
+    const int Eg = router_group(E);
+    const int ntl = (E + Eg - 1) / Eg;
+    return (size_t)ntl * 3 * Eg * d * 2;
+}
+
+cudaError_t launch_router_gemm(const void* x, int T, int d, const float* Wr, const float* br,
+                               int E, void* split_buf, float* logits, DeviceStatus* st,
+                               cudaStream_t s, int* launches) {
+    const int Eg = router_group(E);
+    const int ntl = (E + Eg - 1) / Eg;
+    const int BN = 3 * Eg;
+    router_split_kernel<<<148 * 4, 256, 0, s>>>(Wr, d, E, Eg, ntl,
+                                                reinterpret_cast<__nv_bfloat16*>(split_buf));
+    *launches += 1;
+    CUtensorMap tm;
+    if (!make_tmap(&tm, split_buf, (long long)ntl * BN, d, BN)) return cudaErrorInvalidValue;
+    GemmArgs a{};
+    a.A = reinterpret_cast<const __nv_bfloat16*>(x);
+    a.lda = d;
+    a.a_rows = nullptr;
+    a.a_row_limit = T;
+    a.offsets = nullptr;
+    a.rows0 = T;
+    a.E = 1;
+    a.K = d;
+    a.n_tiles = ntl;
+    a.b_rows_per_group = 0;
+    a.Nout = ntl * Eg;
+    a.bias = br;
+    a.D = logits;
+    a.ldd = E;
+    a.router_E = E;
+    a.st = st;
+    const long long tiles = (long long)((T + kBM - 1) / kBM) * ntl;
+    const int grid = (int)std::min<long long>(num_sms(), std::max<long long>(tiles, 1));
+    cudaError_t e = launch_router_bn(BN, tm, a, grid, s);
+    if (e == cudaSuccess) *launches += 1;
+    return e;
+}
+
+}  // namespace moe

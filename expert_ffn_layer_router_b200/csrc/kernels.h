@@ -1,0 +1,53 @@
+// kernels.h -- launchers of the MoE kernels (internal to the library).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+namespace moe {
+
+struct DeviceStatus;
+
+// route.cu
+void launch_route_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
+                       cudaStream_t s);
+int chunk_count(int T);
+void launch_capacity_select(const int32_t* ids, const float* w, int T, int E, int k, long long K,
+                            int32_t* cnt, int32_t* base, int32_t* nrecv, int32_t* cand,
+                            int32_t* slot, uint8_t* drop, int32_t* counts, int32_t* offsets,
+                            int32_t* rowtok, DeviceStatus* st, cudaStream_t s, int* launches);
+void launch_dispatch(const int32_t* ids, const int32_t* slot, int T, int E, int k,
+                     int32_t* kept_tmp, int32_t* offsets, int32_t* rowtok, DeviceStatus* st,
+                     cudaStream_t s, int* launches);
+void launch_permute_rows(const void* x, const int32_t* rowtok, const int32_t* offsets, int E,
+                         size_t row_bytes, int T, long long max_rows, void* xp, DeviceStatus* st,
+                         cudaStream_t s, int* launches);
+
+// combine.cu
+void launch_combine(int dtype, const void* x, const void* Y, const float* w, const int32_t* ids,
+                    const int32_t* slot, const int32_t* offsets, int T, int d, int E, int k,
+                    void* out, DeviceStatus* st, cudaStream_t s, int* launches);
+void launch_ffn_f32(const float* x, const int32_t* rowtok, const int32_t* offsets, int E, int T,
+                    int d, int F, long long max_rows, const float* W1, const float* b1,
+                    const float* W2, const float* b2, float* H, float* Y, DeviceStatus* st,
+                    cudaStream_t s, int* launches);
+void launch_logits_f32(const float* x, const float* Wr, const float* br, int T, int d, int E,
+                       float* logits, cudaStream_t s, int* launches);
+
+// gemm_tc.cu
+int pick_bn(int nout);
+int router_group(int E);
+size_t router_split_bytes(int d, int E);
+// which = 0: D = SiLU(A W^T + bias) (GEMM1); which = 1: D = A W^T + bias (GEMM2).
+cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const int32_t* a_rows,
+                               int a_row_limit, const int32_t* offsets, int E, int K, int Nout,
+                               const void* W, const float* bias, void* D, long long ldd,
+                               long long max_rows, DeviceStatus* st, cudaStream_t s,
+                               int* launches);
+cudaError_t launch_router_gemm(const void* x, int T, int d, const float* Wr, const float* br,
+                               int E, void* split_buf, float* logits, DeviceStatus* st,
+                               cudaStream_t s, int* launches);
+
+}  // namespace moe

@@ -1,0 +1,323 @@
+// moe_api.cu -- the C ABI of include/moe_b200.h: argument checks, workspace layout and the
+// launch sequence of each call.  Nothing here allocates device memory or synchronises the host
+// (except moe_get_device_status, which by contract reads the status word back).
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+thread_local int32_t g_last_launches = 0;
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool bad_problem(const moe_problem* p) {
+    if (!p) return true;
+    if (p->T < 0 || p->d_model < 1 || p->d_ff < 1 || p->E < 1 || p->E > 1024) return true;
+    if (p->k < 1 || p->k > p->E || p->k > 32) return true;
+    if (std::isnan(p->capacity_factor) || p->capacity_factor < 0.0f) return true;
+    if (p->dtype != MOE_F32 && p->dtype != MOE_BF16) return true;
+    if (p->flags != 0) return true;
+    if ((long long)p->T * p->k > 0x7fffffffLL) return true;
+    if ((long long)p->T * p->E > 0x7fffffffLL) return true;
+    return false;
+}
+
+bool unsupported(const moe_problem* p) {
+    if (p->dtype == MOE_BF16) return (p->d_model % 64) != 0 || (p->d_ff % 64) != 0;
+    return false;
+}
+
+long long capacity_of(const moe_problem* p) {
+    if (std::isinf(p->capacity_factor)) return p->T;
+    const double v = std::floor((double)p->capacity_factor * (double)p->T * (double)p->k /
+                                (double)p->E);
+    return v > (double)p->T ? (long long)p->T : (long long)v;
+}
+
+size_t esize(const moe_problem* p) { return p->dtype == MOE_BF16 ? 2 : 4; }
+
+// Rows of the expert-sorted buffers: at most every pair, at most K per expert.
+long long max_rows_of(const moe_problem* p, long long K) {
+    return std::min<long long>((long long)p->T * p->k, (long long)p->E * K);
+}
+
+struct Plan {
+    size_t status, logits, ids, w, slot, drop, counts, cnt, base, nrecv, cand, offsets, rowtok,
+        kept_tmp, H, Y, split, total;
+};
+
+Plan make_plan(const moe_problem* p) {
+    const long long K = capacity_of(p);
+    const size_t P = (size_t)p->T * p->k;
+    const size_t R = (size_t)max_rows_of(p, K);
+    const size_t nC = (size_t)moe::chunk_count(p->T);
+    Plan q{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align_up(off + std::max<size_t>(bytes, 1));
+        return at;
+    };
+    q.status = take(sizeof(moe::DeviceStatus));
+    q.logits = take((size_t)p->T * p->E * 4);
+    q.ids = take(P * 4);
+    q.w = take(P * 4);
+    q.slot = take(P * 4);
+    q.drop = take(P);
+    q.counts = take((size_t)2 * p->E * 4);
+    q.cnt = take((size_t)p->E * nC * 4);
+    q.base = take((size_t)p->E * nC * 4);
+    q.nrecv = take((size_t)p->E * 4);
+    q.cand = take((size_t)p->E * p->T * 4);
+    q.offsets = take((size_t)(p->E + 1) * 4);
+    q.rowtok = take(R * 4);
+    q.kept_tmp = take((size_t)p->E * 4);
+    q.H = take(R * p->d_ff * esize(p));
+    q.Y = take(R * p->d_model * esize(p));
+    q.split = take(p->dtype == MOE_BF16 ? moe::router_split_bytes(p->d_model, p->E) : 0);
+    q.total = off;
+    return q;
+}
+
+template <class T>
+T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(ws) + off);
+}
+
+bool misaligned(const void* ptr, size_t a) { return ptr && (reinterpret_cast<uintptr_t>(ptr) % a); }
+
+moe_status check_ws(const moe_problem* p, const void* ws, size_t ws_bytes, Plan* plan) {
+    *plan = make_plan(p);
+    if (!ws || ws_bytes < plan->total || misaligned(ws, kAlign)) return MOE_ERR_WORKSPACE;
+    return MOE_OK;
+}
+
+moe_status finish(int launches) {
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    g_last_launches = launches;
+    return MOE_OK;
+}
+
+moe_status pre(const moe_problem* p) {
+    if (bad_problem(p)) return MOE_ERR_INVALID_ARG;
+    if (unsupported(p)) return MOE_ERR_UNSUPPORTED;
+    cudaGetLastError();   // a stale error from unrelated work must not be blamed on this call
+    return MOE_OK;
+}
+
+// Steps 1-2 on device data.  rowtok/offsets may be null (moe_route), counts always written.
+void route_steps(const moe_problem* p, const float* logits, int32_t* ids, float* w,
+                 int32_t* slot, uint8_t* drop, int32_t* counts, int32_t* offsets,
+                 int32_t* rowtok, void* ws, const Plan& q, cudaStream_t s, int* launches) {
+    moe::DeviceStatus* st = at<moe::DeviceStatus>(ws, q.status);
+    const long long K = capacity_of(p);
+    moe::launch_route_topk(logits, p->T, p->E, p->k, ids, w, s);
+    *launches += 1;
+    moe::launch_capacity_select(ids, w, p->T, p->E, p->k, K, at<int32_t>(ws, q.cnt),
+                                at<int32_t>(ws, q.base), at<int32_t>(ws, q.nrecv),
+                                at<int32_t>(ws, q.cand), slot, drop, counts, offsets, rowtok, st,
+                                s, launches);
+}
+
+moe_status ffn_steps(const moe_problem* p, const void* x, const int32_t* offsets,
+                     const int32_t* rowtok, const void* W1, const float* b1, const void* W2,
+                     const float* b2, void* Y, void* ws, const Plan& q, cudaStream_t s,
+                     int* launches) {
+    moe::DeviceStatus* st = at<moe::DeviceStatus>(ws, q.status);
+    const long long R = max_rows_of(p, capacity_of(p));
+    if (R == 0) return MOE_OK;
+    if (p->dtype == MOE_F32) {
+        moe::launch_ffn_f32((const float*)x, rowtok, offsets, p->E, p->T, p->d_model, p->d_ff, R,
+                            (const float*)W1, b1, (const float*)W2, b2, at<float>(ws, q.H),
+                            (float*)Y, st, s, launches);
+        return MOE_OK;
+    }
+    void* H = at<void>(ws, q.H);
+    if (moe::launch_expert_gemm(0, x, p->d_model, rowtok, p->T, offsets, p->E, p->d_model,
+                                p->d_ff, W1, b1, H, p->d_ff, R, st, s, launches) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (moe::launch_expert_gemm(1, H, p->d_ff, nullptr, (int)R, offsets, p->E, p->d_ff,
+                                p->d_model, W2, b2, Y, p->d_model, R, st, s, launches) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_capacity(const moe_problem* p, int64_t* K) {
+    if (bad_problem(p) || !K) return MOE_ERR_INVALID_ARG;
+    *K = capacity_of(p);
+    return MOE_OK;
+}
+
+moe_status moe_workspace_size(const moe_problem* p, size_t* bytes) {
+    if (bad_problem(p) || !bytes) return MOE_ERR_INVALID_ARG;
+    *bytes = make_plan(p).total;
+    return MOE_OK;
+}
+
+moe_status moe_route(const moe_problem* p, const float* logits, int32_t* ids, float* w,
+                     int32_t* slot, uint8_t* drop, int32_t* counts, void* ws, size_t ws_bytes,
+                     void* stream) {
+    moe_status r = pre(p);
+    if (r != MOE_OK) return r;
+    if (!counts || (p->T > 0 && (!logits || !ids || !w || !slot || !drop)))
+        return MOE_ERR_INVALID_ARG;
+    Plan q;
+    if ((r = check_ws(p, ws, ws_bytes, &q)) != MOE_OK) return r;
+    cudaStream_t s = (cudaStream_t)stream;
+    int launches = 0;
+    if (p->T == 0) {
+        cudaMemsetAsync(counts, 0, sizeof(int32_t) * 2 * p->E, s);
+        return finish(0);
+    }
+    route_steps(p, logits, ids, w, slot, drop, counts, nullptr, nullptr, ws, q, s, &launches);
+    return finish(launches);
+}
+
+moe_status moe_dispatch(const moe_problem* p, const int32_t* ids, const int32_t* slot,
+                        int32_t* offsets, int32_t* rowtok, const void* x, void* x_perm,
+                        void* ws, size_t ws_bytes, void* stream) {
+    moe_status r = pre(p);
+    if (r != MOE_OK) return r;
+    if (!offsets || (p->T > 0 && (!ids || !slot || !rowtok))) return MOE_ERR_INVALID_ARG;
+    if (x_perm && !x) return MOE_ERR_INVALID_ARG;
+    Plan q;
+    if ((r = check_ws(p, ws, ws_bytes, &q)) != MOE_OK) return r;
+    cudaStream_t s = (cudaStream_t)stream;
+    int launches = 0;
+    moe::DeviceStatus* st = at<moe::DeviceStatus>(ws, q.status);
+    moe::launch_dispatch(ids, slot, p->T, p->E, p->k, at<int32_t>(ws, q.kept_tmp), offsets,
+                         rowtok, st, s, &launches);
+    if (x_perm && p->T > 0)
+        moe::launch_permute_rows(x, rowtok, offsets, p->E, (size_t)p->d_model * esize(p), p->T,
+                                 max_rows_of(p, capacity_of(p)), x_perm, st, s, &launches);
+    return finish(launches);
+}
+
+moe_status moe_expert_ffn(const moe_problem* p, const void* x, const int32_t* offsets,
+                          const int32_t* rowtok, const void* W1, const float* b1,
+                          const void* W2, const float* b2, void* Y, void* ws, size_t ws_bytes,
+                          void* stream) {
+    moe_status r = pre(p);
+    if (r != MOE_OK) return r;
+    if (!offsets || !W1 || !W2 || (p->T > 0 && (!x || !rowtok || !Y))) return MOE_ERR_INVALID_ARG;
+    if (p->dtype == MOE_BF16 &&
+        (misaligned(x, 16) || misaligned(W1, 16) || misaligned(W2, 16) || misaligned(Y, 16)))
+        return MOE_ERR_INVALID_ARG;
+    Plan q;
+    if ((r = check_ws(p, ws, ws_bytes, &q)) != MOE_OK) return r;
+    int launches = 0;
+    if (p->T == 0) return finish(0);
+    r = ffn_steps(p, x, offsets, rowtok, W1, b1, W2, b2, Y, ws, q, (cudaStream_t)stream,
+                  &launches);
+    if (r != MOE_OK) return r;
+    return finish(launches);
+}
+
+moe_status moe_combine(const moe_problem* p, const void* x, const void* Y, const float* w,
+                       const int32_t* ids, const int32_t* slot, const int32_t* offsets,
+                       void* out, void* stream) {
+    moe_status r = pre(p);
+    if (r != MOE_OK) return r;
+    if (p->T > 0 && (!x || !Y || !w || !ids || !slot || !offsets || !out))
+        return MOE_ERR_INVALID_ARG;
+    if (out && (out == x || out == Y)) return MOE_ERR_INVALID_ARG;
+    int launches = 0;
+    moe::launch_combine(p->dtype, x, Y, w, ids, slot, offsets, p->T, p->d_model, p->E, p->k,
+                        out, nullptr, (cudaStream_t)stream, &launches);
+    return finish(launches);
+}
+
+moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, const float* br,
+                       const void* W1, const float* b1, const void* W2, const float* b2,
+                       void* out, float* logits_out, int32_t* ids_out, float* w_out,
+                       int32_t* slot_out, uint8_t* drop_out, int32_t* counts_out, void* ws,
+                       size_t ws_bytes, void* stream) {
+    moe_status r = pre(p);
+    if (r != MOE_OK) return r;
+    if (!Wr || !W1 || !W2 || (p->T > 0 && (!x || !out))) return MOE_ERR_INVALID_ARG;
+    if (out && out == x) return MOE_ERR_INVALID_ARG;
+    if (p->dtype == MOE_BF16 &&
+        (misaligned(x, 16) || misaligned(W1, 16) || misaligned(W2, 16) || misaligned(out, 16)))
+        return MOE_ERR_INVALID_ARG;
+    Plan q;
+    if ((r = check_ws(p, ws, ws_bytes, &q)) != MOE_OK) return r;
+    cudaStream_t s = (cudaStream_t)stream;
+    int launches = 0;
+    int32_t* counts = counts_out ? counts_out : at<int32_t>(ws, q.counts);
+    if (p->T == 0) {
+        cudaMemsetAsync(counts, 0, sizeof(int32_t) * 2 * p->E, s);
+        return finish(0);
+    }
+    moe::DeviceStatus* st = at<moe::DeviceStatus>(ws, q.status);
+    float* logits = logits_out ? logits_out : at<float>(ws, q.logits);
+    int32_t* ids = ids_out ? ids_out : at<int32_t>(ws, q.ids);
+    float* w = w_out ? w_out : at<float>(ws, q.w);
+    int32_t* slot = slot_out ? slot_out : at<int32_t>(ws, q.slot);
+    uint8_t* drop = drop_out ? drop_out : at<uint8_t>(ws, q.drop);
+    int32_t* offsets = at<int32_t>(ws, q.offsets);
+    int32_t* rowtok = at<int32_t>(ws, q.rowtok);
+    void* Y = at<void>(ws, q.Y);
+
+    if (p->dtype == MOE_BF16) {
+        if (moe::launch_router_gemm(x, p->T, p->d_model, Wr, br, p->E, at<void>(ws, q.split),
+                                    logits, st, s, &launches) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    } else {
+        moe::launch_logits_f32((const float*)x, Wr, br, p->T, p->d_model, p->E, logits, s,
+                               &launches);
+    }
+    route_steps(p, logits, ids, w, slot, drop, counts, offsets, rowtok, ws, q, s, &launches);
+    r = ffn_steps(p, x, offsets, rowtok, W1, b1, W2, b2, Y, ws, q, s, &launches);
+    if (r != MOE_OK) return r;
+    moe::launch_combine(p->dtype, x, Y, w, ids, slot, offsets, p->T, p->d_model, p->E, p->k, out,
+                        st, s, &launches);
+    return finish(launches);
+}
+
+moe_status moe_get_device_status(const void* ws, size_t ws_bytes, void* stream, int32_t* code) {
+    if (!ws || !code || ws_bytes < sizeof(moe::DeviceStatus)) return MOE_ERR_INVALID_ARG;
+    moe::DeviceStatus h{};
+    if (cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, (cudaStream_t)stream) !=
+            cudaSuccess ||
+        cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    *code = h.code;
+    return h.code == MOE_DEV_OK ? MOE_OK : MOE_ERR_DEVICE;
+}
+
+moe_status moe_reset_device_status(void* ws, size_t ws_bytes, void* stream) {
+    if (!ws || ws_bytes < sizeof(moe::DeviceStatus)) return MOE_ERR_INVALID_ARG;
+    if (cudaMemsetAsync(ws, 0, sizeof(moe::DeviceStatus), (cudaStream_t)stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+int32_t moe_last_launch_count(void) { return g_last_launches; }
+
+const char* moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported problem shape";
+        case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case MOE_ERR_CUDA: return "CUDA runtime error";
+        case MOE_ERR_DEVICE: return "device reported an error in the status word";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,489 @@
+// route.cu -- router softmax/top-k and capacity-limited dispatch (sm_100a).
+//
+// Step 1, router ("Dynamic Token Routing AI", How it works): one warp per token computes the
+// softmax of its E logits in fp32 and keeps the k largest in registers.
+// Step 2, capacity ("Expert Networks > Worked Example: Expert Specialization", capacity
+// paragraph; "Some Tokens Do Not Get In", "Why there is a buffer" / "Past the edge"): each
+// expert keeps at most K pairs, those with the highest router weight (ties: lower token), and
+// the slot of a kept pair is its rank among the expert's kept tokens in ascending token order.
+//
+// Dispatch pipeline, all deterministic (no result depends on the order of atomics):
+//   count  : one warp per chunk of 32 tokens counts its pairs per expert  -> cnt[E][nC]
+//   scan   : one block per expert, exclusive prefix over chunks           -> base[E][nC], n[E]
+//   scatter: one warp per chunk writes its pairs into the expert's candidate list at
+//            base + (rank among equal experts inside the chunk)             -> cand[E][T]
+//            (a stable counting sort: every list is in ascending token order)
+//   select : one block per expert; if n_e > K a 4-pass radix select on the fp32 weight bits
+//            finds the K-th largest weight, then one ordered pass with block scans assigns
+//            slots, drop flags, rowtok and the counts.
+#include <cfloat>
+#include <cstdint>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// exp by Cody-Waite range reduction and a degree-7 Taylor polynomial (W. J. Cody and W. Waite,
+// "Software Manual for the Elementary Functions", 1980): x = n ln2 + r, ln2 split into a high
+// part with 16 significant bits and a low correction, exp(r) by Horner's rule with fused
+// multiply-adds, scaling by 2^n through the exponent field.  Every step is one IEEE single
+// operation rounded to nearest even, written with explicit intrinsics so that the compiler can
+// neither contract nor reorder them; the result is therefore the same on any IEEE machine that
+// evaluates the same steps.  Results below 2^-125 flush to +0 (n < -125), none is subnormal.
+__device__ __forceinline__ float exp_cody_waite(float x) {
+    if (isnan(x)) return x;
+    const float kLog2e = (float)1.4426950408889634074;
+    const float kLn2Hi = (float)(45426.0 / 65536.0);
+    const float kLn2Lo = (float)(0.6931471805599453094 - 45426.0 / 65536.0);
+    const float t = __fmul_rn(x, kLog2e);
+    if (t > 200.0f) return __int_as_float(0x7f800000);
+    if (t < -200.0f) return 0.0f;
+    const float nf = rintf(t);
+    const int n = (int)nf;
+    if (n < -125) return 0.0f;
+    float r = __fmaf_rn(-nf, kLn2Hi, x);
+    r = __fmaf_rn(-nf, kLn2Lo, r);
+    float p = (float)(1.0 / 5040.0);
+    p = __fmaf_rn(p, r, (float)(1.0 / 720.0));
+    p = __fmaf_rn(p, r, (float)(1.0 / 120.0));
+    p = __fmaf_rn(p, r, (float)(1.0 / 24.0));
+    p = __fmaf_rn(p, r, (float)(1.0 / 6.0));
+    p = __fmaf_rn(p, r, 0.5f);
+    p = __fmaf_rn(p, r, 1.0f);
+    p = __fmaf_rn(p, r, 1.0f);
+    if (n > 127) return __fmul_rn(__fmul_rn(p, __int_as_float(254 << 23)), 2.0f);
+    return __fmul_rn(p, __int_as_float((n + 127) << 23));
+}
+
+// Order-preserving map of a float (NaN excluded) to uint32; -0 and +0 map to the same key.
+__device__ __forceinline__ uint32_t float_key(float v) {
+    const uint32_t u = __float_as_uint(__fadd_rn(v, 0.0f));
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_float(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Router: softmax over E + top-k, one warp per token.  Lane l holds experts l, l+32, ...
+// Softmax sum order: lane partials left to right, then xor-butterfly 16, 8, 4, 2, 1.
+// ---------------------------------------------------------------------------------------------
+template <int EPL>
+__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T,
+                                                         int E, int k, int32_t* __restrict__ ids,
+                                                         float* __restrict__ w) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const float* L = logits + (size_t)t * E;
+    float v[EPL];
+    uint32_t key[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = e < E ? __ldg(L + e) : 0.0f;
+        key[i] = e < E ? float_key(v[i]) : 0u;
+    }
+    uint32_t lmax = 0;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) lmax = max(lmax, key[i]);
+    const float m = key_float(__reduce_max_sync(kFull, lmax));
+    float u[EPL];
+    float part = 0.0f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        u[i] = e < E ? exp_cody_waite(__fsub_rn(v[i], m)) : 0.0f;
+        if (e < E) part = __fadd_rn(part, u[i]);
+    }
+#pragma unroll
+    for (int h = 16; h >= 1; h >>= 1) part = __fadd_rn(part, __shfl_xor_sync(kFull, part, h));
+    const float S = part;
+
+    int my_id = 0;
+    float my_w = 0.0f;
+    uint32_t taken = 0;
+    for (int j = 0; j < k; ++j) {
+        uint32_t bk = 0;
+        int bi = 0;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const bool ok = !((taken >> i) & 1u) && key[i] > bk;
+            bk = ok ? key[i] : bk;
+            bi = ok ? i : bi;
+        }
+        const uint32_t wk = __reduce_max_sync(kFull, bk);
+        const unsigned cand = (bk == wk && bk != 0u) ? (unsigned)(lane + 32 * bi) : 0x7fffffffu;
+        const int we = (int)__reduce_min_sync(kFull, cand);
+        float up = 0.0f;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) up = (i == bi) ? u[i] : up;
+        const float wu = __shfl_sync(kFull, up, we & 31);
+        if (lane == (we & 31)) taken |= 1u << (we >> 5);
+        if (lane == j) {
+            my_id = we;
+            my_w = __fdiv_rn(wu, S);
+        }
+    }
+    if (lane < k) {
+        ids[(size_t)t * k + lane] = my_id;
+        w[(size_t)t * k + lane] = my_w;
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Dispatch: count pairs per (expert, 32-token chunk).
+// ---------------------------------------------------------------------------------------------
+constexpr int kChunk = 32;   // tokens per chunk
+
+__global__ void __launch_bounds__(128) count_chunks_kernel(const int32_t* __restrict__ ids, int T,
+                                                           int E, int k, int nC,
+                                                           int32_t* __restrict__ cnt,
+                                                           DeviceStatus* st) {
+    extern __shared__ int32_t s_cnt[];                 // [4][E]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int32_t* my = s_cnt + warp * E;
+    for (int e = lane; e < E; e += 32) my[e] = 0;
+    __syncwarp();
+    const int c = blockIdx.x * 4 + warp;
+    if (c >= nC) return;
+    const long long p0 = (long long)c * kChunk * k;
+    const long long p1 = (long long)min(T, (c + 1) * kChunk) * k;
+    for (long long p = p0 + lane; p < p1; p += 32) {
+        const int e = ids[p];
+        if ((unsigned)e >= (unsigned)E) { report(st, MOE_DEV_BAD_INDEX, 101); continue; }
+        atomicAdd(&my[e], 1);
+    }
+    __syncwarp();
+    for (int e = lane; e < E; e += 32) cnt[(size_t)e * nC + c] = my[e];
+}
+
+// Block-wide exclusive scan of one value per thread (blockDim.x a multiple of 32, <= 1024).
+// Returns the exclusive prefix; *total receives the block total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int s = lane < nw ? s_warp[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, s, o);
+            if (lane >= o) s += y;
+        }
+        if (lane < nw) s_warp[lane] = s;       // inclusive prefix of warp totals
+    }
+    __syncthreads();
+    const int before = warp ? s_warp[warp - 1] : 0;
+    *total = s_warp[nw - 1];
+    __syncthreads();
+    return before + x - v;
+}
+
+// One block per expert: base[e][c] = sum of cnt[e][c' < c]; n[e] = total.
+__global__ void __launch_bounds__(256) scan_chunks_kernel(const int32_t* __restrict__ cnt, int nC,
+                                                          int32_t* __restrict__ base,
+                                                          int32_t* __restrict__ nrecv) {
+    __shared__ int s_warp[32];
+    const int e = blockIdx.x;
+    const int32_t* in = cnt + (size_t)e * nC;
+    int32_t* out = base + (size_t)e * nC;
+    int carry = 0;
+    for (int c0 = 0; c0 < nC; c0 += blockDim.x) {
+        const int c = c0 + threadIdx.x;
+        const int v = c < nC ? in[c] : 0;
+        int tot;
+        const int ex = block_exclusive_scan(v, s_warp, &tot);
+        if (c < nC) out[c] = carry + ex;
+        carry += tot;
+    }
+    if (threadIdx.x == 0) nrecv[e] = carry;
+}
+
+// One warp per chunk: stable scatter of the chunk's pairs into cand[e][.] (ascending tokens).
+__global__ void __launch_bounds__(128) scatter_chunks_kernel(const int32_t* __restrict__ ids,
+                                                             int T, int E, int k, int nC,
+                                                             const int32_t* __restrict__ base,
+                                                             int32_t* __restrict__ cand) {
+    extern __shared__ int32_t s_run[];                 // [4][E]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x * 4 + warp;
+    if (c >= nC) return;
+    int32_t* run = s_run + warp * E;
+    for (int e = lane; e < E; e += 32) run[e] = base[(size_t)e * nC + c];
+    __syncwarp();
+    const long long p0 = (long long)c * kChunk * k;
+    const long long p1 = (long long)min(T, (c + 1) * kChunk) * k;
+    for (long long pb = p0; pb < p1; pb += 32) {
+        const long long p = pb + lane;
+        const bool act = p < p1;
+        const unsigned amask = __ballot_sync(kFull, act);
+        int e = act ? ids[p] : -1;
+        if ((unsigned)e >= (unsigned)E) e = -1;        // bad ids were reported by the count pass
+        const unsigned peers = __match_any_sync(kFull, e);
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        const int pos = (e >= 0) ? run[e] + rank : 0;
+        __syncwarp();
+        if (act && e >= 0) {
+            cand[(size_t)e * T + pos] = (int32_t)p;
+            if (lane == __ffs(peers) - 1) run[e] = pos + __popc(peers);
+        }
+        __syncwarp();
+        (void)amask;
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Capacity selection: one block per expert.
+// ---------------------------------------------------------------------------------------------
+constexpr int kSelThreads = 512;
+
+__global__ void __launch_bounds__(kSelThreads) select_kernel(
+    const int32_t* __restrict__ cand, const int32_t* __restrict__ nrecv,
+    const float* __restrict__ w, int T, int E, int k, long long K, int32_t* __restrict__ slot,
+    uint8_t* __restrict__ drop, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ rowtok) {
+    __shared__ int s_warp[32];
+    __shared__ int s_hist[256];
+    __shared__ uint32_t s_prefix;
+    __shared__ int s_remaining;
+    const int e = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int n = nrecv[e];
+    const int kept = (int)min((long long)n, K);
+
+    // Row offset of this expert: sum of kept counts of the experts before it.
+    int part = 0;
+    for (int q = tid; q < e; q += blockDim.x) part += (int)min((long long)nrecv[q], K);
+    int off_tot;
+    (void)block_exclusive_scan(part, s_warp, &off_tot);
+    const int off = off_tot;
+    if (tid == 0) {
+        if (counts) { counts[e] = n; counts[E + e] = kept; }
+        if (offsets) {
+            offsets[e] = off;
+            if (e == E - 1) offsets[E] = off + kept;
+        }
+    }
+    const int32_t* list = cand + (size_t)e * T;
+
+    if (n <= K) {
+        for (int i = tid; i < n; i += blockDim.x) {
+            const int p = list[i];
+            slot[p] = i;
+            drop[p] = 0;
+            if (rowtok) rowtok[off + i] = p / k;
+        }
+        return;
+    }
+
+    // Radix select (most significant byte first) of the K-th largest weight bit pattern.
+    // Weights are >= +0, so their IEEE bit patterns order like the values.
+    uint32_t prefix = 0, mask = 0;
+    int remaining = (int)K;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        for (int b = tid; b < 256; b += blockDim.x) s_hist[b] = 0;
+        __syncthreads();
+        for (int i = tid; i < n; i += blockDim.x) {
+            const uint32_t key = __float_as_uint(w[list[i]]);
+            if ((key & mask) == prefix) atomicAdd(&s_hist[(key >> shift) & 255u], 1);
+        }
+        __syncthreads();
+        if (tid < 32) {
+            // Lane l owns bins 255-8l .. 248-8l (top-down); find the bin where the running
+            // count from the top reaches `remaining`.
+            int loc = 0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) loc += s_hist[255 - 8 * tid - q];
+            int inc = loc;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(kFull, inc, o);
+                if (tid >= o) inc += y;
+            }
+            const int exc = inc - loc;
+            const unsigned hit = __ballot_sync(kFull, inc >= remaining && exc < remaining);
+            const int owner = __ffs(hit) - 1;
+            if (tid == owner) {
+                int run = exc;
+                for (int q = 0; q < 8; ++q) {
+                    const int b = 255 - 8 * tid - q;
+                    if (run + s_hist[b] >= remaining) {
+                        s_prefix = prefix | ((uint32_t)b << shift);
+                        s_remaining = remaining - run;
+                        break;
+                    }
+                    run += s_hist[b];
+                }
+            }
+        }
+        __syncthreads();
+        prefix = s_prefix;
+        remaining = s_remaining;
+        mask |= 255u << shift;
+        __syncthreads();
+    }
+    const uint32_t tau = prefix;        // K-th largest weight bits
+    const int need_eq = remaining;      // how many weights equal to tau are kept (lowest t first)
+
+    int eq_carry = 0, keep_carry = 0;
+    for (int i0 = 0; i0 < n; i0 += blockDim.x) {
+        const int i = i0 + tid;
+        int p = 0;
+        uint32_t key = 0;
+        if (i < n) { p = list[i]; key = __float_as_uint(w[p]); }
+        const int is_eq = (i < n && key == tau) ? 1 : 0;
+        int eq_tot;
+        const int eq_rank = eq_carry + block_exclusive_scan(is_eq, s_warp, &eq_tot);
+        const int keep = (i < n) && (key > tau || (is_eq && eq_rank < need_eq)) ? 1 : 0;
+        int keep_tot;
+        const int s = keep_carry + block_exclusive_scan(keep, s_warp, &keep_tot);
+        if (i < n) {
+            slot[p] = keep ? s : -1;
+            drop[p] = keep ? 0 : 1;
+            if (keep && rowtok) rowtok[off + s] = p / k;
+        }
+        eq_carry += eq_tot;
+        keep_carry += keep_tot;
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Dispatch from a given routing (moe_dispatch).
+// ---------------------------------------------------------------------------------------------
+__global__ void kept_count_kernel(const int32_t* __restrict__ ids,
+                                  const int32_t* __restrict__ slot, long long P, int E, int T,
+                                  int32_t* __restrict__ kept, DeviceStatus* st) {
+    for (long long p = blockIdx.x * (long long)blockDim.x + threadIdx.x; p < P;
+         p += (long long)gridDim.x * blockDim.x) {
+        const int s = slot[p];
+        if (s < 0) continue;
+        const int e = ids[p];
+        if ((unsigned)e >= (unsigned)E || s >= T) { report(st, MOE_DEV_BAD_INDEX, 201); continue; }
+        atomicAdd(&kept[e], 1);
+    }
+}
+
+__global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict__ kept, int E,
+                                                       int32_t* __restrict__ offsets) {
+    __shared__ int s_warp[32];
+    int carry = 0;
+    for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+        const int e = e0 + threadIdx.x;
+        const int v = e < E ? kept[e] : 0;
+        int tot;
+        const int ex = block_exclusive_scan(v, s_warp, &tot);
+        if (e < E) offsets[e] = carry + ex;
+        carry += tot;
+    }
+    if (threadIdx.x == 0) offsets[E] = carry;
+}
+
+__global__ void rowtok_scatter_kernel(const int32_t* __restrict__ ids,
+                                      const int32_t* __restrict__ slot, long long P, int E, int k,
+                                      const int32_t* __restrict__ offsets,
+                                      int32_t* __restrict__ rowtok, DeviceStatus* st) {
+    for (long long p = blockIdx.x * (long long)blockDim.x + threadIdx.x; p < P;
+         p += (long long)gridDim.x * blockDim.x) {
+        const int s = slot[p];
+        if (s < 0) continue;
+        const int e = ids[p];
+        if ((unsigned)e >= (unsigned)E) continue;
+        const int r = offsets[e] + s;
+        if (r >= offsets[e + 1]) { report(st, MOE_DEV_BAD_INDEX, 202); continue; }
+        rowtok[r] = (int32_t)(p / k);
+    }
+}
+
+// x_perm[r] = x[rowtok[r]], 16-byte vectors (row bytes a multiple of 16) or 4-byte words.
+template <typename V>
+__global__ void permute_rows_kernel(const V* __restrict__ x, const int32_t* __restrict__ rowtok,
+                                    const int32_t* __restrict__ offsets, int E, int vpr, int T,
+                                    V* __restrict__ xp, DeviceStatus* st) {
+    const int rows = offsets[E];
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < (long long)rows * vpr;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int r = (int)(i / vpr), c = (int)(i % vpr);
+        const int t = rowtok[r];
+        if ((unsigned)t >= (unsigned)T) { report(st, MOE_DEV_BAD_INDEX, 203); continue; }
+        xp[i] = x[(size_t)t * vpr + c];
+    }
+}
+
+template <int EPL>
+void launch_route_t(const float* logits, int T, int E, int k, int32_t* ids, float* w,
+                    cudaStream_t s) {
+    const int blocks = (T + 7) / 8;
+    route_topk_kernel<EPL><<<blocks, 256, 0, s>>>(logits, T, E, k, ids, w);
+}
+
+}  // namespace
+
+void launch_route_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
+                       cudaStream_t s) {
+    const int epl = (E + 31) / 32;
+    if (epl <= 1) launch_route_t<1>(logits, T, E, k, ids, w, s);
+    else if (epl <= 2) launch_route_t<2>(logits, T, E, k, ids, w, s);
+    else if (epl <= 4) launch_route_t<4>(logits, T, E, k, ids, w, s);
+    else if (epl <= 8) launch_route_t<8>(logits, T, E, k, ids, w, s);
+    else if (epl <= 16) launch_route_t<16>(logits, T, E, k, ids, w, s);
+    else launch_route_t<32>(logits, T, E, k, ids, w, s);
+}
+
+int chunk_count(int T) { return (T + kChunk - 1) / kChunk; }
+
+void launch_capacity_select(const int32_t* ids, const float* w, int T, int E, int k, long long K,
+                            int32_t* cnt, int32_t* base, int32_t* nrecv, int32_t* cand,
+                            int32_t* slot, uint8_t* drop, int32_t* counts, int32_t* offsets,
+                            int32_t* rowtok, DeviceStatus* st, cudaStream_t s, int* launches) {
+    const int nC = chunk_count(T);
+    const int blocks = (nC + 3) / 4;
+    const size_t smem = (size_t)4 * E * sizeof(int32_t);
+    count_chunks_kernel<<<blocks, 128, smem, s>>>(ids, T, E, k, nC, cnt, st);
+    scan_chunks_kernel<<<E, 256, 0, s>>>(cnt, nC, base, nrecv);
+    scatter_chunks_kernel<<<blocks, 128, smem, s>>>(ids, T, E, k, nC, base, cand);
+    select_kernel<<<E, kSelThreads, 0, s>>>(cand, nrecv, w, T, E, k, K, slot, drop, counts,
+                                            offsets, rowtok);
+    *launches += 4;
+}
+
+void launch_dispatch(const int32_t* ids, const int32_t* slot, int T, int E, int k,
+                     int32_t* kept_tmp, int32_t* offsets, int32_t* rowtok, DeviceStatus* st,
+                     cudaStream_t s, int* launches) {
+    const long long P = (long long)T * k;
+    const int blocks = (int)std::min<long long>((P + 255) / 256, 148 * 8);
+    cudaMemsetAsync(kept_tmp, 0, sizeof(int32_t) * E, s);
+    if (P > 0) kept_count_kernel<<<blocks, 256, 0, s>>>(ids, slot, P, E, T, kept_tmp, st);
+    offsets_kernel<<<1, 1024, 0, s>>>(kept_tmp, E, offsets);
+    if (P > 0)
+        rowtok_scatter_kernel<<<blocks, 256, 0, s>>>(ids, slot, P, E, k, offsets, rowtok, st);
+    *launches += (P > 0) ? 3 : 1;
+}
+
+void launch_permute_rows(const void* x, const int32_t* rowtok, const int32_t* offsets, int E,
+                         size_t row_bytes, int T, long long max_rows, void* xp, DeviceStatus* st,
+                         cudaStream_t s, int* launches) {
+    const int blocks = 148 * 8;
+    if (row_bytes % 16 == 0 && ((uintptr_t)x % 16 == 0) && ((uintptr_t)xp % 16 == 0)) {
+        permute_rows_kernel<uint4><<<blocks, 256, 0, s>>>(
+            (const uint4*)x, rowtok, offsets, E, (int)(row_bytes / 16), T, (uint4*)xp, st);
+    } else {
+        permute_rows_kernel<uint32_t><<<blocks, 256, 0, s>>>(
+            (const uint32_t*)x, rowtok, offsets, E, (int)(row_bytes / 4), T, (uint32_t*)xp, st);
+    }
+    (void)max_rows;
+    *launches += 1;
+}
+
+}  // namespace moe

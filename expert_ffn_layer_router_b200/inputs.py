@@ -106,8 +106,11 @@ def _topk_gap_ok(L64: np.ndarray, k: int) -> np.ndarray:
     return (part[:, k - 1] - part[:, k]) >= GAP
 
 
-def make_layer(spec: LayerSpec, seed: int = 0, T: int | None = None) -> dict:
-    """Draw one layer's inputs. ``T`` overrides the token count (x and the gap screen only)."""
+def make_layer(spec: LayerSpec, seed: int = 0, T: int | None = None,
+               weights: bool = True) -> dict:
+    """Draw one layer's inputs. ``T`` overrides the token count (x and the gap screen only).
+
+    ``weights=False`` skips W1/b1/W2/b2 (drawn after x, Wr and br, so those are unchanged)."""
     T = spec.T if T is None else T
     d, F, E, k = spec.d_model, spec.d_ff, spec.E, spec.k
     rng = np.random.default_rng(seed)
@@ -124,12 +127,17 @@ def make_layer(spec: LayerSpec, seed: int = 0, T: int | None = None) -> dict:
     elif spec.router == "normal":
         br = (rng.standard_normal(E, dtype=np.float32) * np.float32(spec.router_bias)
               ).astype(np.float32)
-    W1 = rng.standard_normal((E, F, d), dtype=np.float32) * np.float32(1.0 / math.sqrt(d))
-    b1 = (rng.standard_normal((E, F), dtype=np.float32) * np.float32(spec.bias_std)
-          if spec.bias_std > 0 else np.zeros((E, F), np.float32))
-    W2 = rng.standard_normal((E, d, F), dtype=np.float32) * np.float32(1.0 / math.sqrt(F))
-    b2 = (rng.standard_normal((E, d), dtype=np.float32) * np.float32(spec.bias_std)
-          if spec.bias_std > 0 else np.zeros((E, d), np.float32))
+    if weights:
+        W1 = rng.standard_normal((E, F, d), dtype=np.float32)
+        W1 *= np.float32(1.0 / math.sqrt(d))
+        b1 = (rng.standard_normal((E, F), dtype=np.float32) * np.float32(spec.bias_std)
+              if spec.bias_std > 0 else np.zeros((E, F), np.float32))
+        W2 = rng.standard_normal((E, d, F), dtype=np.float32)
+        W2 *= np.float32(1.0 / math.sqrt(F))
+        b2 = (rng.standard_normal((E, d), dtype=np.float32) * np.float32(spec.bias_std)
+              if spec.bias_std > 0 else np.zeros((E, d), np.float32))
+    else:
+        W1 = b1 = W2 = b2 = None
 
     x = _to_dtype(x32, spec.dtype)
     logits = None
@@ -154,8 +162,9 @@ def make_layer(spec: LayerSpec, seed: int = 0, T: int | None = None) -> dict:
                     break
             else:
                 raise RuntimeError("gap screen failed to redraw token %d" % t)
-    return dict(spec=spec, seed=seed, T=T, x=x, Wr=Wr, br=br, W1=_to_dtype(W1, spec.dtype),
-                b1=b1.astype(np.float32), W2=_to_dtype(W2, spec.dtype), b2=b2.astype(np.float32),
+    if weights:
+        W1, W2 = _to_dtype(W1, spec.dtype), _to_dtype(W2, spec.dtype)
+    return dict(spec=spec, seed=seed, T=T, x=x, Wr=Wr, br=br, W1=W1, b1=b1, W2=W2, b2=b2,
                 logits=logits, redrawn=redrawn)
 
 

@@ -1,0 +1,153 @@
+/*
+ * moe_b200.h -- C ABI of the B200 (sm_100a) forward pass of one capacity-limited
+ * Mixture-of-Experts layer.
+ *
+ * The layer (sources are the pages' titles and sections):
+ *   1. router: softmax over the E router logits of each token, keep the k largest
+ *      ("Dynamic Token Routing AI", How it works: a gating network scores each token and
+ *      picks experts);
+ *   2. capacity: every expert has K = floor(C * T * k / E) slots (at most T); an expert that
+ *      receives more than K (token, expert) pairs keeps the K with the highest router weight
+ *      and drops the rest ("Expert Networks > Worked Example: Expert Specialization", capacity
+ *      paragraph: K = 1.25 * (8/4) rounded down to 2, the lowest-confidence token is dropped;
+ *      "Some Tokens Do Not Get In", "Why there is a buffer": t*k slots, fixed buffer per
+ *      expert);
+ *   3. expert FFN on the kept pairs: h = W1 x + b1, a = SiLU(h), y = W2 a + b2 (worked
+ *      example, trace of token 0);
+ *   4. combine: out = x + sum_j w_j * y_j over the token's kept pairs; a token whose pairs
+ *      were all dropped leaves the layer exactly as it entered (worked example, token 4;
+ *      "Some Tokens Do Not Get In", "Past the edge"; the k outputs of a token are summed back
+ *      in token order as in the fused-MoE dataflow diagram's moe_sum step).
+ *
+ * Conventions for every call:
+ *   - All pointers except `p` and the out-parameters of the host-only queries are DEVICE
+ *     pointers owned by the caller.  The library never allocates device memory: scratch comes
+ *     from the caller's workspace `ws` of `ws_bytes` bytes (size from moe_workspace_size,
+ *     256-byte aligned).
+ *   - Every compute call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and performs no host synchronisation.
+ *   - Host-checkable errors (bad shapes, k > E, negative or NaN capacity factor, null or
+ *     misaligned pointers, workspace too small, unsupported shape) return a non-zero status
+ *     BEFORE anything is launched; outputs are then untouched.
+ *   - Errors the device detects (a pipeline wait that ran out, an index out of range) are
+ *     recorded in a status word at the start of `ws`; read it with moe_get_device_status.
+ *   - Layouts are row-major and dense.  Pair p = t * k + j addresses the j-th expert of token
+ *     t (j = 0 is the largest logit).  W1 is [E, d_ff, d_model] and W2 is [E, d_model, d_ff]
+ *     ("out x in", so h = W1 x).  b1 is [E, d_ff] and b2 is [E, d_model], float32 always.
+ *   - dtype MOE_BF16: x, W1, W2, out and expert outputs are bfloat16, accumulation is float32
+ *     on the tensor cores; d_model and d_ff must be multiples of 64 and bf16 pointers 16-byte
+ *     aligned.  dtype MOE_F32: everything float32 on CUDA cores (small layers).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,  /* bad shape, pointer, alignment or capacity factor */
+    MOE_ERR_UNSUPPORTED = 2,  /* well-formed problem this build does not run */
+    MOE_ERR_WORKSPACE = 3,    /* workspace null or smaller than moe_workspace_size */
+    MOE_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+    MOE_ERR_DEVICE = 5        /* the device status word holds an error */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Device status codes (moe_get_device_status). */
+#define MOE_DEV_OK 0
+#define MOE_DEV_TIMEOUT 1      /* a pipeline wait in a kernel gave up after about 2 s */
+#define MOE_DEV_BAD_INDEX 2    /* an index read from an input was out of range */
+
+typedef struct {
+    int32_t T;                /* tokens, >= 0 */
+    int32_t d_model;          /* model width, >= 1 */
+    int32_t d_ff;             /* expert hidden width, >= 1 */
+    int32_t E;                /* experts, 1..1024 */
+    int32_t k;                /* experts per token, 1..min(E, 32) */
+    float capacity_factor;    /* C >= 0; +INFINITY = dropless (K = T) */
+    int32_t dtype;            /* moe_dtype */
+    uint32_t flags;           /* reserved, must be 0 */
+} moe_problem;
+
+/* Host only.  Per-expert capacity K = min(T, floor(C * T * k / E)) evaluated in double
+ * (worked example, capacity paragraph; generalised to k slots per token as in "Some Tokens Do
+ * Not Get In").  Returns MOE_ERR_INVALID_ARG for a malformed problem. */
+moe_status moe_capacity(const moe_problem* p, int64_t* K);
+
+/* Host only.  Workspace bytes needed by any call below for problem p (the largest, moe_forward,
+ * decides).  A workspace of this size serves every call for that problem. */
+moe_status moe_workspace_size(const moe_problem* p, size_t* bytes);
+
+/* Router + capacity (steps 1-2).
+ *   logits [T, E] float32 in;  ids [T*k] int32, w [T*k] float32 (softmax weight, not
+ *   renormalised), slot [T*k] int32 (rank of t among the expert's kept tokens in ascending
+ *   token order, -1 if dropped), drop [T*k] uint8 (1 = dropped), counts [2E] int32 (pairs
+ *   received per expert, then pairs kept per expert).
+ * Drop priority inside one expert: weight descending, then token index ascending.  Top-k ties
+ * in the logits go to the lower expert index.  The softmax uses a fixed summation order and
+ * its own exp, so ids, w, slot and drop are bit-for-bit functions of the logits.  NaN logits
+ * are a precondition violation (result unspecified). */
+moe_status moe_route(const moe_problem* p, const float* logits, int32_t* ids, float* w,
+                     int32_t* slot, uint8_t* drop, int32_t* counts, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/* Dispatch layout from a routing.
+ *   ids, slot [T*k] in;  offsets [E+1] int32 out (exclusive prefix of kept counts);
+ *   rowtok [min(T*k, E*K)] int32 out: rowtok[offsets[e] + slot] = token of that kept pair.
+ *   x_perm (nullable) [rows, d_model] in x's dtype: when given, receives x[rowtok[r]] in row
+ *   r (the permuted token buffer; the FFN does not need it, it gathers rows itself). */
+moe_status moe_dispatch(const moe_problem* p, const int32_t* ids, const int32_t* slot,
+                        int32_t* offsets, int32_t* rowtok, const void* x, void* x_perm,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* Expert FFN over the kept rows (step 3): for each expert e and row r in
+ * [offsets[e], offsets[e+1]): Y[r] = W2[e] SiLU(W1[e] x[rowtok[r]] + b1[e]) + b2[e].
+ * The token gather is folded into the first GEMM's operand load; nothing is materialised but
+ * the hidden activations (in ws, x's dtype).  Y is [min(T*k, E*K), d_model] in x's dtype.
+ * b1, b2 may be NULL (zero bias). */
+moe_status moe_expert_ffn(const moe_problem* p, const void* x, const int32_t* offsets,
+                          const int32_t* rowtok, const void* W1, const float* b1,
+                          const void* W2, const float* b2, void* Y, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/* Combine (step 4): out[t] = x[t] + sum over kept j (ascending) of w[t*k+j] * Y[offsets[id]
+ * + slot], accumulated in float32 and rounded once; out[t] = x[t] bit for bit when no pair of
+ * t is kept.  out must not alias x or Y. */
+moe_status moe_combine(const moe_problem* p, const void* x, const void* Y, const float* w,
+                       const int32_t* ids, const int32_t* slot, const int32_t* offsets,
+                       void* out, void* stream);
+
+/* The whole layer: logits = x Wr + br (Wr [d_model, E] float32, br [E] float32 or NULL), then
+ * the four steps.  out [T, d_model] in x's dtype.  Optional outputs (NULL = keep in ws):
+ * logits_out [T, E], ids_out, w_out, slot_out [T*k], drop_out [T*k], counts_out [2E].
+ * With dtype MOE_BF16 the logits come from the tensor cores with Wr split exactly into three
+ * bfloat16 terms and float32 accumulation. */
+moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, const float* br,
+                       const void* W1, const float* b1, const void* W2, const float* b2,
+                       void* out, float* logits_out, int32_t* ids_out, float* w_out,
+                       int32_t* slot_out, uint8_t* drop_out, int32_t* counts_out, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/* Reads the device status word of `ws` (synchronises `stream`). */
+moe_status moe_get_device_status(const void* ws, size_t ws_bytes, void* stream, int32_t* code);
+
+/* Clears the device status word of `ws` (asynchronous on `stream`). */
+moe_status moe_reset_device_status(void* ws, size_t ws_bytes, void* stream);
+
+/* Kernel launches made by the most recent successful compute call on this host thread. */
+int32_t moe_last_launch_count(void);
+
+/* Static, never NULL. */
+const char* moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -47,6 +47,10 @@ def lib():
         L.oracle_combine_tokens.restype = ctypes.c_int
         L.oracle_combine_tokens.argtypes = [ctypes.c_int] * 6 + [_vp] * 5 + [
             _i32p, _f32p, _i32p, ctypes.c_int, _i32p, _f64p, _vp, ctypes.c_int]
+        L.oracle_combine_given_y.restype = ctypes.c_int
+        L.oracle_combine_given_y.argtypes = [ctypes.c_int] * 5 + [_vp, _vp, ctypes.c_longlong,
+                                                                  _f32p, _i32p, _i32p, _i32p,
+                                                                  _f64p, _vp]
         L.oracle_bf16_from_double.restype = ctypes.c_uint16
         L.oracle_bf16_from_double.argtypes = [ctypes.c_double]
         _lib = L
@@ -177,6 +181,25 @@ def forward(x, Wr, br, W1, b1, W2, b2, k, C, tokens=None, logits_=None, nthreads
     r = route(L, k, K)
     out64, outx = combine_tokens(x, W1, b1, W2, b2, r, tokens, nthreads)
     return dict(logits=L, K=K, route=r, out_f64=out64, out=outx)
+
+
+def combine_given_y(x, Y, route_, offsets):
+    """Combine alone from given expert outputs ``Y`` (rows in expert-sorted order)."""
+    x = np.ascontiguousarray(x)
+    Y = np.ascontiguousarray(Y, dtype=x.dtype)
+    T, d = x.shape
+    ids, w, slot = (_c(route_["ids"], np.int32), _c(route_["w"], np.float32),
+                    _c(route_["slot"], np.int32))
+    k = ids.shape[1]
+    offsets = _c(offsets, np.int32)
+    E = offsets.size - 1
+    out64 = np.empty((T, d), np.float64)
+    outx = np.empty((T, d), x.dtype)
+    rc = lib().oracle_combine_given_y(T, d, E, k, _dtype_code(x), _ptr(x), _ptr(Y), Y.shape[0],
+                                      w, ids, slot, offsets, out64, _ptr(outx))
+    if rc != 0:
+        raise ValueError("oracle_combine_given_y rejected its arguments")
+    return out64, outx
 
 
 def bf16_from_double(v):

@@ -335,6 +335,37 @@ int oracle_combine_tokens(int T, int d, int F, int E, int k, int dtype, const vo
     return 0;
 }
 
+// Combine alone, given the expert outputs: out[t] = x[t] + sum over kept j (ascending) of
+// w[t*k+j] * Y[offsets[id] + slot] in double, rounded once to x's dtype; a token with no kept
+// pair is copied bit for bit.  Y is [rows, d] in x's dtype.
+int oracle_combine_given_y(int T, int d, int E, int k, int dtype, const void* x, const void* Y,
+                           long long rows, const float* w, const int32_t* ids,
+                           const int32_t* slot, const int32_t* offsets, double* out_f64,
+                           void* out_x) {
+    for (int t = 0; t < T; ++t) {
+        std::vector<double> s(d, 0.0);
+        bool any = false;
+        for (int j = 0; j < k; ++j) {
+            size_t pi = (size_t)t * k + j;
+            if (slot[pi] < 0) continue;
+            int e = ids[pi];
+            if (e < 0 || e >= E) return -1;
+            long long r = (long long)offsets[e] + slot[pi];
+            if (r < 0 || r >= rows || r >= offsets[e + 1]) return -1;
+            for (int c = 0; c < d; ++c) s[c] += (double)w[pi] * load_elem(Y, (size_t)r * d + c, dtype);
+            any = true;
+        }
+        for (int c = 0; c < d; ++c) {
+            size_t xi = (size_t)t * d + c;
+            double v = load_elem(x, xi, dtype) + s[c];
+            if (out_f64) out_f64[xi] = v;
+            if (dtype == 0) ((float*)out_x)[xi] = any ? (float)v : ((const float*)x)[xi];
+            else ((uint16_t*)out_x)[xi] = any ? bf16_from_double(v) : ((const uint16_t*)x)[xi];
+        }
+    }
+    return 0;
+}
+
 uint16_t oracle_bf16_from_double(double v) { return bf16_from_double(v); }
 
 }  // extern "C"
