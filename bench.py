@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Benchmark of the capacity-limited MoE layer forward on B200.
+
+One step = one ``moe_forward`` call (router logits, softmax/top-k, capacity selection and
+dispatch, expert GEMM1 + SiLU, expert GEMM2, combine) over one batch of synthetic tokens whose
+inputs are already in HBM.  Default workload: the skewed E=64 top-6 layer (T=16384,
+d_model=2048, d_ff=1408, capacity factor 1.0).  Under torchrun each rank runs its own batch
+(independent problems, no data-path collective): weak scaling, time = max over ranks.
+
+``--impl reference`` times the CPU oracle on the host cores instead (a bounded sample of the
+same workload per step, extrapolated to the whole batch).
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from expert_ffn_layer_router_b200 import inputs  # noqa: E402
+
+METRIC = "MoE-layer tokens/s; expert grouped-GEMM TFLOP/s as % of B200 bf16 dense peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--config", default="skewed_e64_top6", choices=inputs.CONFIG_ORDER)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(spec):
+    C = "dropless" if math.isinf(spec.C) else "C=%g" % spec.C
+    return "%s: T=%d, d_model=%d, d_ff=%d, E=%d, top-%d, %s, %s" % (
+        spec.name, spec.T, spec.d_model, spec.d_ff, spec.E, spec.k, C, spec.dtype)
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle timing (the reference arm and the cpu_baseline object)
+# ------------------------------------------------------------------------------------------------
+def oracle_step(L, spec, sample, nthreads):
+    """Time the oracle on one bounded sample; returns (seconds extrapolated to T tokens, info)."""
+    import oracle
+    T = spec.T
+    rng = np.random.default_rng(sample)
+    toks = np.sort(rng.choice(T, size=sample, replace=False)).astype(np.int32)
+    t0 = time.perf_counter()
+    Ls = oracle.logits(L["x"][toks], L["Wr"], L["br"], nthreads) if L["logits"] is None else \
+        L["logits"][toks]
+    t_logits = time.perf_counter() - t0
+    # Routing needs the whole batch (capacity competition is per batch): logits of the batch
+    # are formed once outside the timing, and the route itself is timed on all T tokens.
+    full = L["_full_logits"]
+    t0 = time.perf_counter()
+    K = oracle.capacity(T, spec.E, spec.k, spec.C)
+    r = oracle.route(full, spec.k, K)
+    t_route = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.combine_tokens(L["x"], L["W1"], L["b1"], L["W2"], L["b2"], r, toks, nthreads)
+    t_ffn = time.perf_counter() - t0
+    del Ls
+    est = (t_logits + t_ffn) * T / sample + t_route
+    return est, dict(t_logits=t_logits, t_route=t_route, t_ffn=t_ffn,
+                     measured=t_logits + t_route + t_ffn)
+
+
+def prepare_oracle_inputs(L, spec, nthreads):
+    import oracle
+    if L["logits"] is not None:
+        L["_full_logits"] = L["logits"]
+    else:
+        L["_full_logits"] = oracle.logits(L["x"], L["Wr"], L["br"], nthreads)
+
+
+def calibrate_sample(L, spec, target_s, nthreads):
+    """Tokens per sample so that one oracle step takes about target_s seconds."""
+    s = max(1, min(spec.T, 8))
+    est, info = oracle_step(L, spec, s, nthreads)
+    per_tok = max((info["t_logits"] + info["t_ffn"]) / s, 1e-6)
+    budget = max(target_s - info["t_route"], 0.05)
+    return int(max(1, min(spec.T, budget / per_tok)))
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    spec = inputs.CONFIGS[args.config]
+    L = inputs.make_layer(spec, seed=args.seed)
+    cores = cpu_cores()
+    prepare_oracle_inputs(L, spec, cores)
+    step_budget = max(0.2, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    sample = calibrate_sample(L, spec, step_budget, cores)
+    for _ in range(args.warmup):
+        oracle_step(L, spec, sample, cores)
+    ests, meas = [], []
+    for _ in range(args.steps):
+        est, info = oracle_step(L, spec, sample, cores)
+        ests.append(est)
+        meas.append(info["measured"])
+    t = statistics.mean(ests)
+    value = spec.T / t
+    desc = ("oracle on %d of %d tokens per step (logits + expert FFN + combine, scaled by T/%d)"
+            " plus routing of all %d tokens" % (sample, spec.T, sample, spec.T))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(spec), "seed": args.seed},
+            "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": desc, "value": value,
+                             "unit": "tokens/s"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "measured_seconds_per_step": statistics.mean(meas)}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.f = tempfile.TemporaryFile(mode="w+")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.seek(0)
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.f.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------------------------------------------
+# The CUDA arm
+# ------------------------------------------------------------------------------------------------
+def to_dev(a, torch, dev):
+    if a is None:
+        return None
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+
+def traffic_record(kernel):
+    """dram bytes per launch from the committed ncu summary, if taken on the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    src = os.path.join(ROOT, "expert_ffn_layer_router_b200", "csrc", "gemm_tc.cu")
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    r = rec.get(kernel)
+    if not r or r.get("source_sha256_16") != h:
+        return None
+    return r.get("bytes_per_launch")
+
+
+def run_cuda(args):
+    import torch
+    import torch.distributed as dist
+
+    from expert_ffn_layer_router_b200 import moe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d" % (args.gpus, world))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    spec = inputs.CONFIGS[args.config]
+    L = inputs.make_layer(spec, seed=args.seed + rank)
+    layer = moe.MoELayer(spec.T, spec.d_model, spec.d_ff, spec.E, spec.k, spec.C, spec.dtype,
+                         device=dev)
+    names = ("x", "Wr", "br", "W1", "b1", "W2", "b2")
+    d = {n: to_dev(L[n], torch, dev) for n in names}
+    out = torch.empty_like(d["x"])
+    counts = torch.empty(2 * spec.E, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        moe.moe_forward(layer.p, d["x"], d["Wr"], d["br"], d["W1"], d["b1"], d["W2"], d["b2"],
+                        out, layer.ws, counts_out=counts)
+
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    # The clock sampler runs from the warm-up through the timed steps (same load); warm-up lasts
+    # at least W steps and at least half a second so the sampler sees the part under load.
+    sampler.start()
+    t_end = time.perf_counter() + 0.5
+    n_warm = 0
+    while n_warm < max(args.warmup, 3) or time.perf_counter() < t_end:
+        flush.zero_()
+        step()
+        n_warm += 1
+        if n_warm % 8 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    launches_per_step = moe.moe_last_launch_count()
+    kept = int(counts[spec.E:].sum().item())
+    received = int(counts[:spec.E].sum().item())
+
+    # Timed region: K steps, L2 flushed before each (outside the step's events).
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.STAGE_EVENTS)]
+           for _ in range(K)]
+    for row in evs:                       # torch creates the CUDA event at its first record
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        moe.moe_set_stage_events(evs[i])
+        step()
+    moe.moe_set_stage_events(None)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    stage_ms = np.zeros((K, moe.STAGE_EVENTS - 1))
+    for i in range(K):
+        for s in range(moe.STAGE_EVENTS - 1):
+            stage_ms[i, s] = evs[i][s].elapsed_time(evs[i][s + 1])
+    step_ms = np.array([evs[i][0].elapsed_time(evs[i][-1]) for i in range(K)])
+    total_ms = float(step_ms.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    value = world * spec.T / (ms_per_step / 1e3)
+
+    # End to end through the C ABI with host buffers: pinned x -> device, forward, out -> host.
+    x_host = d["x"].cpu().pin_memory()
+    out_host = torch.empty_like(x_host).pin_memory()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    xd = torch.empty_like(d["x"])
+    e2e_ms = 0.0
+    for i in range(K):
+        flush.zero_()
+        e0.record(stream)
+        xd.copy_(x_host, non_blocking=True)
+        moe.moe_forward(layer.p, xd, d["Wr"], d["br"], d["W1"], d["b1"], d["W2"], d["b2"], out,
+                        layer.ws)
+        out_host.copy_(out, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms += e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * spec.T / (e2e_ms / K / 1e3)
+    assert moe.moe_get_device_status(layer.ws) == 0, "device status word reports an error"
+
+    # Roofline bookkeeping (algorithmic work per launch).
+    pk, pk_kind = peaks()
+    esz = 2 if spec.dtype == "bf16" else 4
+    T, dm, F, E, k = spec.T, spec.d_model, spec.d_ff, spec.E, spec.k
+    st_avg = stage_ms.mean(axis=0)
+    names6 = moe.STAGE_NAMES
+    gemm_flop_each = 2.0 * kept * dm * F
+    by = {
+        "router_logits": dict(flop=2.0 * T * dm * E * 3, bytes=T * dm * esz + dm * E * 4 + T * E * 4),
+        "route_topk": dict(bytes=T * E * 4 + T * k * 8),
+        "capacity_dispatch": dict(bytes=T * k * 8 + T * k * 5 + kept * 4 + E * 16),
+        "expert_gemm1": dict(flop=gemm_flop_each,
+                             bytes=kept * dm * esz + E * F * dm * esz + kept * F * esz),
+        "expert_gemm2": dict(flop=gemm_flop_each,
+                             bytes=kept * F * esz + E * dm * F * esz + kept * dm * esz),
+        "combine": dict(bytes=2 * T * dm * esz + kept * dm * esz + T * k * 12 + (E + 1) * 4),
+    }
+    kernels = {}
+    for i, n in enumerate(names6):
+        ms = float(st_avg[i])
+        rec = {"ms": ms}
+        if "flop" in by[n]:
+            rec["tflops"] = by[n]["flop"] / (ms * 1e-3) / 1e12 if ms > 0 else None
+        rec["gbs"] = by[n]["bytes"] / (ms * 1e-3) / 1e9 if ms > 0 else None
+        kernels[n] = rec
+    tensor_peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    g1, g2 = kernels["expert_gemm1"], kernels["expert_gemm2"]
+    dom = "expert_gemm1" if g1["ms"] >= g2["ms"] else "expert_gemm2"
+    achieved = kernels[dom]["tflops"]
+    gemm_ms = g1["ms"] + g2["ms"]
+    gemm_tflops = 2 * gemm_flop_each / (gemm_ms * 1e-3) / 1e12
+    rdc_bytes = sum(by[n]["bytes"] for n in ("route_topk", "capacity_dispatch", "combine"))
+    rdc_ms = sum(kernels[n]["ms"] for n in ("route_topk", "capacity_dispatch", "combine"))
+    rdc_gbs = rdc_bytes / (rdc_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if spec.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded numpy draws; random-init weights of the stated shape)",
+        "config": {"workload": workload_desc(spec), "seed": args.seed + rank,
+                   "per_rank_tokens": T, "parallelism": "dp%d (independent batches)" % world,
+                   "l2": "flushed before every timed step (256 MiB write, outside the step's"
+                         " events); per-step inputs 805 MB also exceed the 126 MB L2",
+                   "kept_pairs": kept, "received_pairs": received,
+                   "dropped_pairs": received - kept},
+        "gpu_launches": launches_per_step * K,
+        "warmup_steps_run": n_warm,
+        "gpu_launches_per_step": launches_per_step,
+        "clocks": clocks,
+        "e2e": {"value": e2e_value, "unit": "tokens/s",
+                "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
+                "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size()),
+                "ms_per_step": e2e_ms / K},
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved,
+                     "peak": tensor_peak, "unit": "TFLOP/s",
+                     "frac": achieved / tensor_peak if achieved else None,
+                     "peak_source": "%s bf16_tflops_sustained (kernel timed inside a long"
+                                    " loop of steps)" % pk_kind,
+                     "traffic": traffic_record(dom)},
+        "expert_gemm": {"tflops": gemm_tflops, "frac_of_peak": gemm_tflops / tensor_peak,
+                        "frac_of_burst_peak": gemm_tflops / pk.get("bf16_tflops", tensor_peak),
+                        "flop_per_step": 2 * gemm_flop_each},
+        "route_dispatch_combine": {"gbs": rdc_gbs, "frac_of_hbm": rdc_gbs / pk["hbm_gbs"],
+                                   "bytes_per_step": rdc_bytes, "hbm_peak_gbs": pk["hbm_gbs"]},
+        "kernels": kernels,
+        "step_ms_min": float(step_ms.min()), "step_ms_median": float(np.median(step_ms)),
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        cores = cpu_cores()
+        prepare_oracle_inputs(L, spec, cores)
+        sample = calibrate_sample(L, spec, max(1.0, args.cpu_seconds / 3), cores)
+        ests = [oracle_step(L, spec, sample, cores)[0] for _ in range(3)]
+        cv = spec.T / statistics.mean(ests)
+        line["cpu_baseline"] = {
+            "value": cv, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": "3 runs of the oracle on %d of %d tokens (logits + expert FFN + combine, "
+                      "scaled by T/%d) plus routing of all %d tokens" % (sample, T, sample, T)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_cuda(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -13,6 +13,12 @@
 namespace {
 
 thread_local int32_t g_last_launches = 0;
+thread_local cudaEvent_t g_stage_events[MOE_STAGE_EVENTS];
+thread_local bool g_stage_on = false;
+
+void stage_mark(int i, cudaStream_t s) {
+    if (g_stage_on) cudaEventRecord(g_stage_events[i], s);
+}
 
 constexpr size_t kAlign = 256;
 
@@ -107,9 +113,11 @@ moe_status finish(int launches) {
     return MOE_OK;
 }
 
-moe_status pre(const moe_problem* p) {
+// Common entry check.  `needs_ffn`: the call runs the expert GEMMs, whose tensor-core tiles need
+// d_model and d_ff to be multiples of 64 in bf16; routing, dispatch and combine take any width.
+moe_status pre(const moe_problem* p, bool needs_ffn) {
     if (bad_problem(p)) return MOE_ERR_INVALID_ARG;
-    if (unsupported(p)) return MOE_ERR_UNSUPPORTED;
+    if (needs_ffn && unsupported(p)) return MOE_ERR_UNSUPPORTED;
     cudaGetLastError();   // a stale error from unrelated work must not be blamed on this call
     return MOE_OK;
 }
@@ -171,7 +179,7 @@ moe_status moe_workspace_size(const moe_problem* p, size_t* bytes) {
 moe_status moe_route(const moe_problem* p, const float* logits, int32_t* ids, float* w,
                      int32_t* slot, uint8_t* drop, int32_t* counts, void* ws, size_t ws_bytes,
                      void* stream) {
-    moe_status r = pre(p);
+    moe_status r = pre(p, false);
     if (r != MOE_OK) return r;
     if (!counts || (p->T > 0 && (!logits || !ids || !w || !slot || !drop)))
         return MOE_ERR_INVALID_ARG;
@@ -190,7 +198,7 @@ moe_status moe_route(const moe_problem* p, const float* logits, int32_t* ids, fl
 moe_status moe_dispatch(const moe_problem* p, const int32_t* ids, const int32_t* slot,
                         int32_t* offsets, int32_t* rowtok, const void* x, void* x_perm,
                         void* ws, size_t ws_bytes, void* stream) {
-    moe_status r = pre(p);
+    moe_status r = pre(p, false);
     if (r != MOE_OK) return r;
     if (!offsets || (p->T > 0 && (!ids || !slot || !rowtok))) return MOE_ERR_INVALID_ARG;
     if (x_perm && !x) return MOE_ERR_INVALID_ARG;
@@ -211,7 +219,7 @@ moe_status moe_expert_ffn(const moe_problem* p, const void* x, const int32_t* of
                           const int32_t* rowtok, const void* W1, const float* b1,
                           const void* W2, const float* b2, void* Y, void* ws, size_t ws_bytes,
                           void* stream) {
-    moe_status r = pre(p);
+    moe_status r = pre(p, true);
     if (r != MOE_OK) return r;
     if (!offsets || !W1 || !W2 || (p->T > 0 && (!x || !rowtok || !Y))) return MOE_ERR_INVALID_ARG;
     if (p->dtype == MOE_BF16 &&
@@ -230,7 +238,7 @@ moe_status moe_expert_ffn(const moe_problem* p, const void* x, const int32_t* of
 moe_status moe_combine(const moe_problem* p, const void* x, const void* Y, const float* w,
                        const int32_t* ids, const int32_t* slot, const int32_t* offsets,
                        void* out, void* stream) {
-    moe_status r = pre(p);
+    moe_status r = pre(p, false);
     if (r != MOE_OK) return r;
     if (p->T > 0 && (!x || !Y || !w || !ids || !slot || !offsets || !out))
         return MOE_ERR_INVALID_ARG;
@@ -246,7 +254,7 @@ moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, con
                        void* out, float* logits_out, int32_t* ids_out, float* w_out,
                        int32_t* slot_out, uint8_t* drop_out, int32_t* counts_out, void* ws,
                        size_t ws_bytes, void* stream) {
-    moe_status r = pre(p);
+    moe_status r = pre(p, true);
     if (r != MOE_OK) return r;
     if (!Wr || !W1 || !W2 || (p->T > 0 && (!x || !out))) return MOE_ERR_INVALID_ARG;
     if (out && out == x) return MOE_ERR_INVALID_ARG;
@@ -272,6 +280,7 @@ moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, con
     int32_t* rowtok = at<int32_t>(ws, q.rowtok);
     void* Y = at<void>(ws, q.Y);
 
+    stage_mark(0, s);
     if (p->dtype == MOE_BF16) {
         if (moe::launch_router_gemm(x, p->T, p->d_model, Wr, br, p->E, at<void>(ws, q.split),
                                     logits, st, s, &launches) != cudaSuccess)
@@ -280,11 +289,38 @@ moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, con
         moe::launch_logits_f32((const float*)x, Wr, br, p->T, p->d_model, p->E, logits, s,
                                &launches);
     }
-    route_steps(p, logits, ids, w, slot, drop, counts, offsets, rowtok, ws, q, s, &launches);
-    r = ffn_steps(p, x, offsets, rowtok, W1, b1, W2, b2, Y, ws, q, s, &launches);
-    if (r != MOE_OK) return r;
+    stage_mark(1, s);
+    const long long K = capacity_of(p);
+    moe::launch_route_topk(logits, p->T, p->E, p->k, ids, w, s);
+    launches += 1;
+    stage_mark(2, s);
+    moe::launch_capacity_select(ids, w, p->T, p->E, p->k, K, at<int32_t>(ws, q.cnt),
+                                at<int32_t>(ws, q.base), at<int32_t>(ws, q.nrecv),
+                                at<int32_t>(ws, q.cand), slot, drop, counts, offsets, rowtok, st,
+                                s, &launches);
+    stage_mark(3, s);
+    const long long R = max_rows_of(p, K);
+    if (R > 0 && p->dtype == MOE_BF16) {
+        void* H = at<void>(ws, q.H);
+        if (moe::launch_expert_gemm(0, x, p->d_model, rowtok, p->T, offsets, p->E, p->d_model,
+                                    p->d_ff, W1, b1, H, p->d_ff, R, st, s, &launches) !=
+            cudaSuccess)
+            return MOE_ERR_CUDA;
+        stage_mark(4, s);
+        if (moe::launch_expert_gemm(1, H, p->d_ff, nullptr, (int)R, offsets, p->E, p->d_ff,
+                                    p->d_model, W2, b2, Y, p->d_model, R, st, s, &launches) !=
+            cudaSuccess)
+            return MOE_ERR_CUDA;
+        stage_mark(5, s);
+    } else {
+        r = ffn_steps(p, x, offsets, rowtok, W1, b1, W2, b2, Y, ws, q, s, &launches);
+        if (r != MOE_OK) return r;
+        stage_mark(4, s);
+        stage_mark(5, s);
+    }
     moe::launch_combine(p->dtype, x, Y, w, ids, slot, offsets, p->T, p->d_model, p->E, p->k, out,
                         st, s, &launches);
+    stage_mark(6, s);
     return finish(launches);
 }
 
@@ -307,6 +343,20 @@ moe_status moe_reset_device_status(void* ws, size_t ws_bytes, void* stream) {
 }
 
 int32_t moe_last_launch_count(void) { return g_last_launches; }
+
+moe_status moe_set_stage_events(void* const* events, int32_t n) {
+    if (!events || n == 0) {
+        g_stage_on = false;
+        return MOE_OK;
+    }
+    if (n < MOE_STAGE_EVENTS) return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < MOE_STAGE_EVENTS; ++i) {
+        if (!events[i]) return MOE_ERR_INVALID_ARG;
+        g_stage_events[i] = (cudaEvent_t)events[i];
+    }
+    g_stage_on = true;
+    return MOE_OK;
+}
 
 const char* moe_status_string(moe_status s) {
     switch (s) {

@@ -277,6 +277,14 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     }
     const int32_t* list = cand + (size_t)e * T;
 
+    if (K == 0) {                       // no slots: every pair of this expert is dropped
+        for (int i = tid; i < n; i += blockDim.x) {
+            const int p = list[i];
+            slot[p] = -1;
+            drop[p] = 1;
+        }
+        return;
+    }
     if (n <= K) {
         for (int i = tid; i < n; i += blockDim.x) {
             const int p = list[i];

@@ -51,6 +51,7 @@ def _load():
         "moe_forward": [P] + [vp] * 15 + [sz, vp],
         "moe_get_device_status": [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)],
         "moe_reset_device_status": [vp, sz, vp],
+        "moe_set_stage_events": [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -67,7 +68,11 @@ _lib = _load()
 
 EXPORTS = ("moe_capacity", "moe_workspace_size", "moe_route", "moe_dispatch", "moe_expert_ffn",
            "moe_combine", "moe_forward", "moe_get_device_status", "moe_reset_device_status",
-           "moe_last_launch_count", "moe_status_string")
+           "moe_last_launch_count", "moe_status_string", "moe_set_stage_events")
+
+STAGE_EVENTS = 7
+STAGE_NAMES = ("router_logits", "route_topk", "capacity_dispatch", "expert_gemm1",
+               "expert_gemm2", "combine")
 
 
 def lib():
@@ -165,6 +170,15 @@ def moe_reset_device_status(ws, stream=None):
 
 def moe_last_launch_count() -> int:
     return int(_lib.moe_last_launch_count())
+
+
+def moe_set_stage_events(events):
+    """``events``: STAGE_EVENTS torch.cuda.Event objects (or None to turn recording off)."""
+    if not events:
+        _check(_lib.moe_set_stage_events(None, 0), "moe_set_stage_events")
+        return
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(_lib.moe_set_stage_events(arr, len(events)), "moe_set_stage_events")
 
 
 # ----------------------------------------------------------------------------------------------

@@ -134,6 +134,14 @@ moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, con
                        int32_t* slot_out, uint8_t* drop_out, int32_t* counts_out, void* ws,
                        size_t ws_bytes, void* stream);
 
+/* Profiling aid, host only, per calling thread.  With n >= MOE_STAGE_EVENTS, moe_forward records
+ * events[0..6] (cudaEvent_t handles owned by the caller) on its stream at: entry, after the
+ * router logits, after softmax/top-k, after capacity selection and dispatch, after the first
+ * expert GEMM, after the second expert GEMM, after the combine.  n = 0 (or events NULL) turns
+ * it off.  Recording adds no synchronisation; the handles must outlive the calls that use them. */
+#define MOE_STAGE_EVENTS 7
+moe_status moe_set_stage_events(void* const* events, int32_t n);
+
 /* Reads the device status word of `ws` (synchronises `stream`). */
 moe_status moe_get_device_status(const void* ws, size_t ws_bytes, void* stream, int32_t* code);
 

@@ -74,7 +74,10 @@ def _c(a, dt):
 
 
 def capacity(T, E, k, C):
-    return int(lib().oracle_capacity(T, E, k, float(C)))
+    """K = min(T, floor(C*T*k/E)).  The library's interface carries C as a float32, so the
+    oracle evaluates that same float32 value (e.g. 0.9 -> 0.89999998 gives 629, not 630, for
+    T=700, k=3, E=3)."""
+    return int(lib().oracle_capacity(T, E, k, float(np.float32(C))))
 
 
 def own_exp(x):
