@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -371,3 +372,98 @@ const char* moe_status_string(moe_status s) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------------
+// moe_route_static: moe_route for callers that cannot allocate device memory.
+//
+// Some callers have no way to hand the library a workspace: plug-ins inside an inference engine
+// that owns all device memory and gives its plug-ins no allocator, and latency-bound serving
+// loops whose policy forbids cudaMalloc/cudaFree on the request path (an allocation can
+// synchronise the device and stall every stream).  This entry point runs the same router and
+// capacity kernels as moe_route, with their scratch (per-chunk counts and prefixes, per-expert
+// candidate lists, the status word) placed in one file-scope __device__ array below.
+//
+// The array is a fixed kRouteStaticBytes per GPU, held by every GPU that loads the library until
+// the process exits.  Host code only sees a stand-in for it, so the device address is fetched
+// with cudaGetSymbolAddress once per device (first call on that device, with it current) and
+// cached.  The call allocates nothing and calls no allocating routine.
+// ------------------------------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kRouteStaticBytes = 8u << 20;   // 8 MiB per device
+constexpr int kMaxStaticDevices = 64;
+
+__device__ __align__(256) unsigned char g_route_static_scratch[kRouteStaticBytes];
+
+std::mutex g_static_mu;
+std::atomic<void*> g_static_ptr[kMaxStaticDevices];
+
+// Scratch layout of moe_route inside the static array; returns the bytes it needs.
+size_t route_static_layout(const moe_problem* p, size_t* cnt, size_t* base, size_t* nrecv,
+                           size_t* cand) {
+    const size_t nC = (size_t)moe::chunk_count(p->T);
+    size_t off = align_up(sizeof(moe::DeviceStatus));
+    *cnt = off;
+    off = align_up(off + (size_t)p->E * nC * 4);
+    *base = off;
+    off = align_up(off + (size_t)p->E * nC * 4);
+    *nrecv = off;
+    off = align_up(off + (size_t)p->E * 4);
+    *cand = off;
+    off = align_up(off + (size_t)p->E * p->T * 4);
+    return off;
+}
+
+void* static_scratch_for_current_device(cudaError_t* err) {
+    int dev = 0;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess) return nullptr;
+    if (dev < 0 || dev >= kMaxStaticDevices) {
+        *err = cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    void* ptr = g_static_ptr[dev].load(std::memory_order_acquire);
+    if (ptr) return ptr;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    ptr = g_static_ptr[dev].load(std::memory_order_relaxed);
+    if (!ptr) {
+        *err = cudaGetSymbolAddress(&ptr, g_route_static_scratch);
+        if (*err != cudaSuccess) return nullptr;
+        g_static_ptr[dev].store(ptr, std::memory_order_release);
+    }
+    return ptr;
+}
+
+}  // namespace
+
+extern "C" moe_status moe_route_static(const moe_problem* p, const float* logits, int32_t* ids,
+                                       float* w, int32_t* slot, uint8_t* drop, int32_t* counts,
+                                       void* stream) {
+    moe_status r = pre(p, false);
+    if (r != MOE_OK) return r;
+    if (!counts || (p->T > 0 && (!logits || !ids || !w || !slot || !drop)))
+        return MOE_ERR_INVALID_ARG;
+    size_t o_cnt, o_base, o_nrecv, o_cand;
+    if (route_static_layout(p, &o_cnt, &o_base, &o_nrecv, &o_cand) > kRouteStaticBytes)
+        return MOE_ERR_WORKSPACE;
+    cudaError_t err;
+    void* scratch = static_scratch_for_current_device(&err);
+    if (!scratch) return MOE_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (p->T == 0) {
+        cudaMemsetAsync(counts, 0, sizeof(int32_t) * 2 * p->E, s);
+        return finish(0);
+    }
+    // The array keeps the previous call's contents: the status word must start at zero; every
+    // other region is fully written by this call before it is read.
+    moe::DeviceStatus* st = at<moe::DeviceStatus>(scratch, 0);
+    cudaMemsetAsync(st, 0, sizeof(moe::DeviceStatus), s);
+    int launches = 0;
+    moe::launch_route_topk(logits, p->T, p->E, p->k, ids, w, s);
+    launches += 1;
+    moe::launch_capacity_select(ids, w, p->T, p->E, p->k, capacity_of(p),
+                                at<int32_t>(scratch, o_cnt), at<int32_t>(scratch, o_base),
+                                at<int32_t>(scratch, o_nrecv), at<int32_t>(scratch, o_cand),
+                                slot, drop, counts, nullptr, nullptr, st, s, &launches);
+    return finish(launches);
+}

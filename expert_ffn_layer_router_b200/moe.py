@@ -52,6 +52,7 @@ def _load():
         "moe_get_device_status": [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)],
         "moe_reset_device_status": [vp, sz, vp],
         "moe_set_stage_events": [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32],
+        "moe_route_static": [P, vp, vp, vp, vp, vp, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -68,7 +69,8 @@ _lib = _load()
 
 EXPORTS = ("moe_capacity", "moe_workspace_size", "moe_route", "moe_dispatch", "moe_expert_ffn",
            "moe_combine", "moe_forward", "moe_get_device_status", "moe_reset_device_status",
-           "moe_last_launch_count", "moe_status_string", "moe_set_stage_events")
+           "moe_last_launch_count", "moe_status_string", "moe_set_stage_events",
+           "moe_route_static")
 
 STAGE_EVENTS = 7
 STAGE_NAMES = ("router_logits", "route_topk", "capacity_dispatch", "expert_gemm1",

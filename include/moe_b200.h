@@ -142,6 +142,24 @@ moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, con
 #define MOE_STAGE_EVENTS 7
 moe_status moe_set_stage_events(void* const* events, int32_t n);
 
+/* moe_route without a workspace, for callers that cannot allocate device memory: plug-ins of an
+ * inference engine that owns all device memory and gives its plug-ins no allocator, and serving
+ * loops that may not call cudaMalloc/cudaFree on the request path (an allocation can
+ * synchronise the device).  The paper has no counterpart; it is a deployment aid.
+ *   Same arguments, outputs and results as moe_route (bit for bit), minus ws/ws_bytes.  The
+ *   router/capacity scratch lives in one fixed 8 MiB array of device memory per GPU, part of the
+ *   library image and held by every GPU that loads the library until the process exits.  Needs
+ *   16 + 8*E*ceil(T/32) + 4*E + 4*E*T bytes (each part rounded up to 256); larger problems get
+ *   MOE_ERR_WORKSPACE before anything is launched (T=16384 with E=64 fits; T=65536 with E=128
+ *   does not).
+ *   The first call on a device looks up the array's device address (with that device current)
+ *   and caches it; make that first call before any stream capture.
+ *   Every call on a device shares the one array: calls that overlap on the GPU (other streams,
+ *   other host threads) race and corrupt each other's results; serialise them.  Nothing is
+ *   allocated, and no allocating routine is called. */
+moe_status moe_route_static(const moe_problem* p, const float* logits, int32_t* ids, float* w,
+                            int32_t* slot, uint8_t* drop, int32_t* counts, void* stream);
+
 /* Reads the device status word of `ws` (synchronises `stream`). */
 moe_status moe_get_device_status(const void* ws, size_t ws_bytes, void* stream, int32_t* code);
 
