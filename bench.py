@@ -11,6 +11,7 @@ d_model=2048, d_ff=1408, capacity factor 1.0).  Under torchrun each rank runs it
 same workload per step, extrapolated to the whole batch).
 """
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -46,6 +47,10 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--min-warmup-s", type=float, default=0.5,
+                    help="warm-up lasts at least this long (clock sampler coverage)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's token count (profiling of smaller cases)")
     return ap.parse_args()
 
 
@@ -249,6 +254,8 @@ def run_cuda(args):
                                 device_id=dev)
 
     spec = inputs.CONFIGS[args.config]
+    if args.tokens:
+        spec = dataclasses.replace(spec, T=args.tokens)
     L = inputs.make_layer(spec, seed=args.seed + rank)
     layer = moe.MoELayer(spec.T, spec.d_model, spec.d_ff, spec.E, spec.k, spec.C, spec.dtype,
                          device=dev)
@@ -268,7 +275,7 @@ def run_cuda(args):
     # The clock sampler runs from the warm-up through the timed steps (same load); warm-up lasts
     # at least W steps and at least half a second so the sampler sees the part under load.
     sampler.start()
-    t_end = time.perf_counter() + 0.5
+    t_end = time.perf_counter() + args.min_warmup_s
     n_warm = 0
     while n_warm < max(args.warmup, 3) or time.perf_counter() < t_end:
         flush.zero_()
