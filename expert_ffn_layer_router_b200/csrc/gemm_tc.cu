@@ -26,6 +26,7 @@
 
 #include <cstdint>
 #include <cstdio>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -143,9 +144,10 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, const int* s_mt, int E
     return c;
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
     using C = Cfg<BN>;
     constexpr int S = C::kStages;
     extern __shared__ uint8_t smem_raw[];
@@ -168,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(full_bar(s), 1 + 128);
+            mbar_init(full_bar(s), GATHER ? 1 + 128 : 1);
             mbar_init(empty_bar(s), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -177,6 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
+        if (!GATHER) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
     }
     if (warp == 1) {
         __syncwarp();
@@ -223,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kIdesc = idesc_bf16_m128(BN);
 
     if (warp == 0) {
-        // ---------------- B producer (TMA) ----------------
+        // ---------------- TMA producer: B (weights), and A when its rows are contiguous --------
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
@@ -234,7 +237,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1u;
                     if (!mbar_wait(empty_bar(s), ph ^ 1u, st, 1)) { ok = false; break; }
-                    mbar_arrive_expect_tx(full_bar(s), C::kBBytes);
+                    mbar_arrive_expect_tx(full_bar(s),
+                                          GATHER ? C::kBBytes : C::kABytes + C::kBBytes);
+                    if (!GATHER) tma_load_2d(sA(s), &tmA, full_bar(s), kb * kBK, tc.row0);
                     tma_load_2d(sB(s), &tmB, full_bar(s), kb * kBK, brow);
                 }
             }
@@ -253,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1u;
                     if (!mbar_wait(full_bar(s), ph, st, 3)) { ok = false; break; }
+                    if (GATHER) fence_proxy_async_smem();   // cp.async rows -> tensor-core reads
                     tc_fence_after();
                     const uint64_t da = smem_desc_sw128(sA(s));
                     const uint64_t db = smem_desc_sw128(sB(s));
@@ -314,15 +320,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     else tmem_ld16_wait(taddr + c0, v);
                     if (!row_ok || n0 + c0 >= args.Nout) continue;
                     const int nc = min(ncol, args.Nout - (n0 + c0));     // 16 or 32
+                    if (bias) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4) {
+                            if (i >= nc) break;
+                            const float4 bv = __ldg(reinterpret_cast<const float4*>(bias + c0 + i));
+                            v[i] += bv.x; v[i + 1] += bv.y; v[i + 2] += bv.z; v[i + 3] += bv.w;
+                        }
+                    }
                     uint32_t pk[16];
 #pragma unroll
                     for (int i = 0; i < 32; i += 2) {
                         if (i >= nc) break;
                         float a0 = v[i], a1 = v[i + 1];
-                        if (bias) {
-                            a0 = __fadd_rn(a0, __ldg(bias + c0 + i));
-                            a1 = __fadd_rn(a1, __ldg(bias + c0 + i + 1));
-                        }
                         if (EPI == kEpiSiLU) {
                             a0 = __fdividef(a0, 1.0f + __expf(-a0));
                             a1 = __fdividef(a1, 1.0f + __expf(-a1));
@@ -343,8 +353,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             mbar_arrive(tempty_bar(b));
         }
-    } else {
+    } else if (GATHER) {
         // ---------------- A producers (cp.async, gathered rows) ----------------
+        // Each thread issues its 16-byte copies for a stage and lets the hardware arrive on the
+        // stage's full barrier when they have landed (cp.async.mbarrier.arrive.noinc), so all
+        // stages can be in flight at once and no producer thread ever blocks on its own copies.
+        // The MMA thread makes the landed rows visible to the tensor cores with a proxy fence.
         const int at = threadIdx.x - 192;             // 0..127
         const int chunk = at & 7;                     // 16-byte chunk of the 128-byte row
         const int rbase = at >> 3;                    // rows rbase + 16 i
@@ -379,17 +393,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
                     if (valid[i]) cp_async_16(dA + dst_off[i], src[i] + kb * kBK);
-                cp_async_commit();
-                if (it > 0) {
-                    cp_async_wait<1>();
-                    fence_proxy_async_smem();
-                    mbar_arrive(full_bar((it - 1) % S));
-                }
+                cp_async_arrive_noinc(full_bar(s));
             }
         }
         cp_async_wait<0>();
-        fence_proxy_async_smem();
-        if (ok && it > 0) mbar_arrive(full_bar((it - 1) % S));
     }
 
     tc_fence_before();
@@ -469,39 +476,44 @@ int num_sms() {
     return g_num_sms;
 }
 
-template <int BN, int EPI>
-cudaError_t launch_gemm_t(const CUtensorMap& tm, const GemmArgs& a, int grid, cudaStream_t s) {
+// The dynamic shared-memory attribute is per device; remember which devices have it.
+template <int BN, int EPI, bool GATHER>
+cudaError_t launch_gemm_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
+                          int grid, cudaStream_t s) {
     using C = Cfg<BN>;
-    static bool attr_done = false;
-    if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<BN, EPI>,
+    static std::atomic<uint64_t> attr_done{0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(attr_done.load() & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<BN, EPI, GATHER>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kSmemBytes);
         if (e != cudaSuccess) return e;
-        attr_done = true;
+        attr_done.fetch_or(bit);
     }
-    grouped_gemm_kernel<BN, EPI><<<grid, kThreads, C::kSmemBytes, s>>>(tm, a);
+    grouped_gemm_kernel<BN, EPI, GATHER><<<grid, kThreads, C::kSmemBytes, s>>>(tmA, tmB, a);
     return cudaGetLastError();
 }
 
-template <int EPI>
-cudaError_t launch_gemm_bn(int BN, const CUtensorMap& tm, const GemmArgs& a, int grid,
-                           cudaStream_t s) {
+template <int EPI, bool GATHER>
+cudaError_t launch_gemm_bn(int BN, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                           const GemmArgs& a, int grid, cudaStream_t s) {
     switch (BN) {
-        case 256: return launch_gemm_t<256, EPI>(tm, a, grid, s);
-        case 192: return launch_gemm_t<192, EPI>(tm, a, grid, s);
-        case 176: return launch_gemm_t<176, EPI>(tm, a, grid, s);
-        case 128: return launch_gemm_t<128, EPI>(tm, a, grid, s);
+        case 256: return launch_gemm_t<256, EPI, GATHER>(tmA, tmB, a, grid, s);
+        case 192: return launch_gemm_t<192, EPI, GATHER>(tmA, tmB, a, grid, s);
+        case 176: return launch_gemm_t<176, EPI, GATHER>(tmA, tmB, a, grid, s);
+        case 128: return launch_gemm_t<128, EPI, GATHER>(tmA, tmB, a, grid, s);
         default: return cudaErrorInvalidValue;
     }
 }
 
-cudaError_t launch_router_bn(int BN, const CUtensorMap& tm, const GemmArgs& a, int grid,
-                             cudaStream_t s) {
+cudaError_t launch_router_bn(int BN, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                             const GemmArgs& a, int grid, cudaStream_t s) {
     switch (BN) {
-        case 192: return launch_gemm_t<192, kEpiRouter>(tm, a, grid, s);
-        case 96: return launch_gemm_t<96, kEpiRouter>(tm, a, grid, s);
-        case 48: return launch_gemm_t<48, kEpiRouter>(tm, a, grid, s);
+        case 192: return launch_gemm_t<192, kEpiRouter, false>(tmA, tmB, a, grid, s);
+        case 96: return launch_gemm_t<96, kEpiRouter, false>(tmA, tmB, a, grid, s);
+        case 48: return launch_gemm_t<48, kEpiRouter, false>(tmA, tmB, a, grid, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -549,8 +561,21 @@ cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const in
     a.st = st;
     const long long max_tiles = ((max_rows + kBM - 1) / kBM + E) * a.n_tiles;
     const int grid = (int)std::min<long long>(num_sms(), std::max<long long>(max_tiles, 1));
-    cudaError_t e = which == 0 ? launch_gemm_bn<kEpiSiLU>(BN, tm, a, grid, s)
-                               : launch_gemm_bn<kEpiBias>(BN, tm, a, grid, s);
+    // Contiguous A rows (no gather): a TMA tile map over the A buffer, 128-row boxes.
+    CUtensorMap tmA;
+    const bool gather = a_rows != nullptr;
+    if (gather) {
+        tmA = tm;                                       // unused by the gathering kernel
+    } else if (!make_tmap(&tmA, A, (long long)a_row_limit, K, kBM)) {
+        return cudaErrorInvalidValue;
+    }
+    cudaError_t e;
+    if (which == 0)
+        e = gather ? launch_gemm_bn<kEpiSiLU, true>(BN, tmA, tm, a, grid, s)
+                   : launch_gemm_bn<kEpiSiLU, false>(BN, tmA, tm, a, grid, s);
+    else
+        e = gather ? launch_gemm_bn<kEpiBias, true>(BN, tmA, tm, a, grid, s)
+                   : launch_gemm_bn<kEpiBias, false>(BN, tmA, tm, a, grid, s);
     if (e == cudaSuccess) *launches += 1;
     return e;
 }
@@ -591,7 +616,9 @@ cudaError_t launch_router_gemm(const void* x, int T, int d, const float* Wr, con
     a.st = st;
     const long long tiles = (long long)((T + kBM - 1) / kBM) * ntl;
     const int grid = (int)std::min<long long>(num_sms(), std::max<long long>(tiles, 1));
-    cudaError_t e = launch_router_bn(BN, tm, a, grid, s);
+    CUtensorMap tmA;
+    if (!make_tmap(&tmA, x, (long long)T, d, kBM)) return cudaErrorInvalidValue;
+    cudaError_t e = launch_router_bn(BN, tmA, tm, a, grid, s);
     if (e == cudaSuccess) *launches += 1;
     return e;
 }

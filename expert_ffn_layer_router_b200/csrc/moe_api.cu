@@ -224,7 +224,8 @@ moe_status moe_expert_ffn(const moe_problem* p, const void* x, const int32_t* of
     if (r != MOE_OK) return r;
     if (!offsets || !W1 || !W2 || (p->T > 0 && (!x || !rowtok || !Y))) return MOE_ERR_INVALID_ARG;
     if (p->dtype == MOE_BF16 &&
-        (misaligned(x, 16) || misaligned(W1, 16) || misaligned(W2, 16) || misaligned(Y, 16)))
+        (misaligned(x, 16) || misaligned(W1, 16) || misaligned(W2, 16) || misaligned(Y, 16) ||
+         misaligned(b1, 16) || misaligned(b2, 16)))
         return MOE_ERR_INVALID_ARG;
     Plan q;
     if ((r = check_ws(p, ws, ws_bytes, &q)) != MOE_OK) return r;
@@ -260,7 +261,8 @@ moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, con
     if (!Wr || !W1 || !W2 || (p->T > 0 && (!x || !out))) return MOE_ERR_INVALID_ARG;
     if (out && out == x) return MOE_ERR_INVALID_ARG;
     if (p->dtype == MOE_BF16 &&
-        (misaligned(x, 16) || misaligned(W1, 16) || misaligned(W2, 16) || misaligned(out, 16)))
+        (misaligned(x, 16) || misaligned(W1, 16) || misaligned(W2, 16) || misaligned(out, 16) ||
+         misaligned(b1, 16) || misaligned(b2, 16)))
         return MOE_ERR_INVALID_ARG;
     Plan q;
     if ((r = check_ws(p, ws, ws_bytes, &q)) != MOE_OK) return r;

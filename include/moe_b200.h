@@ -35,8 +35,8 @@
  *     t (j = 0 is the largest logit).  W1 is [E, d_ff, d_model] and W2 is [E, d_model, d_ff]
  *     ("out x in", so h = W1 x).  b1 is [E, d_ff] and b2 is [E, d_model], float32 always.
  *   - dtype MOE_BF16: x, W1, W2, out and expert outputs are bfloat16, accumulation is float32
- *     on the tensor cores; d_model and d_ff must be multiples of 64 and bf16 pointers 16-byte
- *     aligned.  dtype MOE_F32: everything float32 on CUDA cores (small layers).
+ *     on the tensor cores; d_model and d_ff must be multiples of 64, and bf16 pointers and the
+ *     biases 16-byte aligned.  dtype MOE_F32: everything float32 on CUDA cores (small layers).
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
