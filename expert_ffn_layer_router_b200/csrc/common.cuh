@@ -47,26 +47,39 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                  : "memory");
 }
 
+// kCluster: acquire at cluster scope (the phase was completed by arrivals from the other CTA of
+// a pair); otherwise at CTA scope.
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
+    if (kCluster)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
     return ok != 0;
 }
 
 // Waits for the phase of parity `parity` to complete.  Gives up after kWaitLimitNs, or as soon
 // as another thread has recorded an error, and then returns false after recording a timeout.
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, DeviceStatus* st,
                                           int where) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait<kCluster>(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait<kCluster>(bar, parity)) return true;
         if (*reinterpret_cast<volatile int32_t*>(&st->code) != 0) return false;
         if (global_ns() - t0 > kWaitLimitNs) {
             report(st, MOE_DEV_TIMEOUT, where);
@@ -158,13 +171,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
     return d;
 }
 
-// Instruction descriptor: bf16 x bf16 -> fp32, both operands K-major, M = 128, N = n.
-__host__ __device__ constexpr uint32_t idesc_bf16_m128(int n) {
+// Instruction descriptor: bf16 x bf16 -> fp32, both operands K-major, M = m (128, or 256 for a
+// CTA pair), N = n.
+__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
     return (1u << 4)                       // D format fp32
            | (1u << 7)                     // A format bf16
            | (1u << 10)                    // B format bf16
            | ((uint32_t)(n >> 3) << 17)    // N / 8
-           | ((uint32_t)(128 >> 4) << 24); // M / 16
+           | ((uint32_t)(m >> 4) << 24);   // M / 16
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

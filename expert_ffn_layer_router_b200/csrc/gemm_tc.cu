@@ -26,6 +26,7 @@
 
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 #include <atomic>
 #include <mutex>
 
@@ -36,9 +37,10 @@ namespace moe {
 
 namespace {
 
-constexpr int kBM = 128;            // rows per tile (tcgen05 M)
+constexpr int kBM = 128;            // rows per CTA tile (TMEM lanes)
 constexpr int kBK = 64;             // K per stage: one 128-byte swizzle atom of bf16
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;       // 14 warps (roles below)
+constexpr int kEpiWarps = 8;        // two per TMEM lane quadrant, each half of the columns
 constexpr int kTmemCols = 512;      // two accumulators at column 0 and 256
 constexpr int kMaxGroups = 1024;
 
@@ -63,18 +65,26 @@ struct GemmArgs {
     DeviceStatus* st;
 };
 
-template <int BN>
+// PAIR: two CTAs of a cluster share one 256-row tile; each holds its 128 A rows and half of the
+// BN B rows in shared memory, the pair's tensor cores compute the 256 x BN product together.
+template <int BN, bool PAIR>
 struct Cfg {
-    static constexpr int kABytes = kBM * kBK * 2;           // 16 KB
-    static constexpr int kBBytes = BN * kBK * 2;
+    static constexpr int kTileM = PAIR ? 256 : 128;
+    static constexpr int kBRows = PAIR ? BN / 2 : BN;          // B rows held by this CTA
+    static constexpr int kABytes = kBM * kBK * 2;                // 16 KB
+    static constexpr int kBBytes = kBRows * kBK * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStages = (200 * 1024) / kStageBytes > 8 ? 8 : (200 * 1024) / kStageBytes;
-    static constexpr int kBarOff = kStages * kStageBytes;
-    static constexpr int kTableOff = kBarOff + 256;
+    static constexpr int kStgOff = kStages * kStageBytes;        // epilogue staging, 2 KB a warp
+    static constexpr int kStgBytes = kEpiWarps * 2048;
+    static constexpr int kBarOff = kStgOff + kStgBytes;
+    static constexpr int kTableOff = kBarOff + 512;
     static constexpr int kSmemBytes = 1024 + kTableOff + (kMaxGroups + 1) * 4;
     static_assert(kStages >= 2, "at least two stages");
-    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 N for M=128");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 N for M=128 / M=256");
     static_assert(kBBytes % 1024 == 0, "B stage must stay 1024-byte aligned");
+    static_assert(8 * (3 * kStages + 4) + 4 <= 512, "barrier area");
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
 __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c,
@@ -121,13 +131,93 @@ __device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, float* v) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Tile t -> (group, first row, valid rows, column tile).  s_mt[e] = m-tiles before group e.
+// ---- pair (cta_group::2) primitives ----
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Address of the same shared-memory location in CTA `cta` of this cluster.
+__device__ __forceinline__ uint32_t map_to_cta(uint32_t addr, uint32_t cta) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(cta));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                     cluster_addr)
+                 : "memory");
+}
+// TMA 2-D load whose completion is counted on a barrier of either CTA of the pair.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap, uint32_t bar,
+                                                 int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(tmap), "r"(bar), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     dst_smem),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc,
+                                                 uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrives on the barrier at this shared offset in both CTAs of the pair once the pair's MMAs
+// issued so far have completed.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], m;\n\t}" ::"r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
+
+// Tile t -> (group, first row of this CTA, valid rows of this CTA, column tile).
+// s_mt[e] = tiles of kTileM rows before group e; `half` = this CTA's 128-row half (pairs).
 struct TileCoord {
     int e, row0, rows, nt;
 };
 
+template <int kTileM>
 __device__ __forceinline__ TileCoord tile_coord(int tile, const int* s_mt, int E, int n_tiles,
-                                                const GemmArgs& a) {
+                                                const GemmArgs& a, int half) {
     TileCoord c;
     const int mt = tile / n_tiles;
     c.nt = tile - mt * n_tiles;
@@ -139,17 +229,19 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, const int* s_mt, int E
     c.e = lo;
     const int g0 = a.offsets ? __ldg(a.offsets + lo) : 0;
     const int g1 = a.offsets ? __ldg(a.offsets + lo + 1) : a.rows0;
-    c.row0 = g0 + (mt - s_mt[lo]) * kBM;
-    c.rows = min(kBM, g1 - c.row0);
+    c.row0 = g0 + (mt - s_mt[lo]) * kTileM + half * kBM;
+    c.rows = min(kBM, g1 - c.row0);         // <= 0: this CTA's half of the tile is empty
     return c;
 }
 
-template <int BN, int EPI, bool GATHER>
+template <int BN, int EPI, bool GATHER, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
-    using C = Cfg<BN>;
+    static_assert(!(GATHER && PAIR), "gathered A rows run on single-CTA tiles");
+    using C = Cfg<BN, PAIR>;
     constexpr int S = C::kStages;
+    constexpr int TM = C::kTileM;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -157,9 +249,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar0 = base + C::kBarOff;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
-    auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * S + b); };
-    auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * S + 2 + b); };
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base_ptr + C::kBarOff + 8 * (2 * S + 4));
+    auto tfull_bar = [&](int b) { return bar0 + 8u * (3 * S + b); };
+    auto tempty_bar = [&](int b) { return bar0 + 8u * (3 * S + 2 + b); };
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base_ptr + C::kBarOff + 8 * (3 * S + 4));
     int* s_mt = reinterpret_cast<int*>(base_ptr + C::kTableOff);
     auto sA = [&](int s) { return base + (uint32_t)s * C::kABytes; };
     auto sB = [&](int s) { return base + (uint32_t)S * C::kABytes + (uint32_t)s * C::kBBytes; };
@@ -167,15 +259,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = args.E;
     DeviceStatus* st = args.st;
+    const uint32_t crank = PAIR ? cluster_rank() : 0u;
+    const bool leader = crank == 0;
+    const int cid = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;      // tile walker id
+    const int ncl = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < S; ++s) {
+            // producer arrive + expected bytes; gathered rows add one arrival per A thread
             mbar_init(full_bar(s), GATHER ? 1 + 128 : 1);
             mbar_init(empty_bar(s), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar(b), 1);
-            mbar_init(tempty_bar(b), 128);
+            mbar_init(tempty_bar(b), (PAIR ? 2 : 1) * kEpiWarps * 32);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
@@ -183,11 +280,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (warp == 1) {
         __syncwarp();
-        tmem_alloc(smem_u32(s_tmem), kTmemCols);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(smem_u32(s_tmem), kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(s_tmem), kTmemCols);
+            tmem_relinquish();
+        }
     }
     if (warp == 2) {
-        // m-tile prefix over groups: lane l sums groups [l*per, (l+1)*per).
+        // Tile prefix over groups: lane l sums groups [l*per, (l+1)*per).
         const int per = (E + 31) / 32;
         int loc = 0;
         for (int q = 0; q < per; ++q) {
@@ -195,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (e < E) {
                 const int n = args.offsets ? __ldg(args.offsets + e + 1) - __ldg(args.offsets + e)
                                            : args.rows0;
-                loc += (max(n, 0) + kBM - 1) / kBM;
+                loc += (max(n, 0) + TM - 1) / TM;
             }
         }
         int inc = loc;
@@ -211,99 +313,125 @@ __global__ void __launch_bounds__(kThreads, 1)
                 s_mt[e] = run;
                 const int n = args.offsets ? __ldg(args.offsets + e + 1) - __ldg(args.offsets + e)
                                            : args.rows0;
-                run += (max(n, 0) + kBM - 1) / kBM;
+                run += (max(n, 0) + TM - 1) / TM;
             }
         }
         if (lane == 31) s_mt[E] = inc;
     }
     tc_fence_before();
-    __syncthreads();
+    __syncwarp();
+    if (PAIR) cluster_sync_all(); else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
     const int n_tiles = args.n_tiles;
     const int total = s_mt[E] * n_tiles;
     const int nkb = args.K / kBK;
-    constexpr uint32_t kIdesc = idesc_bf16_m128(BN);
+    constexpr uint32_t kIdesc = idesc_bf16(TM, BN);
+    // Barriers of the pair's leader that both CTAs signal.
+    auto lead = [&](uint32_t addr) { return PAIR ? map_to_cta(addr, 0) : addr; };
 
     if (warp == 0) {
         // ---------------- TMA producer: B (weights), and A when its rows are contiguous --------
         if (lane == 0) {
+            constexpr uint32_t kTx = (PAIR ? 2u : 1u) * ((GATHER ? 0u : (uint32_t)C::kABytes) +
+                                                         (uint32_t)C::kBBytes);
             uint32_t it = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-                const TileCoord tc = tile_coord(tile, s_mt, E, n_tiles, args);
-                const int brow = tc.e * args.b_rows_per_group + tc.nt * BN;
+            for (int tile = cid; ok && tile < total; tile += ncl) {
+                const TileCoord tc = tile_coord<TM>(tile, s_mt, E, n_tiles, args, (int)crank);
+                const int brow = tc.e * args.b_rows_per_group + tc.nt * BN + (int)crank * C::kBRows;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1u;
-                    if (!mbar_wait(empty_bar(s), ph ^ 1u, st, 1)) { ok = false; break; }
-                    mbar_arrive_expect_tx(full_bar(s),
-                                          GATHER ? C::kBBytes : C::kABytes + C::kBBytes);
-                    if (!GATHER) tma_load_2d(sA(s), &tmA, full_bar(s), kb * kBK, tc.row0);
-                    tma_load_2d(sB(s), &tmB, full_bar(s), kb * kBK, brow);
+                    if (!mbar_wait<PAIR>(empty_bar(s), ph ^ 1u, st, 1)) { ok = false; break; }
+                    if (leader) mbar_arrive_expect_tx(full_bar(s), kTx);
+                    if (PAIR) {
+                        const uint32_t fb = lead(full_bar(s));
+                        tma_load_2d_pair(sA(s), &tmA, fb, kb * kBK, tc.row0);
+                        tma_load_2d_pair(sB(s), &tmB, fb, kb * kBK, brow);
+                    } else {
+                        if (!GATHER) tma_load_2d(sA(s), &tmA, full_bar(s), kb * kBK, tc.row0);
+                        tma_load_2d(sB(s), &tmB, full_bar(s), kb * kBK, brow);
+                    }
                 }
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
-        if (lane == 0) {
+        // ---------------- MMA issuer (the pair's leader only) ----------------
+        if (lane == 0 && leader) {
             uint32_t it = 0, lt = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++lt) {
+            for (int tile = cid; ok && tile < total; tile += ncl, ++lt) {
                 const uint32_t b = lt & 1u, use = lt >> 1;
-                if (!mbar_wait(tempty_bar(b), (use & 1u) ^ 1u, st, 2)) { ok = false; break; }
+                if (!mbar_wait<PAIR>(tempty_bar(b), (use & 1u) ^ 1u, st, 2)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + b * 256u;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1u;
-                    if (!mbar_wait(full_bar(s), ph, st, 3)) { ok = false; break; }
+                    if (!mbar_wait<PAIR>(full_bar(s), ph, st, 3)) { ok = false; break; }
                     if (GATHER) fence_proxy_async_smem();   // cp.async rows -> tensor-core reads
                     tc_fence_after();
                     const uint64_t da = smem_desc_sw128(sA(s));
                     const uint64_t db = smem_desc_sw128(sB(s));
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)
-                        tc_mma_bf16(d_tmem, da + 2u * kk, db + 2u * kk, kIdesc,
-                                    (kb | kk) != 0 ? 1u : 0u);
-                    tc_commit(empty_bar(s));
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        if (PAIR)
+                            tc_mma_bf16_pair(d_tmem, da + 2u * kk, db + 2u * kk, kIdesc,
+                                             (kb | kk) != 0 ? 1u : 0u);
+                        else
+                            tc_mma_bf16(d_tmem, da + 2u * kk, db + 2u * kk, kIdesc,
+                                        (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    if (PAIR) tc_commit_pair(empty_bar(s)); else tc_commit(empty_bar(s));
                 }
                 if (!ok) break;
-                tc_commit(tfull_bar(b));
+                if (PAIR) tc_commit_pair(tfull_bar(b)); else tc_commit(tfull_bar(b));
             }
         }
-    } else if (warp < 6) {
-        // ---------------- epilogue ----------------
-        const int q = warp & 3;                       // TMEM lane quadrant of this warp
-        const int r = q * 32 + lane;                  // tile row of this thread
+    } else if (warp < 2 + kEpiWarps) {
+        // ---------------- epilogue (this CTA's 128 rows) ----------------
+        // Warp w reads TMEM lane quadrant w % 4 (rows 32q..32q+31) and half h of the tile's
+        // 32-column chunks.  Each 32x32 block goes through a 2 KB staging buffer (64-byte rows,
+        // 16-byte chunks swizzled by (row / 2) % 4, conflict-free both ways) and leaves with
+        // stores that cover whole 64-byte row segments, 8 rows per warp instruction.
+        const int q = warp & 3;
+        const int h = (warp - 2) >> 2;
+        const uint32_t tempty_target0 = lead(tempty_bar(0));
+        const uint32_t tempty_target1 = lead(tempty_bar(1));
+        const uint32_t stg = base + C::kStgOff + (uint32_t)(warp - 2) * 2048u;
+        constexpr int kChunks = (BN + 31) / 32;
+        constexpr int kHalf = (kChunks + 1) / 2;
         uint32_t lt = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++lt) {
-            const TileCoord tc = tile_coord(tile, s_mt, E, n_tiles, args);
+        for (int tile = cid; tile < total; tile += ncl, ++lt) {
+            const TileCoord tc = tile_coord<TM>(tile, s_mt, E, n_tiles, args, (int)crank);
             const uint32_t b = lt & 1u, use = lt >> 1;
-            if (!mbar_wait(tfull_bar(b), use & 1u, st, 4)) break;
+            if (!mbar_wait<PAIR>(tfull_bar(b), use & 1u, st, 4)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + b * 256u;
-            const bool row_ok = r < tc.rows;
-            const long long orow = (long long)tc.row0 + r;
+            const int wrows = min(32, max(0, tc.rows - q * 32));      // valid rows of the warp
+            const long long wrow0 = (long long)tc.row0 + q * 32;
             if (EPI == kEpiRouter) {
                 constexpr int Eg = BN / 3;
+                if (h == 0) {
 #pragma unroll 1
-                for (int c0 = 0; c0 < Eg; c0 += 16) {
-                    float hi[16], mi[16], lo[16];
-                    __syncwarp();
-                    tmem_ld16_wait(taddr + c0, hi);
-                    tmem_ld16_wait(taddr + Eg + c0, mi);
-                    tmem_ld16_wait(taddr + 2 * Eg + c0, lo);
-                    const int e0 = tc.nt * Eg + c0;
-                    if (row_ok) {
-                        float* out = reinterpret_cast<float*>(args.D) + orow * args.ldd;
+                    for (int c0 = 0; c0 < Eg; c0 += 16) {
+                        float hi[16], mi[16], lo[16];
+                        __syncwarp();
+                        tmem_ld16_wait(taddr + c0, hi);
+                        tmem_ld16_wait(taddr + Eg + c0, mi);
+                        tmem_ld16_wait(taddr + 2 * Eg + c0, lo);
+                        const int e0 = tc.nt * Eg + c0;
+                        if (lane < wrows) {
+                            float* out = reinterpret_cast<float*>(args.D) + (wrow0 + lane) * args.ldd;
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int e = e0 + i;
-                            if (e < args.router_E) {
-                                float v = __fadd_rn(hi[i], __fadd_rn(mi[i], lo[i]));
-                                if (args.bias) v = __fadd_rn(v, __ldg(args.bias + e));
-                                out[e] = v;
+                            for (int i = 0; i < 16; ++i) {
+                                const int e = e0 + i;
+                                if (e < args.router_E) {
+                                    float v = __fadd_rn(hi[i], __fadd_rn(mi[i], lo[i]));
+                                    if (args.bias) v = __fadd_rn(v, __ldg(args.bias + e));
+                                    out[e] = v;
+                                }
                             }
                         }
                     }
@@ -312,13 +440,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int n0 = tc.nt * BN;
                 const float* bias = args.bias ? args.bias + (size_t)tc.e * args.Nout + n0 : nullptr;
 #pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 32) {
-                    float v[32];
+                for (int ci = h * kHalf; ci < kChunks && ci < (h + 1) * kHalf; ++ci) {
+                    const int c0 = ci * 32;
                     const int ncol = (BN - c0) >= 32 ? 32 : 16;
+                    float v[32];
                     __syncwarp();
                     if (ncol == 32) tmem_ld32_wait(taddr + c0, v);
                     else tmem_ld16_wait(taddr + c0, v);
-                    if (!row_ok || n0 + c0 >= args.Nout) continue;
+                    if (n0 + c0 >= args.Nout || wrows == 0) continue;
                     const int nc = min(ncol, args.Nout - (n0 + c0));     // 16 or 32
                     if (bias) {
 #pragma unroll
@@ -339,19 +468,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         pk[i >> 1] = pack_bf16x2(a0, a1);
                     }
-                    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(args.D) +
-                                         orow * args.ldd + n0 + c0;
-                    st_global_v4(out, pk[0], pk[1], pk[2], pk[3]);
-                    st_global_v4(out + 8, pk[4], pk[5], pk[6], pk[7]);
-                    if (nc == 32) {
-                        st_global_v4(out + 16, pk[8], pk[9], pk[10], pk[11]);
-                        st_global_v4(out + 24, pk[12], pk[13], pk[14], pk[15]);
+                    // Stage: this thread's row (= lane), nc/8 chunks of 16 bytes.
+                    const uint32_t rowp = stg + (uint32_t)lane * 64u;
+                    const uint32_t sw = (uint32_t)((lane >> 1) & 3);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if (j < nc / 8)
+                            st_shared_v4(rowp + ((j ^ sw) << 4), pk[4 * j], pk[4 * j + 1],
+                                         pk[4 * j + 2], pk[4 * j + 3]);
+                    __syncwarp();
+                    // Copy out: lane handles chunk lane % 4 of rows lane / 4 + 8 i.
+                    const int cc = lane & 3;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int R = (lane >> 2) + 8 * i;
+                        if (R < wrows && cc < nc / 8) {
+                            const uint4 val = ld_shared_v4(
+                                stg + (uint32_t)R * 64u + ((uint32_t)(cc ^ ((R >> 1) & 3)) << 4));
+                            __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(args.D) +
+                                                 (wrow0 + R) * args.ldd + n0 + c0 + cc * 8;
+                            st_global_v4(out, val.x, val.y, val.z, val.w);
+                        }
                     }
                 }
             }
             __syncwarp();
             tc_fence_before();
-            mbar_arrive(tempty_bar(b));
+            if (PAIR) mbar_arrive_cluster(b ? tempty_target1 : tempty_target0);
+            else mbar_arrive(tempty_bar(b));
         }
     } else if (GATHER) {
         // ---------------- A producers (cp.async, gathered rows) ----------------
@@ -359,13 +503,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // stage's full barrier when they have landed (cp.async.mbarrier.arrive.noinc), so all
         // stages can be in flight at once and no producer thread ever blocks on its own copies.
         // The MMA thread makes the landed rows visible to the tensor cores with a proxy fence.
-        const int at = threadIdx.x - 192;             // 0..127
-        const int chunk = at & 7;                     // 16-byte chunk of the 128-byte row
-        const int rbase = at >> 3;                    // rows rbase + 16 i
+        const int at = threadIdx.x - 32 * (2 + kEpiWarps);   // 0..127
+        const int chunk = at & 7;                             // 16-byte chunk of the row
+        const int rbase = at >> 3;                            // rows rbase + 16 i
         uint32_t it = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-            const TileCoord tc = tile_coord(tile, s_mt, E, n_tiles, args);
+        for (int tile = cid; ok && tile < total; tile += ncl) {
+            const TileCoord tc = tile_coord<TM>(tile, s_mt, E, n_tiles, args, 0);
             const __nv_bfloat16* src[8];
             uint32_t dst_off[8];
             bool valid[8];
@@ -374,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int r = rbase + 16 * i;
                 valid[i] = r < tc.rows;
                 long long ar = tc.row0 + r;
-                if (valid[i] && args.a_rows) {
+                if (valid[i]) {
                     const int g = __ldg(args.a_rows + tc.row0 + r);
                     if ((unsigned)g >= (unsigned)args.a_row_limit) {
                         report(st, MOE_DEV_BAD_INDEX, 501);
@@ -388,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kb = 0; kb < nkb; ++kb, ++it) {
                 const int s = it % S;
                 const uint32_t ph = (it / S) & 1u;
-                if (!mbar_wait(empty_bar(s), ph ^ 1u, st, 5)) { ok = false; break; }
+                if (!mbar_wait<PAIR>(empty_bar(s), ph ^ 1u, st, 5)) { ok = false; break; }
                 const uint32_t dA = sA(s);
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
@@ -400,11 +544,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     tc_fence_before();
-    __syncthreads();
+    __syncwarp();
+    if (PAIR) cluster_sync_all(); else __syncthreads();
     tc_fence_after();
     if (warp == 1) {
         __syncwarp();
-        tmem_dealloc(tmem_base, kTmemCols);
+        if (PAIR) tmem_dealloc_pair(tmem_base, kTmemCols);
+        else tmem_dealloc(tmem_base, kTmemCols);
     }
 }
 
@@ -450,18 +596,23 @@ bool encode_fn_ready() {
     return g_encode != nullptr;
 }
 
-// 2-D bf16 tensor map over rows x K (K contiguous), box 64 x box_rows, 128-byte swizzle.
-bool make_tmap(CUtensorMap* tm, const void* ptr, long long rows, int K, int box_rows) {
+// 2-D bf16 tensor map over rows x cols (cols contiguous, row pitch `ld` elements).
+bool make_tmap_2d(CUtensorMap* tm, const void* ptr, long long rows, int cols, long long ld,
+                  int box_cols, int box_rows, CUtensorMapSwizzle swz) {
     if (!encode_fn_ready()) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
-                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// Operand tile map: rows x K (K contiguous), box 64 x box_rows, 128-byte swizzle.
+bool make_tmap(CUtensorMap* tm, const void* ptr, long long rows, int K, int box_rows) {
+    return make_tmap_2d(tm, ptr, rows, K, K, kBK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 int g_num_sms = 0;
@@ -477,43 +628,79 @@ int num_sms() {
 }
 
 // The dynamic shared-memory attribute is per device; remember which devices have it.
-template <int BN, int EPI, bool GATHER>
+template <int BN, int EPI, bool GATHER, bool PAIR>
 cudaError_t launch_gemm_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
-                          int grid, cudaStream_t s) {
-    using C = Cfg<BN>;
+                          long long tiles, cudaStream_t s) {
+    using C = Cfg<BN, PAIR>;
+    auto kern = grouped_gemm_kernel<BN, EPI, GATHER, PAIR>;
     static std::atomic<uint64_t> attr_done{0};
+    static std::atomic<int> pair_slots[64];
     int dev = 0;
     cudaGetDevice(&dev);
     const uint64_t bit = 1ull << (dev & 63);
     if (!(attr_done.load() & bit)) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<BN, EPI, GATHER>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kSmemBytes);
         if (e != cudaSuccess) return e;
+        if (PAIR) {
+            cudaLaunchConfig_t cfg = {};
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeClusterDimension;
+            at[0].val.clusterDim.x = 2;
+            at[0].val.clusterDim.y = 1;
+            at[0].val.clusterDim.z = 1;
+            cfg.gridDim = dim3(2 * 74, 1, 1);
+            cfg.blockDim = dim3(kThreads, 1, 1);
+            cfg.dynamicSmemBytes = C::kSmemBytes;
+            cfg.attrs = at;
+            cfg.numAttrs = 1;
+            int nclusters = 0;
+            e = cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg);
+            if (e != cudaSuccess || nclusters <= 0) nclusters = num_sms() / 2;
+            pair_slots[dev & 63].store(nclusters);
+        }
         attr_done.fetch_or(bit);
     }
-    grouped_gemm_kernel<BN, EPI, GATHER><<<grid, kThreads, C::kSmemBytes, s>>>(tmA, tmB, a);
-    return cudaGetLastError();
+    if (!PAIR) {
+        const int grid = (int)std::min<long long>(num_sms(), std::max<long long>(tiles, 1));
+        kern<<<grid, kThreads, C::kSmemBytes, s>>>(tmA, tmB, a);
+        return cudaGetLastError();
+    }
+    const int clusters =
+        (int)std::min<long long>(pair_slots[dev & 63].load(), std::max<long long>(tiles, 1));
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * clusters, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = s;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, a);
 }
 
-template <int EPI, bool GATHER>
+template <int EPI, bool GATHER, bool PAIR>
 cudaError_t launch_gemm_bn(int BN, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                           const GemmArgs& a, int grid, cudaStream_t s) {
+                           const GemmArgs& a, long long tiles, cudaStream_t s) {
     switch (BN) {
-        case 256: return launch_gemm_t<256, EPI, GATHER>(tmA, tmB, a, grid, s);
-        case 192: return launch_gemm_t<192, EPI, GATHER>(tmA, tmB, a, grid, s);
-        case 176: return launch_gemm_t<176, EPI, GATHER>(tmA, tmB, a, grid, s);
-        case 128: return launch_gemm_t<128, EPI, GATHER>(tmA, tmB, a, grid, s);
+        case 256: return launch_gemm_t<256, EPI, GATHER, PAIR>(tmA, tmB, a, tiles, s);
+        case 192: return launch_gemm_t<192, EPI, GATHER, PAIR>(tmA, tmB, a, tiles, s);
+        case 176: return launch_gemm_t<176, EPI, GATHER, PAIR>(tmA, tmB, a, tiles, s);
+        case 128: return launch_gemm_t<128, EPI, GATHER, PAIR>(tmA, tmB, a, tiles, s);
         default: return cudaErrorInvalidValue;
     }
 }
 
 cudaError_t launch_router_bn(int BN, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                             const GemmArgs& a, int grid, cudaStream_t s) {
+                             const GemmArgs& a, long long tiles, cudaStream_t s) {
     switch (BN) {
-        case 192: return launch_gemm_t<192, kEpiRouter, false>(tmA, tmB, a, grid, s);
-        case 96: return launch_gemm_t<96, kEpiRouter, false>(tmA, tmB, a, grid, s);
-        case 48: return launch_gemm_t<48, kEpiRouter, false>(tmA, tmB, a, grid, s);
+        case 192: return launch_gemm_t<192, kEpiRouter, false, false>(tmA, tmB, a, tiles, s);
+        case 96: return launch_gemm_t<96, kEpiRouter, false, false>(tmA, tmB, a, tiles, s);
+        case 48: return launch_gemm_t<48, kEpiRouter, false, false>(tmA, tmB, a, tiles, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -534,14 +721,28 @@ int pick_bn(int nout) {
 
 int router_group(int E) { return E <= 16 ? 16 : (E <= 32 ? 32 : 64); }
 
+// Pair (2-SM) tiles when the experts' rows fill 256-row tiles well enough; 1-SM otherwise.
+int g_pair_mode = -1;      // -1 automatic, 0 never, 1 always (MOE_GEMM_PAIR in the environment)
+
+bool use_pair(long long max_rows, int E) {
+    if (g_pair_mode < 0) {
+        const char* v = getenv("MOE_GEMM_PAIR");
+        g_pair_mode = v ? (v[0] == '1' ? 1 : (v[0] == '0' ? 0 : 2)) : 2;
+    }
+    if (g_pair_mode == 0) return false;
+    if (g_pair_mode == 1) return true;
+    return max_rows >= 256LL * E;
+}
+
 cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const int32_t* a_rows,
                                int a_row_limit, const int32_t* offsets, int E, int K, int Nout,
                                const void* W, const float* bias, void* D, long long ldd,
                                long long max_rows, DeviceStatus* st, cudaStream_t s,
                                int* launches) {
     const int BN = pick_bn(Nout);
+    const bool pair = a_rows == nullptr && use_pair(max_rows, E);
     CUtensorMap tm;
-    if (!make_tmap(&tm, W, (long long)E * Nout, K, BN)) return cudaErrorInvalidValue;
+    if (!make_tmap(&tm, W, (long long)E * Nout, K, pair ? BN / 2 : BN)) return cudaErrorInvalidValue;
     GemmArgs a{};
     a.A = reinterpret_cast<const __nv_bfloat16*>(A);
     a.lda = lda;
@@ -559,23 +760,24 @@ cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const in
     a.ldd = ldd;
     a.router_E = 0;
     a.st = st;
-    const long long max_tiles = ((max_rows + kBM - 1) / kBM + E) * a.n_tiles;
-    const int grid = (int)std::min<long long>(num_sms(), std::max<long long>(max_tiles, 1));
-    // Contiguous A rows (no gather): a TMA tile map over the A buffer, 128-row boxes.
-    CUtensorMap tmA;
+    const int tm_rows = pair ? 256 : kBM;
+    const long long max_tiles = ((max_rows + tm_rows - 1) / tm_rows + E) * a.n_tiles;
+    // Contiguous A rows: a TMA tile map over the A buffer, 128-row boxes (unused when gathering).
+    CUtensorMap tmA = tm;
     const bool gather = a_rows != nullptr;
-    if (gather) {
-        tmA = tm;                                       // unused by the gathering kernel
-    } else if (!make_tmap(&tmA, A, (long long)a_row_limit, K, kBM)) {
+    if (!gather && !make_tmap(&tmA, A, (long long)a_row_limit, K, kBM))
         return cudaErrorInvalidValue;
-    }
     cudaError_t e;
-    if (which == 0)
-        e = gather ? launch_gemm_bn<kEpiSiLU, true>(BN, tmA, tm, a, grid, s)
-                   : launch_gemm_bn<kEpiSiLU, false>(BN, tmA, tm, a, grid, s);
-    else
-        e = gather ? launch_gemm_bn<kEpiBias, true>(BN, tmA, tm, a, grid, s)
-                   : launch_gemm_bn<kEpiBias, false>(BN, tmA, tm, a, grid, s);
+    if (gather) {
+        e = which == 0 ? launch_gemm_bn<kEpiSiLU, true, false>(BN, tmA, tm, a, max_tiles, s)
+                       : launch_gemm_bn<kEpiBias, true, false>(BN, tmA, tm, a, max_tiles, s);
+    } else if (pair) {
+        e = which == 0 ? launch_gemm_bn<kEpiSiLU, false, true>(BN, tmA, tm, a, max_tiles, s)
+                       : launch_gemm_bn<kEpiBias, false, true>(BN, tmA, tm, a, max_tiles, s);
+    } else {
+        e = which == 0 ? launch_gemm_bn<kEpiSiLU, false, false>(BN, tmA, tm, a, max_tiles, s)
+                       : launch_gemm_bn<kEpiBias, false, false>(BN, tmA, tm, a, max_tiles, s);
+    }
     if (e == cudaSuccess) *launches += 1;
     return e;
 }
@@ -615,10 +817,9 @@ cudaError_t launch_router_gemm(const void* x, int T, int d, const float* Wr, con
     a.router_E = E;
     a.st = st;
     const long long tiles = (long long)((T + kBM - 1) / kBM) * ntl;
-    const int grid = (int)std::min<long long>(num_sms(), std::max<long long>(tiles, 1));
     CUtensorMap tmA;
     if (!make_tmap(&tmA, x, (long long)T, d, kBM)) return cudaErrorInvalidValue;
-    cudaError_t e = launch_router_bn(BN, tmA, tm, a, grid, s);
+    cudaError_t e = launch_router_bn(BN, tmA, tm, a, tiles, s);
     if (e == cudaSuccess) *launches += 1;
     return e;
 }
