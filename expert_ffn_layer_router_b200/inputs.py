@@ -59,15 +59,22 @@ CONFIG_ORDER = ["tiny_f32", "bf16_e8_top2", "skewed_e64_top6", "decode_e64_top8"
 
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
-    """Round float32 to bfloat16 (nearest, ties to even) and return the raw 16-bit patterns."""
+    """Round float32 to bfloat16 (nearest, ties to even) and return the raw 16-bit patterns.
+
+    Works in uint32 (no overflow for any non-NaN pattern: the largest, -FLT_MAX, plus 0x8000
+    stays below 2^32) in chunks, so multi-GB weight tensors need no 64-bit temporaries."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    b = a.view(np.uint32).astype(np.uint64)
-    rounded = (b + 0x7FFF + ((b >> 16) & 1)) >> 16
-    out = rounded.astype(np.uint16)
-    nan = np.isnan(a)
-    if nan.any():
-        out[nan] = 0x7FC0
-    return out
+    flat = a.reshape(-1)
+    out = np.empty(flat.size, np.uint16)
+    step = 1 << 24
+    for i in range(0, flat.size, step):
+        b = flat[i:i + step].view(np.uint32)
+        r = b + np.uint32(0x7FFF) + ((b >> np.uint32(16)) & np.uint32(1))
+        out[i:i + step] = (r >> np.uint32(16)).astype(np.uint16)
+        nan = np.isnan(flat[i:i + step])
+        if nan.any():
+            out[i:i + step][nan] = 0x7FC0
+    return out.reshape(a.shape)
 
 
 def bf16_bits_to_f32(h: np.ndarray) -> np.ndarray:

@@ -197,20 +197,26 @@ def _forward_check(spec, seed, tokens=None, logit_rel=1e-4):
     lerr = np.abs(g["logits_out"] - Lref).max()
     assert lerr <= logit_rel * max(1.0, float(np.abs(Lref).max())), lerr
     ro = oracle.route(Lref, spec.k, layer.K)
-    # Expert choice is pinned by the gap screen; capacity decisions may only differ where the
-    # oracle's own weights tie within the logit error.
-    assert np.array_equal(g["ids_out"], ro["ids"])
-    dw = np.abs(g["w_out"] - ro["w"])
-    assert dw.max() <= 4 * lerr * max(1.0, float(ro["w"].max())) + 1e-6
-    mism = np.nonzero((g["slot_out"] >= 0) != (ro["slot"] >= 0))
+    # The logits differ from the oracle's by rounding, so the order of a token's experts can
+    # differ where two of its top-k logits are that close; compare per (token, expert) pair.
+    # Expert choice itself is pinned by the gap screen; capacity decisions may only differ where
+    # the oracle's own weights tie within the logit error at an expert's capacity boundary.
+    og = np.argsort(g["ids_out"], axis=1, kind="stable")
+    oo = np.argsort(ro["ids"], axis=1, kind="stable")
+    gi, gw, gs = (np.take_along_axis(g[n], og, 1) for n in ("ids_out", "w_out", "slot_out"))
+    oi, ow, os_ = (np.take_along_axis(ro[n], oo, 1) for n in ("ids", "w", "slot"))
+    assert np.array_equal(gi, oi), "expert sets differ"
+    dw = np.abs(gw - ow)
+    assert dw.max() <= 4 * lerr * max(1.0, float(ow.max())) + 1e-6
+    mism = np.nonzero((gs >= 0) != (os_ >= 0))
     for t, j in zip(*mism):
-        e = ro["ids"][t, j]
-        same_e = ro["ids"] == e
-        kept_w = ro["w"][same_e & (ro["slot"] >= 0)]
-        drop_w = ro["w"][same_e & (ro["slot"] < 0)]
+        e = oi[t, j]
+        same_e = oi == e
+        kept_w = ow[same_e & (os_ >= 0)]
+        drop_w = ow[same_e & (os_ < 0)]
         boundary = (kept_w.min() + drop_w.max()) / 2
-        assert abs(float(ro["w"][t, j]) - boundary) <= 8 * dw.max() + 1e-7, "not a near-tie"
-    agree = ((g["slot_out"] >= 0) == (ro["slot"] >= 0)).all(axis=1)
+        assert abs(float(ow[t, j]) - boundary) <= 8 * dw.max() + 1e-7, "not a near-tie"
+    agree = ((gs >= 0) == (os_ >= 0)).all(axis=1)
     assert agree.mean() >= 0.99
     T = spec.T
     if tokens is None:
