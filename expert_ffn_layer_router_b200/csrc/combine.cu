@@ -133,6 +133,79 @@ __global__ void __launch_bounds__(256) combine_kernel(
     }
 }
 
+// One warp per token, 16-byte vectors.  The token's kept pairs (row, weight), in j order, are
+// held in registers of every lane (KMAX slots, filled by shuffles); for each vector a lane issues
+// the loads of x and of all kept rows before any arithmetic (the pair loop is unrolled to KMAX
+// with predicates), so k + 1 reads per lane are in flight together.
+template <class Tr, int KMAX>
+__global__ void __launch_bounds__(256) combine_vec_kernel(
+    const uint4* __restrict__ x, const uint4* __restrict__ Y, const float* __restrict__ w,
+    const int32_t* __restrict__ ids, const int32_t* __restrict__ slot,
+    const int32_t* __restrict__ offsets, int T, int nv, int E, int k, uint4* __restrict__ out,
+    DeviceStatus* st) {
+    constexpr int V = Tr::kVec;
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    int row = -1;
+    float wt = 0.0f;
+    if (lane < k) {
+        const size_t p = (size_t)t * k + lane;
+        const int s = slot[p];
+        if (s >= 0) {
+            const int e = ids[p];
+            if ((unsigned)e < (unsigned)E) {
+                const int r = offsets[e] + s;
+                if (r < offsets[e + 1]) { row = r; wt = w[p]; }
+                else report(st, MOE_DEV_BAD_INDEX, 303);
+            } else {
+                report(st, MOE_DEV_BAD_INDEX, 304);
+            }
+        }
+    }
+    unsigned m = __ballot_sync(0xffffffffu, row >= 0);
+    const int nk = __popc(m);
+    const uint4* xr = x + (size_t)t * nv;
+    uint4* orow = out + (size_t)t * nv;
+    if (nk == 0) {
+        for (int c = lane; c < nv; c += 32) orow[c] = __ldg(xr + c);
+        return;
+    }
+    size_t rbase[KMAX];
+    float wq[KMAX];
+#pragma unroll
+    for (int q = 0; q < KMAX; ++q) {
+        const int src = m ? __ffs(m) - 1 : 0;
+        m &= m - 1;
+        rbase[q] = (size_t)__shfl_sync(0xffffffffu, row, src) * nv;
+        wq[q] = __shfl_sync(0xffffffffu, wt, src);
+    }
+    for (int c = lane; c < nv; c += 32) {
+        const uint4 xv4 = __ldg(xr + c);
+        uint4 yv4[KMAX];
+#pragma unroll
+        for (int q = 0; q < KMAX; ++q)
+            if (q < nk) yv4[q] = __ldg(Y + rbase[q] + c);
+        float acc[V];
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] = 0.0f;
+#pragma unroll
+        for (int q = 0; q < KMAX; ++q) {
+            if (q < nk) {
+                float yv[V];
+                Tr::unpack(yv4[q], yv);
+#pragma unroll
+                for (int i = 0; i < V; ++i) acc[i] = __fmaf_rn(wq[q], yv[i], acc[i]);
+            }
+        }
+        float xv[V];
+        Tr::unpack(xv4, xv);
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] = __fadd_rn(xv[i], acc[i]);
+        orow[c] = Tr::pack(acc);
+    }
+}
+
 // ---------------------------------------------------------------------------------------------
 // fp32 expert FFN on CUDA cores (small fp32 layers): one block per kept row.
 //   h = W1[e] x + b1[e]; a = SiLU(h) = h / (1 + exp(-h)); Y = W2[e] a + b2[e]
@@ -215,6 +288,13 @@ void launch_combine(int dtype, const void* x, const void* Y, const float* w, con
     const int blocks = (T + 7) / 8;
     const bool aligned = ((uintptr_t)x % 16 == 0) && ((uintptr_t)Y % 16 == 0) &&
                          ((uintptr_t)out % 16 == 0);
+    if (dtype == MOE_BF16 && aligned && d % 8 == 0 && k <= 8) {
+        combine_vec_kernel<BF16Traits, 8><<<blocks, 256, 0, s>>>(
+            (const uint4*)x, (const uint4*)Y, w, ids, slot, offsets, T, d / 8, E, k, (uint4*)out,
+            st);
+        *launches += 1;
+        return;
+    }
     if (dtype == MOE_BF16) {
         if (aligned && d % 8 == 0)
             combine_kernel<BF16Traits, true><<<blocks, 256, 0, s>>>(x, Y, w, ids, slot, offsets,

@@ -238,7 +238,6 @@ template <int BN, int EPI, bool GATHER, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
-    static_assert(!(GATHER && PAIR), "gathered A rows run on single-CTA tiles");
     using C = Cfg<BN, PAIR>;
     constexpr int S = C::kStages;
     constexpr int TM = C::kTileM;
@@ -267,7 +266,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < S; ++s) {
             // producer arrive + expected bytes; gathered rows add one arrival per A thread
-            mbar_init(full_bar(s), GATHER ? 1 + 128 : 1);
+            // (of both CTAs for a pair: the leader's threads locally, the peer's remotely)
+            mbar_init(full_bar(s), GATHER ? 1 + (PAIR ? 256 : 128) : 1);
             mbar_init(empty_bar(s), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -347,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (leader) mbar_arrive_expect_tx(full_bar(s), kTx);
                     if (PAIR) {
                         const uint32_t fb = lead(full_bar(s));
-                        tma_load_2d_pair(sA(s), &tmA, fb, kb * kBK, tc.row0);
+                        if (!GATHER) tma_load_2d_pair(sA(s), &tmA, fb, kb * kBK, tc.row0);
                         tma_load_2d_pair(sB(s), &tmB, fb, kb * kBK, brow);
                     } else {
                         if (!GATHER) tma_load_2d(sA(s), &tmA, full_bar(s), kb * kBK, tc.row0);
@@ -503,13 +503,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         // stage's full barrier when they have landed (cp.async.mbarrier.arrive.noinc), so all
         // stages can be in flight at once and no producer thread ever blocks on its own copies.
         // The MMA thread makes the landed rows visible to the tensor cores with a proxy fence.
+        // The peer CTA of a pair cannot arrive asynchronously on the leader's barrier, so each
+        // of its threads waits for its own copies with kLag stages still in flight, fences them
+        // for the tensor cores and arrives on the leader's barrier itself.
+        constexpr int kLag = S - 3 > 1 ? S - 3 : 1;
+        const bool remote = PAIR && !leader;
         const int at = threadIdx.x - 32 * (2 + kEpiWarps);   // 0..127
         const int chunk = at & 7;                             // 16-byte chunk of the row
         const int rbase = at >> 3;                            // rows rbase + 16 i
-        uint32_t it = 0;
+        uint32_t it = 0, arrived = 0;
         bool ok = true;
         for (int tile = cid; ok && tile < total; tile += ncl) {
-            const TileCoord tc = tile_coord<TM>(tile, s_mt, E, n_tiles, args, 0);
+            const TileCoord tc = tile_coord<TM>(tile, s_mt, E, n_tiles, args, (int)crank);
             const __nv_bfloat16* src[8];
             uint32_t dst_off[8];
             bool valid[8];
@@ -537,10 +542,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
                     if (valid[i]) cp_async_16(dA + dst_off[i], src[i] + kb * kBK);
-                cp_async_arrive_noinc(full_bar(s));
+                if (!remote) {
+                    cp_async_arrive_noinc(full_bar(s));
+                } else {
+                    cp_async_commit();
+                    if (it + 1 - arrived > (uint32_t)kLag) {
+                        cp_async_wait<kLag>();
+                        fence_proxy_async_smem();
+                        mbar_arrive_cluster(lead(full_bar(arrived % S)));
+                        ++arrived;
+                    }
+                }
             }
         }
         cp_async_wait<0>();
+        if (remote && ok) {
+            fence_proxy_async_smem();
+            for (; arrived < it; ++arrived) mbar_arrive_cluster(lead(full_bar(arrived % S)));
+        }
     }
 
     tc_fence_before();
@@ -707,14 +726,25 @@ cudaError_t launch_router_bn(int BN, const CUtensorMap& tmA, const CUtensorMap& 
 
 }  // namespace
 
-// Column tile for an output width: least padded work, then the wider tile.
+// Column tile for an output width: least padded work, then the wider tile.  MOE_GEMM_BN in the
+// environment (256, 192, 176 or 128) overrides the choice, for tuning runs.
 int pick_bn(int nout) {
+    static int forced = -1;
+    if (forced < 0) {
+        const char* v = getenv("MOE_GEMM_BN");
+        const int f = v ? atoi(v) : 0;
+        forced = (f == 256 || f == 192 || f == 176 || f == 128) ? f : 0;
+    }
+    if (forced > 0) return forced;
+    // Cost of a column tile ~ BN + 128: per-tile work that does not shrink with BN (A operand
+    // loads, pipeline turn-around) is about half a 256-wide tile's MMA time.  Measured on B200
+    // at d_ff = 1408: 256-wide tiles (9% padding) beat the exact 176-wide ones by 15%.
     const int cands[] = {256, 192, 176, 128};
     int best = 256;
-    long long best_pad = -1;
+    long long best_cost = -1;
     for (int bn : cands) {
-        const long long pad = (long long)((nout + bn - 1) / bn) * bn;
-        if (best_pad < 0 || pad < best_pad) { best = bn; best_pad = pad; }
+        const long long cost = (long long)((nout + bn - 1) / bn) * (bn + 128);
+        if (best_cost < 0 || cost < best_cost) { best = bn; best_cost = cost; }
     }
     return best;
 }
@@ -740,7 +770,9 @@ cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const in
                                long long max_rows, DeviceStatus* st, cudaStream_t s,
                                int* launches) {
     const int BN = pick_bn(Nout);
-    const bool pair = a_rows == nullptr && use_pair(max_rows, E);
+    // Gathered A on pairs needs the peer's rows forwarded to the leader's barrier by the copying
+    // threads themselves, which measured slower than single-CTA tiles; only when forced.
+    const bool pair = use_pair(max_rows, E) && (a_rows == nullptr || g_pair_mode == 1);
     CUtensorMap tm;
     if (!make_tmap(&tm, W, (long long)E * Nout, K, pair ? BN / 2 : BN)) return cudaErrorInvalidValue;
     GemmArgs a{};
@@ -768,7 +800,10 @@ cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const in
     if (!gather && !make_tmap(&tmA, A, (long long)a_row_limit, K, kBM))
         return cudaErrorInvalidValue;
     cudaError_t e;
-    if (gather) {
+    if (gather && pair) {
+        e = which == 0 ? launch_gemm_bn<kEpiSiLU, true, true>(BN, tmA, tm, a, max_tiles, s)
+                       : launch_gemm_bn<kEpiBias, true, true>(BN, tmA, tm, a, max_tiles, s);
+    } else if (gather) {
         e = which == 0 ? launch_gemm_bn<kEpiSiLU, true, false>(BN, tmA, tm, a, max_tiles, s)
                        : launch_gemm_bn<kEpiBias, true, false>(BN, tmA, tm, a, max_tiles, s);
     } else if (pair) {

@@ -16,6 +16,7 @@
 //   select : one block per expert; if n_e > K a 4-pass radix select on the fp32 weight bits
 //            finds the K-th largest weight, then one ordered pass with block scans assigns
 //            slots, drop flags, rowtok and the counts.
+#include <atomic>
 #include <cfloat>
 #include <cstdint>
 
@@ -246,13 +247,15 @@ __global__ void __launch_bounds__(128) scatter_chunks_kernel(const int32_t* __re
 // ---------------------------------------------------------------------------------------------
 // Capacity selection: one block per expert.
 // ---------------------------------------------------------------------------------------------
-constexpr int kSelThreads = 512;
+constexpr int kSelThreads = 1024;
+constexpr int kSelSmemKeys = 32768;   // weight keys of one expert's candidates kept on chip
 
 __global__ void __launch_bounds__(kSelThreads) select_kernel(
     const int32_t* __restrict__ cand, const int32_t* __restrict__ nrecv,
     const float* __restrict__ w, int T, int E, int k, long long K, int32_t* __restrict__ slot,
     uint8_t* __restrict__ drop, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
     int32_t* __restrict__ rowtok) {
+    extern __shared__ uint32_t s_keys[];              // [kSelSmemKeys]
     __shared__ int s_warp[32];
     __shared__ int s_hist[256];
     __shared__ uint32_t s_prefix;
@@ -295,8 +298,17 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
         return;
     }
 
-    // Radix select (most significant byte first) of the K-th largest weight bit pattern.
-    // Weights are >= +0, so their IEEE bit patterns order like the values.
+    // Weight bit patterns of the candidates (weights are >= +0, so the bits order like the
+    // values), gathered once into shared memory when they fit.
+    const bool on_chip = n <= kSelSmemKeys;
+    if (on_chip)
+        for (int i = tid; i < n; i += blockDim.x) s_keys[i] = __float_as_uint(w[list[i]]);
+    __syncthreads();
+    auto key_of = [&](int i) -> uint32_t {
+        return on_chip ? s_keys[i] : __float_as_uint(w[list[i]]);
+    };
+
+    // Radix select (most significant byte first) of the K-th largest key.
     uint32_t prefix = 0, mask = 0;
     int remaining = (int)K;
     for (int pass = 0; pass < 4; ++pass) {
@@ -304,7 +316,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
         for (int b = tid; b < 256; b += blockDim.x) s_hist[b] = 0;
         __syncthreads();
         for (int i = tid; i < n; i += blockDim.x) {
-            const uint32_t key = __float_as_uint(w[list[i]]);
+            const uint32_t key = key_of(i);
             if ((key & mask) == prefix) atomicAdd(&s_hist[(key >> shift) & 255u], 1);
         }
         __syncthreads();
@@ -350,7 +362,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
         const int i = i0 + tid;
         int p = 0;
         uint32_t key = 0;
-        if (i < n) { p = list[i]; key = __float_as_uint(w[p]); }
+        if (i < n) { p = list[i]; key = key_of(i); }
         const int is_eq = (i < n && key == tau) ? 1 : 0;
         int eq_tot;
         const int eq_rank = eq_carry + block_exclusive_scan(is_eq, s_warp, &eq_tot);
@@ -461,8 +473,17 @@ void launch_capacity_select(const int32_t* ids, const float* w, int T, int E, in
     count_chunks_kernel<<<blocks, 128, smem, s>>>(ids, T, E, k, nC, cnt, st);
     scan_chunks_kernel<<<E, 256, 0, s>>>(cnt, nC, base, nrecv);
     scatter_chunks_kernel<<<blocks, 128, smem, s>>>(ids, T, E, k, nC, base, cand);
-    select_kernel<<<E, kSelThreads, 0, s>>>(cand, nrecv, w, T, E, k, K, slot, drop, counts,
-                                            offsets, rowtok);
+    static std::atomic<uint64_t> attr_done{0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(attr_done.load() & bit)) {
+        cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSelSmemKeys * 4);
+        attr_done.fetch_or(bit);
+    }
+    select_kernel<<<E, kSelThreads, kSelSmemKeys * 4, s>>>(cand, nrecv, w, T, E, k, K, slot, drop,
+                                                            counts, offsets, rowtok);
     *launches += 4;
 }
 
