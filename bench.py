@@ -321,28 +321,53 @@ def run_cuda(args):
     ms_per_step = total_ms / K
     value = world * spec.T / (ms_per_step / 1e3)
 
-    # End to end through the C ABI with host buffers: pinned x -> device, forward, out -> host.
+    # End to end through the C ABI with host buffers, as a serving loop runs it: every step
+    # copies its x from pinned host memory to the device, runs the layer and copies its output
+    # back to pinned host memory.  Copy-in, compute and copy-out run on three streams with
+    # double-buffered device x/out, so step i's copies overlap steps i-1 and i+1.
     x_host = d["x"].cpu().pin_memory()
-    out_host = torch.empty_like(x_host).pin_memory()
+    out_host = [torch.empty_like(x_host).pin_memory() for _ in range(2)]
+    xd = [torch.empty_like(d["x"]) for _ in range(2)]
+    od = [torch.empty_like(d["x"]) for _ in range(2)]
+    s_in, s_cmp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
+    ev = lambda: torch.cuda.Event(enable_timing=False)
+    h2d_done = [ev() for _ in range(K)]
+    cmp_done = [ev() for _ in range(K)]
+    d2h_done = [ev() for _ in range(K)]
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    xd = torch.empty_like(d["x"])
-    e2e_ms = 0.0
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0.record(s_in)
     for i in range(K):
-        flush.zero_()
-        e0.record(stream)
-        xd.copy_(x_host, non_blocking=True)
-        moe.moe_forward(layer.p, xd, d["Wr"], d["br"], d["W1"], d["b1"], d["W2"], d["b2"], out,
-                        layer.ws)
-        out_host.copy_(out, non_blocking=True)
-        e1.record(stream)
-        e1.synchronize()
-        e2e_ms += e0.elapsed_time(e1)
+        b = i % 2
+        if i >= 2:
+            s_in.wait_event(cmp_done[i - 2])             # xd[b] no longer read
+        with torch.cuda.stream(s_in):
+            xd[b].copy_(x_host, non_blocking=True)
+        h2d_done[i].record(s_in)
+        s_cmp.wait_event(h2d_done[i])
+        if i >= 2:
+            s_cmp.wait_event(d2h_done[i - 2])            # od[b] already copied out
+        moe.moe_forward(layer.p, xd[b], d["Wr"], d["br"], d["W1"], d["b1"], d["W2"], d["b2"],
+                        od[b], layer.ws, stream=s_cmp)
+        cmp_done[i].record(s_cmp)
+        s_out.wait_event(cmp_done[i])
+        with torch.cuda.stream(s_out):
+            out_host[b].copy_(od[b], non_blocking=True)
+        d2h_done[i].record(s_out)
+    s_in.wait_event(d2h_done[K - 1])
+    e1.record(s_in)
+    e1.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
     if world > 1:
         t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
     e2e_value = world * spec.T / (e2e_ms / K / 1e3)
+    # The last step's output must equal the device-timed path's output (same inputs).
+    assert torch.equal(out_host[(K - 1) % 2], out.cpu()), "e2e output differs"
     assert moe.moe_get_device_status(layer.ws) == 0, "device status word reports an error"
 
     # Roofline bookkeeping (algorithmic work per launch).
@@ -396,8 +421,10 @@ def run_cuda(args):
         "clocks": clocks,
         "e2e": {"value": e2e_value, "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
-                "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size()),
-                "ms_per_step": e2e_ms / K},
+                "d2h_bytes_per_step": int(out_host[0].numel() * out_host[0].element_size()),
+                "ms_per_step": e2e_ms / K,
+                "pipeline": "copy-in / compute / copy-out streams, double-buffered device x and"
+                            " out; pinned host buffers"},
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved,
                      "peak": tensor_peak, "unit": "TFLOP/s",
                      "frac": achieved / tensor_peak if achieved else None,
