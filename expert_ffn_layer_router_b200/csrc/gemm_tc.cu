@@ -32,6 +32,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "softmax.cuh"
 
 namespace moe {
 
@@ -44,7 +45,9 @@ constexpr int kEpiWarps = 8;        // two per TMEM lane quadrant, each half of 
 constexpr int kTmemCols = 512;      // two accumulators at column 0 and 256
 constexpr int kMaxGroups = 1024;
 
-enum Epi { kEpiSiLU = 0, kEpiBias = 1, kEpiRouter = 2 };
+// kEpiRouterFused: the router epilogue also forms the softmax, the top-k and the per-chunk
+// expert counts of its tokens (all E <= 64 experts of a token sit in one thread's TMEM lane).
+enum Epi { kEpiSiLU = 0, kEpiBias = 1, kEpiRouter = 2, kEpiRouterFused = 3 };
 
 struct GemmArgs {
     const __nv_bfloat16* A;   // [*, lda] row-major
@@ -62,6 +65,11 @@ struct GemmArgs {
     void* D;                  // output
     long long ldd;            // elements
     int router_E;             // router epilogue: number of experts (columns of D)
+    int32_t* r_ids;           // fused router: [T*k] expert ids
+    float* r_w;               // fused router: [T*k] softmax weights
+    int32_t* r_cnt;           // fused router: [E][r_nC] pairs per expert and 32-token chunk
+    int r_nC;
+    int r_k;
     DeviceStatus* st;
 };
 
@@ -436,6 +444,82 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
+            } else if (EPI == kEpiRouterFused) {
+                // One thread = one token: logits of all E experts from TMEM, then the softmax in
+                // the warp router's order (lane partials of experts l, l+32, then the pairwise
+                // tree 16, 8, 4, 2, 1), the top-k by (logit desc, expert asc) and this warp's
+                // 32-token chunk histogram.
+                constexpr int Eg = BN / 3;
+                if (h == 0) {
+                    const int Er = args.router_E;
+                    int* s_cnt = reinterpret_cast<int*>(base_ptr + C::kStgOff) + (warp - 2) * 512;
+                    for (int e = lane; e < Er; e += 32) s_cnt[e] = 0;
+                    float L[Eg];
+#pragma unroll
+                    for (int c0 = 0; c0 < Eg; c0 += 16) {
+                        float hi[16], mi[16], lo[16];
+                        __syncwarp();
+                        tmem_ld16_wait(taddr + c0, hi);
+                        tmem_ld16_wait(taddr + Eg + c0, mi);
+                        tmem_ld16_wait(taddr + 2 * Eg + c0, lo);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            float v = __fadd_rn(hi[i], __fadd_rn(mi[i], lo[i]));
+                            if (args.bias && c0 + i < Er) v = __fadd_rn(v, __ldg(args.bias + c0 + i));
+                            L[c0 + i] = v;
+                        }
+                    }
+                    __syncwarp();
+                    if (lane < wrows) {
+                        const long long t = wrow0 + lane;
+                        if (args.D) {
+                            float* out = reinterpret_cast<float*>(args.D) + t * args.ldd;
+#pragma unroll
+                            for (int e = 0; e < Eg; ++e)
+                                if (e < Er) out[e] = L[e];
+                        }
+                        float m = L[0];
+#pragma unroll
+                        for (int e = 1; e < Eg; ++e)
+                            if (e < Er && L[e] > m) m = L[e];
+                        float part[32];
+#pragma unroll
+                        for (int l = 0; l < 32; ++l) {
+                            float acc = 0.0f;
+#pragma unroll
+                            for (int e = l; e < Eg; e += 32)
+                                if (e < Er) acc = __fadd_rn(acc, exp_cody_waite(__fsub_rn(L[e], m)));
+                            part[l] = acc;
+                        }
+#pragma unroll
+                        for (int hh = 16; hh >= 1; hh >>= 1)
+#pragma unroll
+                            for (int l = 0; l < hh; ++l) part[l] = __fadd_rn(part[l], part[l + hh]);
+                        const float S = part[0];
+                        uint64_t taken = 0;
+                        for (int j = 0; j < args.r_k; ++j) {
+                            int best = -1;
+                            float bl = 0.0f;
+#pragma unroll
+                            for (int e = 0; e < Eg; ++e) {
+                                if (e < Er && !((taken >> e) & 1ull) && (best < 0 || L[e] > bl)) {
+                                    best = e;
+                                    bl = L[e];
+                                }
+                            }
+                            taken |= 1ull << best;
+                            const size_t pj = (size_t)t * args.r_k + j;
+                            args.r_ids[pj] = best;
+                            args.r_w[pj] = __fdiv_rn(exp_cody_waite(__fsub_rn(bl, m)), S);
+                            atomicAdd(&s_cnt[best], 1);
+                        }
+                    }
+                    __syncwarp();
+                    const int chunk = (int)(wrow0 >> 5);
+                    if (chunk < args.r_nC)
+                        for (int e = lane; e < Er; e += 32)
+                            args.r_cnt[(size_t)e * args.r_nC + chunk] = s_cnt[e];
+                }
             } else {
                 const int n0 = tc.nt * BN;
                 const float* bias = args.bias ? args.bias + (size_t)tc.e * args.Nout + n0 : nullptr;
@@ -714,12 +798,13 @@ cudaError_t launch_gemm_bn(int BN, const CUtensorMap& tmA, const CUtensorMap& tm
     }
 }
 
+template <int EPI>
 cudaError_t launch_router_bn(int BN, const CUtensorMap& tmA, const CUtensorMap& tmB,
                              const GemmArgs& a, long long tiles, cudaStream_t s) {
     switch (BN) {
-        case 192: return launch_gemm_t<192, kEpiRouter, false, false>(tmA, tmB, a, tiles, s);
-        case 96: return launch_gemm_t<96, kEpiRouter, false, false>(tmA, tmB, a, tiles, s);
-        case 48: return launch_gemm_t<48, kEpiRouter, false, false>(tmA, tmB, a, tiles, s);
+        case 192: return launch_gemm_t<192, EPI, false, false>(tmA, tmB, a, tiles, s);
+        case 96: return launch_gemm_t<96, EPI, false, false>(tmA, tmB, a, tiles, s);
+        case 48: return launch_gemm_t<48, EPI, false, false>(tmA, tmB, a, tiles, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -825,10 +910,11 @@ size_t router_split_bytes(int d, int E) {
 
 cudaError_t launch_router_gemm(const void* x, int T, int d, const float* Wr, const float* br,
                                int E, void* split_buf, float* logits, DeviceStatus* st,
-                               cudaStream_t s, int* launches) {
+                               cudaStream_t s, int* launches, const RouterFused* fused) {
     const int Eg = router_group(E);
     const int ntl = (E + Eg - 1) / Eg;
     const int BN = 3 * Eg;
+    const bool fuse = fused != nullptr && ntl == 1;
     router_split_kernel<<<148 * 4, 256, 0, s>>>(Wr, d, E, Eg, ntl,
                                                 reinterpret_cast<__nv_bfloat16*>(split_buf));
     *launches += 1;
@@ -851,12 +937,22 @@ cudaError_t launch_router_gemm(const void* x, int T, int d, const float* Wr, con
     a.ldd = E;
     a.router_E = E;
     a.st = st;
+    if (fuse) {
+        a.r_ids = fused->ids;
+        a.r_w = fused->w;
+        a.r_cnt = fused->cnt;
+        a.r_nC = fused->nC;
+        a.r_k = fused->k;
+    }
     const long long tiles = (long long)((T + kBM - 1) / kBM) * ntl;
     CUtensorMap tmA;
     if (!make_tmap(&tmA, x, (long long)T, d, kBM)) return cudaErrorInvalidValue;
-    cudaError_t e = launch_router_bn(BN, tmA, tm, a, tiles, s);
+    cudaError_t e = fuse ? launch_router_bn<kEpiRouterFused>(BN, tmA, tm, a, tiles, s)
+                         : launch_router_bn<kEpiRouter>(BN, tmA, tm, a, tiles, s);
     if (e == cudaSuccess) *launches += 1;
     return e;
 }
+
+bool router_can_fuse(int E) { return E <= 64; }
 
 }  // namespace moe

@@ -14,10 +14,12 @@ struct DeviceStatus;
 void launch_route_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
                        cudaStream_t s);
 int chunk_count(int T);
+// counts_ready: cnt already holds the per-chunk counts (fused router), skip the count pass.
 void launch_capacity_select(const int32_t* ids, const float* w, int T, int E, int k, long long K,
                             int32_t* cnt, int32_t* base, int32_t* nrecv, int32_t* cand,
                             int32_t* slot, uint8_t* drop, int32_t* counts, int32_t* offsets,
-                            int32_t* rowtok, DeviceStatus* st, cudaStream_t s, int* launches);
+                            int32_t* rowtok, DeviceStatus* st, cudaStream_t s, int* launches,
+                            bool counts_ready = false);
 void launch_dispatch(const int32_t* ids, const int32_t* slot, int T, int E, int k,
                      int32_t* kept_tmp, int32_t* offsets, int32_t* rowtok, DeviceStatus* st,
                      cudaStream_t s, int* launches);
@@ -46,8 +48,18 @@ cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const in
                                const void* W, const float* bias, void* D, long long ldd,
                                long long max_rows, DeviceStatus* st, cudaStream_t s,
                                int* launches);
+// Outputs of the fused router epilogue (softmax, top-k and per-chunk counts of each token).
+struct RouterFused {
+    int32_t* ids;
+    float* w;
+    int32_t* cnt;     // [E][nC]
+    int nC;
+    int k;
+};
+bool router_can_fuse(int E);
+// logits may be null when fused (logits are then not stored).  fused == null: logits only.
 cudaError_t launch_router_gemm(const void* x, int T, int d, const float* Wr, const float* br,
                                int E, void* split_buf, float* logits, DeviceStatus* st,
-                               cudaStream_t s, int* launches);
+                               cudaStream_t s, int* launches, const RouterFused* fused);
 
 }  // namespace moe

@@ -284,9 +284,14 @@ moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, con
     void* Y = at<void>(ws, q.Y);
 
     stage_mark(0, s);
+    // bf16 with E <= 64: the logits GEMM's epilogue also forms the softmax, top-k and per-chunk
+    // counts (one fused launch instead of logits + router + count kernels).
+    const bool fused = p->dtype == MOE_BF16 && moe::router_can_fuse(p->E);
     if (p->dtype == MOE_BF16) {
+        moe::RouterFused rf{ids, w, at<int32_t>(ws, q.cnt), moe::chunk_count(p->T), p->k};
         if (moe::launch_router_gemm(x, p->T, p->d_model, Wr, br, p->E, at<void>(ws, q.split),
-                                    logits, st, s, &launches) != cudaSuccess)
+                                    fused ? logits_out : logits, st, s, &launches,
+                                    fused ? &rf : nullptr) != cudaSuccess)
             return MOE_ERR_CUDA;
     } else {
         moe::launch_logits_f32((const float*)x, Wr, br, p->T, p->d_model, p->E, logits, s,
@@ -294,13 +299,15 @@ moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, con
     }
     stage_mark(1, s);
     const long long K = capacity_of(p);
-    moe::launch_route_topk(logits, p->T, p->E, p->k, ids, w, s);
-    launches += 1;
+    if (!fused) {
+        moe::launch_route_topk(logits, p->T, p->E, p->k, ids, w, s);
+        launches += 1;
+    }
     stage_mark(2, s);
     moe::launch_capacity_select(ids, w, p->T, p->E, p->k, K, at<int32_t>(ws, q.cnt),
                                 at<int32_t>(ws, q.base), at<int32_t>(ws, q.nrecv),
                                 at<int32_t>(ws, q.cand), slot, drop, counts, offsets, rowtok, st,
-                                s, &launches);
+                                s, &launches, fused);
     stage_mark(3, s);
     const long long R = max_rows_of(p, K);
     if (R > 0 && p->dtype == MOE_BF16) {

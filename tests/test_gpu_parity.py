@@ -270,3 +270,30 @@ def test_unsupported_and_invalid():
         moe.MoELayer(16, 100, 64, 4, 2, 1.0, "bf16").forward(
             *[torch.zeros(1, device="cuda")] * 7)
     assert ei.value.status in (1, 2)
+
+
+# ------------------------------------------------------------------------------------------
+# Fused router: with bf16 and E <= 64 the logits GEMM's epilogue also forms the softmax, the
+# top-k and the per-chunk counts.  Its routing must equal moe_route's on the same logits bit for
+# bit (moe_route itself is bit-exact against the oracle above), so the chain reaches the oracle
+# without feeding it anything computed on the GPU.
+# ------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("T,d,E,k,C", [(3000, 128, 64, 6, 1.0), (1000, 256, 8, 2, 1.25),
+                                       (777, 64, 33, 4, 0.75), (200, 64, 16, 8, math.inf),
+                                       (5000, 64, 64, 6, 0.5), (129, 64, 1, 1, 1.0)])
+def test_fused_router_matches_route(T, d, E, k, C):
+    moe = _moe()
+    spec = inputs.LayerSpec("fused", T, d, 64, E, k, C, "bf16", router="normal",
+                            router_bias=0.5)
+    L = inputs.make_layer(spec, seed=E + T)
+    layer = moe.MoELayer(T, d, 64, E, k, C, "bf16")
+    args = [to_dev(L[n]) for n in ("x", "Wr", "br", "W1", "b1", "W2", "b2")]
+    _, rt = layer.forward(*args, want_routing=True)
+    r = layer.route(rt["logits_out"])
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(layer.ws) == 0
+    assert torch.equal(rt["ids_out"], r["ids"])
+    assert torch.equal(rt["w_out"].view(torch.int32), r["w"].view(torch.int32))
+    assert torch.equal(rt["slot_out"], r["slot"])
+    assert torch.equal(rt["drop_out"], r["drop"])
+    assert torch.equal(rt["counts_out"], r["counts"])
