@@ -75,13 +75,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // as another thread has recorded an error, and then returns false after recording a timeout.
 template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, DeviceStatus* st,
-                                          int where) {
+                                          int where, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait<kCluster>(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     while (true) {
         if (mbar_try_wait<kCluster>(bar, parity)) return true;
         if (*reinterpret_cast<volatile int32_t*>(&st->code) != 0) return false;
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (global_ns() - t0 > limit_ns) {
             report(st, MOE_DEV_TIMEOUT, where);
             return false;
         }

@@ -70,6 +70,7 @@ struct GemmArgs {
     int32_t* r_cnt;           // fused router: [E][r_nC] pairs per expert and 32-token chunk
     int r_nC;
     int r_k;
+    unsigned r_flags;
     DeviceStatus* st;
 };
 
@@ -497,6 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int l = 0; l < hh; ++l) part[l] = __fadd_rn(part[l], part[l + hh]);
                         const float S = part[0];
                         uint64_t taken = 0;
+                        float wsum = 0.0f;
                         for (int j = 0; j < args.r_k; ++j) {
                             int best = -1;
                             float bl = 0.0f;
@@ -509,10 +511,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                             taken |= 1ull << best;
                             const size_t pj = (size_t)t * args.r_k + j;
+                            const float wj = __fdiv_rn(exp_cody_waite(__fsub_rn(bl, m)), S);
                             args.r_ids[pj] = best;
-                            args.r_w[pj] = __fdiv_rn(exp_cody_waite(__fsub_rn(bl, m)), S);
+                            args.r_w[pj] = wj;
+                            wsum = __fadd_rn(wsum, wj);
                             atomicAdd(&s_cnt[best], 1);
                         }
+                        if (args.r_flags & MOE_FLAG_RENORMALIZE)
+                            for (int j = 0; j < args.r_k; ++j) {
+                                const size_t pj = (size_t)t * args.r_k + j;
+                                args.r_w[pj] = __fdiv_rn(args.r_w[pj], wsum);
+                            }
                     }
                     __syncwarp();
                     const int chunk = (int)(wrow0 >> 5);
@@ -943,6 +952,7 @@ cudaError_t launch_router_gemm(const void* x, int T, int d, const float* Wr, con
         a.r_cnt = fused->cnt;
         a.r_nC = fused->nC;
         a.r_k = fused->k;
+        a.r_flags = fused->flags;
     }
     const long long tiles = (long long)((T + kBM - 1) / kBM) * ntl;
     CUtensorMap tmA;

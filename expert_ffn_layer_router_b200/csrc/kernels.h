@@ -11,15 +11,24 @@ namespace moe {
 struct DeviceStatus;
 
 // route.cu
+// flags: MOE_FLAG_RENORMALIZE divides each token's k weights by their sum.
 void launch_route_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
-                       cudaStream_t s);
+                       cudaStream_t s, unsigned flags);
 int chunk_count(int T);
 // counts_ready: cnt already holds the per-chunk counts (fused router), skip the count pass.
+// flags: MOE_FLAG_ARRIVAL_ORDER keeps an overflowing expert's first K pairs in token order.
 void launch_capacity_select(const int32_t* ids, const float* w, int T, int E, int k, long long K,
                             int32_t* cnt, int32_t* base, int32_t* nrecv, int32_t* cand,
                             int32_t* slot, uint8_t* drop, int32_t* counts, int32_t* offsets,
                             int32_t* rowtok, DeviceStatus* st, cudaStream_t s, int* launches,
-                            bool counts_ready = false);
+                            bool counts_ready, unsigned flags);
+// Small batches (T*k <= 1024): the whole capacity selection in one single-block launch.
+bool dispatch_small_fits(int T, int k);
+void launch_dispatch_small(const int32_t* ids, const float* w, int T, int E, int k, long long K,
+                           unsigned flags, int32_t* slot, uint8_t* drop, int32_t* counts,
+                           int32_t* offsets, int32_t* rowtok, DeviceStatus* st, cudaStream_t s,
+                           int* launches);
+void launch_wait_timeout_selftest(DeviceStatus* st, long long limit_ns, cudaStream_t s);
 void launch_dispatch(const int32_t* ids, const int32_t* slot, int T, int E, int k,
                      int32_t* kept_tmp, int32_t* offsets, int32_t* rowtok, DeviceStatus* st,
                      cudaStream_t s, int* launches);
@@ -55,6 +64,7 @@ struct RouterFused {
     int32_t* cnt;     // [E][nC]
     int nC;
     int k;
+    unsigned flags;   // MOE_FLAG_RENORMALIZE honoured
 };
 bool router_can_fuse(int E);
 // logits may be null when fused (logits are then not stored).  fused == null: logits only.

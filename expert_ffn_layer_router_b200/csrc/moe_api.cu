@@ -31,7 +31,7 @@ bool bad_problem(const moe_problem* p) {
     if (p->k < 1 || p->k > p->E || p->k > 32) return true;
     if (std::isnan(p->capacity_factor) || p->capacity_factor < 0.0f) return true;
     if (p->dtype != MOE_F32 && p->dtype != MOE_BF16) return true;
-    if (p->flags != 0) return true;
+    if (p->flags & ~(MOE_FLAG_RENORMALIZE | MOE_FLAG_ARRIVAL_ORDER)) return true;
     if ((long long)p->T * p->k > 0x7fffffffLL) return true;
     if ((long long)p->T * p->E > 0x7fffffffLL) return true;
     return false;
@@ -129,12 +129,16 @@ void route_steps(const moe_problem* p, const float* logits, int32_t* ids, float*
                  int32_t* rowtok, void* ws, const Plan& q, cudaStream_t s, int* launches) {
     moe::DeviceStatus* st = at<moe::DeviceStatus>(ws, q.status);
     const long long K = capacity_of(p);
-    moe::launch_route_topk(logits, p->T, p->E, p->k, ids, w, s);
+    moe::launch_route_topk(logits, p->T, p->E, p->k, ids, w, s, p->flags);
     *launches += 1;
-    moe::launch_capacity_select(ids, w, p->T, p->E, p->k, K, at<int32_t>(ws, q.cnt),
-                                at<int32_t>(ws, q.base), at<int32_t>(ws, q.nrecv),
-                                at<int32_t>(ws, q.cand), slot, drop, counts, offsets, rowtok, st,
-                                s, launches);
+    if (moe::dispatch_small_fits(p->T, p->k))
+        moe::launch_dispatch_small(ids, w, p->T, p->E, p->k, K, p->flags, slot, drop, counts,
+                                   offsets, rowtok, st, s, launches);
+    else
+        moe::launch_capacity_select(ids, w, p->T, p->E, p->k, K, at<int32_t>(ws, q.cnt),
+                                    at<int32_t>(ws, q.base), at<int32_t>(ws, q.nrecv),
+                                    at<int32_t>(ws, q.cand), slot, drop, counts, offsets, rowtok,
+                                    st, s, launches, false, p->flags);
 }
 
 moe_status ffn_steps(const moe_problem* p, const void* x, const int32_t* offsets,
@@ -288,7 +292,8 @@ moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, con
     // counts (one fused launch instead of logits + router + count kernels).
     const bool fused = p->dtype == MOE_BF16 && moe::router_can_fuse(p->E);
     if (p->dtype == MOE_BF16) {
-        moe::RouterFused rf{ids, w, at<int32_t>(ws, q.cnt), moe::chunk_count(p->T), p->k};
+        moe::RouterFused rf{ids, w, at<int32_t>(ws, q.cnt), moe::chunk_count(p->T), p->k,
+                            p->flags};
         if (moe::launch_router_gemm(x, p->T, p->d_model, Wr, br, p->E, at<void>(ws, q.split),
                                     fused ? logits_out : logits, st, s, &launches,
                                     fused ? &rf : nullptr) != cudaSuccess)
@@ -300,14 +305,18 @@ moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, con
     stage_mark(1, s);
     const long long K = capacity_of(p);
     if (!fused) {
-        moe::launch_route_topk(logits, p->T, p->E, p->k, ids, w, s);
+        moe::launch_route_topk(logits, p->T, p->E, p->k, ids, w, s, p->flags);
         launches += 1;
     }
     stage_mark(2, s);
-    moe::launch_capacity_select(ids, w, p->T, p->E, p->k, K, at<int32_t>(ws, q.cnt),
-                                at<int32_t>(ws, q.base), at<int32_t>(ws, q.nrecv),
-                                at<int32_t>(ws, q.cand), slot, drop, counts, offsets, rowtok, st,
-                                s, &launches, fused);
+    if (moe::dispatch_small_fits(p->T, p->k))
+        moe::launch_dispatch_small(ids, w, p->T, p->E, p->k, K, p->flags, slot, drop, counts,
+                                   offsets, rowtok, st, s, &launches);
+    else
+        moe::launch_capacity_select(ids, w, p->T, p->E, p->k, K, at<int32_t>(ws, q.cnt),
+                                    at<int32_t>(ws, q.base), at<int32_t>(ws, q.nrecv),
+                                    at<int32_t>(ws, q.cand), slot, drop, counts, offsets, rowtok,
+                                    st, s, &launches, fused, p->flags);
     stage_mark(3, s);
     const long long R = max_rows_of(p, K);
     if (R > 0 && p->dtype == MOE_BF16) {
@@ -353,6 +362,15 @@ moe_status moe_reset_device_status(void* ws, size_t ws_bytes, void* stream) {
 }
 
 int32_t moe_last_launch_count(void) { return g_last_launches; }
+
+moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, int32_t limit_us, void* stream) {
+    if (!ws || ws_bytes < sizeof(moe::DeviceStatus) || limit_us < 1 || limit_us > 10000000)
+        return MOE_ERR_INVALID_ARG;
+    cudaGetLastError();
+    moe::launch_wait_timeout_selftest(reinterpret_cast<moe::DeviceStatus*>(ws),
+                                      (long long)limit_us * 1000, (cudaStream_t)stream);
+    return finish(1);
+}
 
 moe_status moe_set_stage_events(void* const* events, int32_t n) {
     if (!events || n == 0) {
@@ -468,11 +486,12 @@ extern "C" moe_status moe_route_static(const moe_problem* p, const float* logits
     moe::DeviceStatus* st = at<moe::DeviceStatus>(scratch, 0);
     cudaMemsetAsync(st, 0, sizeof(moe::DeviceStatus), s);
     int launches = 0;
-    moe::launch_route_topk(logits, p->T, p->E, p->k, ids, w, s);
+    moe::launch_route_topk(logits, p->T, p->E, p->k, ids, w, s, p->flags);
     launches += 1;
     moe::launch_capacity_select(ids, w, p->T, p->E, p->k, capacity_of(p),
                                 at<int32_t>(scratch, o_cnt), at<int32_t>(scratch, o_base),
                                 at<int32_t>(scratch, o_nrecv), at<int32_t>(scratch, o_cand),
-                                slot, drop, counts, nullptr, nullptr, st, s, &launches);
+                                slot, drop, counts, nullptr, nullptr, st, s, &launches, false,
+                                p->flags);
     return finish(launches);
 }

@@ -36,7 +36,7 @@ constexpr unsigned kFull = 0xffffffffu;
 template <int EPL>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T,
                                                          int E, int k, int32_t* __restrict__ ids,
-                                                         float* __restrict__ w) {
+                                                         float* __restrict__ w, unsigned flags) {
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T) return;
@@ -89,6 +89,12 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
             my_id = we;
             my_w = __fdiv_rn(wu, S);
         }
+    }
+    if (flags & MOE_FLAG_RENORMALIZE) {
+        // Sum of the k weights in j order, then one division each.
+        float sum = 0.0f;
+        for (int j = 0; j < k; ++j) sum = __fadd_rn(sum, __shfl_sync(kFull, my_w, j));
+        my_w = __fdiv_rn(my_w, sum);
     }
     if (lane < k) {
         ids[(size_t)t * k + lane] = my_id;
@@ -214,7 +220,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     const int32_t* __restrict__ cand, const int32_t* __restrict__ nrecv,
     const float* __restrict__ w, int T, int E, int k, long long K, int32_t* __restrict__ slot,
     uint8_t* __restrict__ drop, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-    int32_t* __restrict__ rowtok) {
+    int32_t* __restrict__ rowtok, unsigned flags) {
     extern __shared__ uint32_t s_keys[];              // [kSelSmemKeys]
     __shared__ int s_warp[32];
     __shared__ int s_hist[256];
@@ -248,12 +254,14 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
         }
         return;
     }
-    if (n <= K) {
+    if (n <= K || (flags & MOE_FLAG_ARRIVAL_ORDER)) {
+        // Everything fits, or arrival order: the first K candidates (ascending token) get in.
         for (int i = tid; i < n; i += blockDim.x) {
             const int p = list[i];
-            slot[p] = i;
-            drop[p] = 0;
-            if (rowtok) rowtok[off + i] = p / k;
+            const bool keep = i < K;
+            slot[p] = keep ? i : -1;
+            drop[p] = keep ? 0 : 1;
+            if (keep && rowtok) rowtok[off + i] = p / k;
         }
         return;
     }
@@ -340,6 +348,114 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
 }
 
 // ---------------------------------------------------------------------------------------------
+// Small batches (T*k <= kSmallPairs): counting, capacity selection, slots, offsets and the row
+// map in one block, one launch.  Same results as the chunked pipeline above: candidates of an
+// expert are kept in ascending token order (warp-serial stable placement), an overflowing
+// expert keeps its K pairs of largest (weight, then lower token) -- or its first K with
+// MOE_FLAG_ARRIVAL_ORDER -- and slots rank the kept tokens in ascending token order.
+// ---------------------------------------------------------------------------------------------
+constexpr int kSmallPairs = 1024;
+
+__global__ void __launch_bounds__(1024) dispatch_small_kernel(
+    const int32_t* __restrict__ ids, const float* __restrict__ w, int T, int E, int k,
+    long long K, unsigned flags, int32_t* __restrict__ slot, uint8_t* __restrict__ drop,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ rowtok,
+    DeviceStatus* st) {
+    extern __shared__ int32_t sm[];
+    __shared__ int s_warp[32];
+    const int P = T * k;
+    int32_t* cnt = sm;                 // [E]
+    int32_t* start = cnt + E;          // [E + 1]
+    int32_t* run = start + E + 1;      // [E]
+    int32_t* koff = run + E;           // [E + 1] kept offsets
+    int32_t* list = koff + E + 1;      // [P] pair index, grouped by expert, ascending token
+    int32_t* lexp = list + P;          // [P] expert of each list position
+    uint8_t* keep = reinterpret_cast<uint8_t*>(lexp + P);   // [P]
+    const int tid = threadIdx.x;
+    for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
+    __syncthreads();
+    for (int p = tid; p < P; p += blockDim.x) {
+        const int e = ids[p];
+        if ((unsigned)e < (unsigned)E) atomicAdd(&cnt[e], 1);
+        else report(st, MOE_DEV_BAD_INDEX, 111);
+    }
+    __syncthreads();
+    // start = exclusive prefix of received counts, koff = of kept counts.
+    int carry = 0, kcarry = 0;
+    for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+        const int e = e0 + tid;
+        const int v = e < E ? cnt[e] : 0;
+        const int kv = e < E ? (int)min((long long)v, K) : 0;
+        int tot, ktot;
+        const int ex = block_exclusive_scan(v, s_warp, &tot);
+        const int kex = block_exclusive_scan(kv, s_warp, &ktot);
+        if (e < E) { start[e] = carry + ex; run[e] = carry + ex; koff[e] = kcarry + kex; }
+        carry += tot;
+        kcarry += ktot;
+    }
+    if (tid == 0) { start[E] = carry; koff[E] = kcarry; }
+    __syncthreads();
+    if (tid < 32) {                                   // stable placement, 32 pairs at a time
+        for (int pb = 0; pb < P; pb += 32) {
+            const int p = pb + tid;
+            int e = p < P ? ids[p] : -1;
+            if ((unsigned)e >= (unsigned)E) e = -1;
+            const unsigned peers = __match_any_sync(kFull, e);
+            const int rank = __popc(peers & ((1u << tid) - 1u));
+            const int pos = e >= 0 ? run[e] + rank : 0;
+            __syncwarp();
+            if (e >= 0) {
+                list[pos] = p;
+                lexp[pos] = e;
+                if (tid == __ffs(peers) - 1) run[e] = pos + __popc(peers);
+            }
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+    const bool arrival = (flags & MOE_FLAG_ARRIVAL_ORDER) != 0;
+    for (int i = tid; i < carry; i += blockDim.x) {
+        const int e = lexp[i];
+        const int b0 = start[e], n = start[e + 1] - b0, pos = i - b0;
+        bool kp;
+        if (n <= K || arrival) {
+            kp = pos < K;
+        } else {
+            const int p = list[i];
+            const float wi = w[p];
+            int rank = 0;
+            for (int j = b0; j < b0 + n; ++j) {
+                const float wj = w[list[j]];
+                rank += (wj > wi || (wj == wi && j < i)) ? 1 : 0;
+            }
+            kp = rank < K;
+        }
+        keep[i] = kp ? 1 : 0;
+    }
+    __syncthreads();
+    for (int i = tid; i < carry; i += blockDim.x) {
+        const int e = lexp[i];
+        const int b0 = start[e];
+        const int p = list[i];
+        if (keep[i]) {
+            int s = 0;
+            for (int j = b0; j < i; ++j) s += keep[j];
+            slot[p] = s;
+            drop[p] = 0;
+            if (rowtok) rowtok[koff[e] + s] = p / k;
+        } else {
+            slot[p] = -1;
+            drop[p] = 1;
+        }
+    }
+    for (int e = tid; e < E; e += blockDim.x) {
+        if (counts) { counts[e] = cnt[e]; counts[E + e] = koff[e + 1] - koff[e]; }
+        if (offsets) offsets[e] = koff[e];
+    }
+    if (tid == 0 && offsets) offsets[E] = koff[E];
+}
+
+// ---------------------------------------------------------------------------------------------
 // Dispatch from a given routing (moe_dispatch).
 // ---------------------------------------------------------------------------------------------
 __global__ void kept_count_kernel(const int32_t* __restrict__ ids,
@@ -403,31 +519,61 @@ __global__ void permute_rows_kernel(const V* __restrict__ x, const int32_t* __re
 
 template <int EPL>
 void launch_route_t(const float* logits, int T, int E, int k, int32_t* ids, float* w,
-                    cudaStream_t s) {
+                    cudaStream_t s, unsigned flags) {
     const int blocks = (T + 7) / 8;
-    route_topk_kernel<EPL><<<blocks, 256, 0, s>>>(logits, T, E, k, ids, w);
+    route_topk_kernel<EPL><<<blocks, 256, 0, s>>>(logits, T, E, k, ids, w, flags);
 }
 
 }  // namespace
 
 void launch_route_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
-                       cudaStream_t s) {
+                       cudaStream_t s, unsigned flags) {
     const int epl = (E + 31) / 32;
-    if (epl <= 1) launch_route_t<1>(logits, T, E, k, ids, w, s);
-    else if (epl <= 2) launch_route_t<2>(logits, T, E, k, ids, w, s);
-    else if (epl <= 4) launch_route_t<4>(logits, T, E, k, ids, w, s);
-    else if (epl <= 8) launch_route_t<8>(logits, T, E, k, ids, w, s);
-    else if (epl <= 16) launch_route_t<16>(logits, T, E, k, ids, w, s);
-    else launch_route_t<32>(logits, T, E, k, ids, w, s);
+    if (epl <= 1) launch_route_t<1>(logits, T, E, k, ids, w, s, flags);
+    else if (epl <= 2) launch_route_t<2>(logits, T, E, k, ids, w, s, flags);
+    else if (epl <= 4) launch_route_t<4>(logits, T, E, k, ids, w, s, flags);
+    else if (epl <= 8) launch_route_t<8>(logits, T, E, k, ids, w, s, flags);
+    else if (epl <= 16) launch_route_t<16>(logits, T, E, k, ids, w, s, flags);
+    else launch_route_t<32>(logits, T, E, k, ids, w, s, flags);
 }
 
 int chunk_count(int T) { return (T + kChunk - 1) / kChunk; }
+
+bool dispatch_small_fits(int T, int k) { return (long long)T * k <= kSmallPairs; }
+
+namespace {
+// Failure-detection self-test: waits on an mbarrier that nothing arrives on, with the same
+// bounded wait the pipelines use; the wait gives up and records MOE_DEV_TIMEOUT.
+__global__ void wait_timeout_selftest_kernel(DeviceStatus* st, unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = smem_u32(&bar);
+    if (threadIdx.x == 0) mbar_init(b, 1);
+    __syncthreads();
+    if (threadIdx.x == 0) (void)mbar_wait(b, 0, st, 901, limit_ns);
+    __syncthreads();
+}
+}  // namespace
+
+void launch_wait_timeout_selftest(DeviceStatus* st, long long limit_ns, cudaStream_t s) {
+    wait_timeout_selftest_kernel<<<1, 32, 0, s>>>(st, (unsigned long long)limit_ns);
+}
+
+void launch_dispatch_small(const int32_t* ids, const float* w, int T, int E, int k, long long K,
+                           unsigned flags, int32_t* slot, uint8_t* drop, int32_t* counts,
+                           int32_t* offsets, int32_t* rowtok, DeviceStatus* st, cudaStream_t s,
+                           int* launches) {
+    const int P = T * k;
+    const size_t smem = sizeof(int32_t) * (4 * (size_t)E + 2 + 2 * (size_t)P) + (size_t)P;
+    dispatch_small_kernel<<<1, 1024, smem, s>>>(ids, w, T, E, k, K, flags, slot, drop, counts,
+                                               offsets, rowtok, st);
+    *launches += 1;
+}
 
 void launch_capacity_select(const int32_t* ids, const float* w, int T, int E, int k, long long K,
                             int32_t* cnt, int32_t* base, int32_t* nrecv, int32_t* cand,
                             int32_t* slot, uint8_t* drop, int32_t* counts, int32_t* offsets,
                             int32_t* rowtok, DeviceStatus* st, cudaStream_t s, int* launches,
-                            bool counts_ready) {
+                            bool counts_ready, unsigned flags) {
     const int nC = chunk_count(T);
     const int blocks = (nC + 3) / 4;
     const size_t smem = (size_t)4 * E * sizeof(int32_t);
@@ -447,7 +593,7 @@ void launch_capacity_select(const int32_t* ids, const float* w, int T, int E, in
         attr_done.fetch_or(bit);
     }
     select_kernel<<<E, kSelThreads, kSelSmemKeys * 4, s>>>(cand, nrecv, w, T, E, k, K, slot, drop,
-                                                            counts, offsets, rowtok);
+                                                            counts, offsets, rowtok, flags);
     *launches += 3;
 }
 

@@ -17,6 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 MOE_F32, MOE_BF16 = 0, 1
+FLAG_RENORMALIZE, FLAG_ARRIVAL_ORDER = 1, 2
 MOE_OK = 0
 DEV_OK, DEV_TIMEOUT, DEV_BAD_INDEX = 0, 1, 2
 
@@ -53,6 +54,7 @@ def _load():
         "moe_reset_device_status": [vp, sz, vp],
         "moe_set_stage_events": [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32],
         "moe_route_static": [P, vp, vp, vp, vp, vp, vp, vp],
+        "moe_selftest_wait_timeout": [vp, sz, ctypes.c_int32, vp],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -70,7 +72,7 @@ _lib = _load()
 EXPORTS = ("moe_capacity", "moe_workspace_size", "moe_route", "moe_dispatch", "moe_expert_ffn",
            "moe_combine", "moe_forward", "moe_get_device_status", "moe_reset_device_status",
            "moe_last_launch_count", "moe_status_string", "moe_set_stage_events",
-           "moe_route_static")
+           "moe_route_static", "moe_selftest_wait_timeout")
 
 STAGE_EVENTS = 7
 STAGE_NAMES = ("router_logits", "route_topk", "capacity_dispatch", "expert_gemm1",
@@ -104,13 +106,13 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
 
 
-def problem(T, d_model, d_ff, E, k, capacity_factor, dtype) -> Problem:
+def problem(T, d_model, d_ff, E, k, capacity_factor, dtype, flags=0) -> Problem:
     if isinstance(dtype, str):
         dtype = {"f32": MOE_F32, "bf16": MOE_BF16}[dtype]
     elif isinstance(dtype, torch.dtype):
         dtype = MOE_BF16 if dtype == torch.bfloat16 else MOE_F32
     return Problem(int(T), int(d_model), int(d_ff), int(E), int(k), float(capacity_factor),
-                   int(dtype), 0)
+                   int(dtype), int(flags))
 
 
 def moe_capacity(p: Problem) -> int:
@@ -170,6 +172,11 @@ def moe_reset_device_status(ws, stream=None):
                                         _stream(stream)), "moe_reset_device_status")
 
 
+def moe_selftest_wait_timeout(ws, limit_us, stream=None):
+    _check(_lib.moe_selftest_wait_timeout(_ptr(ws), ws.numel() * ws.element_size(), int(limit_us),
+                                          _stream(stream)), "moe_selftest_wait_timeout")
+
+
 def moe_last_launch_count() -> int:
     return int(_lib.moe_last_launch_count())
 
@@ -190,8 +197,8 @@ class MoELayer:
     """Holds a problem description and a workspace; calls the C ABI on torch tensors."""
 
     def __init__(self, T, d_model, d_ff, E, k, capacity_factor=math.inf, dtype="bf16",
-                 device="cuda"):
-        self.p = problem(T, d_model, d_ff, E, k, capacity_factor, dtype)
+                 device="cuda", flags=0):
+        self.p = problem(T, d_model, d_ff, E, k, capacity_factor, dtype, flags)
         self.K = moe_capacity(self.p)
         self.device = torch.device(device)
         nbytes = moe_workspace_size(self.p)

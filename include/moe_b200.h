@@ -72,8 +72,19 @@ typedef struct {
     int32_t k;                /* experts per token, 1..min(E, 32) */
     float capacity_factor;    /* C >= 0; +INFINITY = dropless (K = T) */
     int32_t dtype;            /* moe_dtype */
-    uint32_t flags;           /* reserved, must be 0 */
+    uint32_t flags;           /* MOE_FLAG_* below; other bits must be 0 */
 } moe_problem;
+
+/* Routing-policy variants (flags of moe_problem).  Default (0): softmax weights over all E,
+ * not renormalised; an overflowing expert keeps its K highest-weight pairs.
+ *   MOE_FLAG_RENORMALIZE: each token's k weights are divided by their sum (formed in fp32 over
+ *     j = 0..k-1, one correctly rounded division each); the renormalised weights are the ones
+ *     reported, used for drop priority and in the combine.
+ *   MOE_FLAG_ARRIVAL_ORDER: an overflowing expert keeps the first K pairs in token order, the
+ *     reading of "Some Tokens Do Not Get In", "Past the edge" (tokens are assigned in order and
+ *     the next one does not get in once the buffer is full), instead of the highest weights. */
+#define MOE_FLAG_RENORMALIZE 1u
+#define MOE_FLAG_ARRIVAL_ORDER 2u
 
 /* Host only.  Per-expert capacity K = min(T, floor(C * T * k / E)) evaluated in double
  * (worked example, capacity paragraph; generalised to k slots per token as in "Some Tokens Do
@@ -159,6 +170,13 @@ moe_status moe_set_stage_events(void* const* events, int32_t n);
  *   allocated, and no allocating routine is called. */
 moe_status moe_route_static(const moe_problem* p, const float* logits, int32_t* ids, float* w,
                             int32_t* slot, uint8_t* drop, int32_t* counts, void* stream);
+
+/* Failure-detection self-test: launches one kernel that waits on a pipeline barrier nothing
+ * ever arrives on, using the same bounded wait as the layer's kernels but with a limit of
+ * `limit_us` microseconds (1..10^7).  The wait gives up, records MOE_DEV_TIMEOUT in the status
+ * word of `ws` and the kernel returns; the GPU context stays usable.  Asynchronous on `stream`;
+ * read the result with moe_get_device_status. */
+moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, int32_t limit_us, void* stream);
 
 /* Reads the device status word of `ws` (synchronises `stream`). */
 moe_status moe_get_device_status(const void* ws, size_t ws_bytes, void* stream, int32_t* code);

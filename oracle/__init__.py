@@ -38,7 +38,7 @@ def lib():
         L.oracle_logits.argtypes = [ctypes.c_int] * 4 + [_vp, _f32p, _vp, _f32p, ctypes.c_int]
         L.oracle_route.restype = ctypes.c_int
         L.oracle_route.argtypes = [ctypes.c_int] * 3 + [ctypes.c_longlong, _f32p, _i32p, _f32p,
-                                                        _i32p, _u8p, _i32p]
+                                                        _i32p, _u8p, _i32p, ctypes.c_int]
         L.oracle_dispatch.restype = ctypes.c_int
         L.oracle_dispatch.argtypes = [ctypes.c_int] * 3 + [_i32p, _i32p, _i32p, _i32p]
         L.oracle_expert_rows.restype = ctypes.c_int
@@ -106,7 +106,11 @@ def logits(x, Wr, br=None, nthreads=0):
     return out
 
 
-def route(logits_, k, K):
+RENORMALIZE = 1
+ARRIVAL_ORDER = 2
+
+
+def route(logits_, k, K, flags=0):
     L = _c(logits_, np.float32)
     T, E = L.shape
     ids = np.empty((T, k), np.int32)
@@ -114,7 +118,7 @@ def route(logits_, k, K):
     slot = np.empty((T, k), np.int32)
     drop = np.empty((T, k), np.uint8)
     counts = np.empty(2 * E, np.int32)
-    rc = lib().oracle_route(T, E, k, int(K), L, ids, w, slot, drop, counts)
+    rc = lib().oracle_route(T, E, k, int(K), L, ids, w, slot, drop, counts, int(flags))
     if rc != 0:
         raise ValueError("oracle_route rejected its arguments")
     return dict(ids=ids, w=w, slot=slot, drop=drop, received=counts[:E].copy(),
@@ -175,13 +179,13 @@ def combine_tokens(x, W1, b1, W2, b2, route_, tokens=None, nthreads=0):
     return out64, outx
 
 
-def forward(x, Wr, br, W1, b1, W2, b2, k, C, tokens=None, logits_=None, nthreads=0):
+def forward(x, Wr, br, W1, b1, W2, b2, k, C, tokens=None, logits_=None, nthreads=0, flags=0):
     """The whole layer: logits (unless given), routing, and outputs for ``tokens``."""
     T = x.shape[0]
     E = W1.shape[0]
     L = logits(x, Wr, br, nthreads) if logits_ is None else _c(logits_, np.float32)
     K = capacity(T, E, k, C)
-    r = route(L, k, K)
+    r = route(L, k, K, flags)
     out64, outx = combine_tokens(x, W1, b1, W2, b2, r, tokens, nthreads)
     return dict(logits=L, K=K, route=r, out_f64=out64, out=outx)
 

@@ -215,8 +215,11 @@ void oracle_logits(int T, int d, int E, int dtype, const void* x, const float* W
 //   slot[T*k]: rank among the expert's kept tokens (ascending t), -1 if dropped;
 //   drop[T*k]: 1 if dropped;  counts[2E]: received per expert, then kept per expert.
 // Returns 0, or -1 on bad arguments.
+// flags: 1 = renormalise each token's k weights by their sum (fp32, j ascending, one division
+// each); 2 = capacity by arrival (token) order instead of by weight ("Some Tokens Do Not Get
+// In", "Past the edge").
 int oracle_route(int T, int E, int k, long long K, const float* logits, int32_t* ids, float* w,
-                 int32_t* slot, uint8_t* drop, int32_t* counts) {
+                 int32_t* slot, uint8_t* drop, int32_t* counts, int flags) {
     if (T < 0 || E <= 0 || k <= 0 || k > E || K < 0) return -1;
     std::vector<float> p(E);
     for (int t = 0; t < T; ++t) {
@@ -233,6 +236,11 @@ int oracle_route(int T, int E, int k, long long K, const float* logits, int32_t*
             ids[(size_t)t * k + j] = best;
             w[(size_t)t * k + j] = p[best];
         }
+        if (flags & 1) {
+            float sum = 0.0f;
+            for (int j = 0; j < k; ++j) sum = sum + w[(size_t)t * k + j];
+            for (int j = 0; j < k; ++j) w[(size_t)t * k + j] = w[(size_t)t * k + j] / sum;
+        }
     }
     // Candidate pairs of each expert, ascending token index.
     std::vector<std::vector<int>> cand(E);
@@ -243,11 +251,12 @@ int oracle_route(int T, int E, int k, long long K, const float* logits, int32_t*
         // order[] holds positions into c, sorted by (weight descending, token ascending).
         std::vector<int> order(c.size());
         for (size_t i = 0; i < c.size(); ++i) order[i] = (int)i;
-        std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
-            float wa = w[c[a]], wb = w[c[b]];
-            if (wa != wb) return wa > wb;
-            return c[a] / k < c[b] / k;
-        });
+        if (!(flags & 2))                               // by weight; else keep arrival order
+            std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+                float wa = w[c[a]], wb = w[c[b]];
+                if (wa != wb) return wa > wb;
+                return c[a] / k < c[b] / k;
+            });
         std::vector<char> keep(c.size(), 0);
         long long nkeep = std::min<long long>(K, (long long)order.size());
         for (long long i = 0; i < nkeep; ++i) keep[order[i]] = 1;

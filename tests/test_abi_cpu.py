@@ -81,10 +81,14 @@ def test_malformed_problems_rejected(moe, bad):
     assert rc == 1
 
 
-def test_flags_must_be_zero(moe):
-    p = moe.Problem(16, 64, 64, 4, 2, 1.0, 1, 1)
+def test_unknown_flags_rejected(moe):
     n = ctypes.c_size_t()
-    assert moe.lib().moe_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 1
+    for bad in (4, 8, 0x80000000):
+        p = moe.Problem(16, 64, 64, 4, 2, 1.0, 1, bad)
+        assert moe.lib().moe_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 1
+    for good in (0, moe.FLAG_RENORMALIZE, moe.FLAG_ARRIVAL_ORDER, 3):
+        p = moe.Problem(16, 64, 64, 4, 2, 1.0, 1, good)
+        assert moe.lib().moe_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
 
 
 def test_status_strings(moe):

@@ -23,13 +23,13 @@ def _moe():
     return moe
 
 
-def _route_both(L, T, E, k, C, dtype="bf16", d=64, F=64):
+def _route_both(L, T, E, k, C, dtype="bf16", d=64, F=64, flags=0):
     moe = _moe()
-    layer = moe.MoELayer(T, d, F, E, k, C, dtype)
+    layer = moe.MoELayer(T, d, F, E, k, C, dtype, flags=flags)
     r = layer.route(to_dev(L))
     torch.cuda.synchronize()
     assert moe.moe_get_device_status(layer.ws) == 0
-    ro = oracle.route(L, k, layer.K)
+    ro = oracle.route(L, k, layer.K, flags)
     return layer, {k_: to_host(v) for k_, v in r.items()}, ro
 
 
@@ -184,10 +184,11 @@ def test_combine_parity(T, d, E, k, C, dtype):
 # ------------------------------------------------------------------------------------------
 # The fused forward against the oracle's whole layer.
 # ------------------------------------------------------------------------------------------
-def _forward_check(spec, seed, tokens=None, logit_rel=1e-4):
+def _forward_check(spec, seed, tokens=None, logit_rel=1e-4, flags=0):
     moe = _moe()
     L = inputs.make_layer(spec, seed=seed)
-    layer = moe.MoELayer(spec.T, spec.d_model, spec.d_ff, spec.E, spec.k, spec.C, spec.dtype)
+    layer = moe.MoELayer(spec.T, spec.d_model, spec.d_ff, spec.E, spec.k, spec.C, spec.dtype,
+                         flags=flags)
     args = [to_dev(L[n]) for n in ("x", "Wr", "br", "W1", "b1", "W2", "b2")]
     out, rt = layer.forward(*args, want_routing=True)
     torch.cuda.synchronize()
@@ -196,7 +197,7 @@ def _forward_check(spec, seed, tokens=None, logit_rel=1e-4):
     Lref = oracle.logits(L["x"], L["Wr"], L["br"])
     lerr = np.abs(g["logits_out"] - Lref).max()
     assert lerr <= logit_rel * max(1.0, float(np.abs(Lref).max())), lerr
-    ro = oracle.route(Lref, spec.k, layer.K)
+    ro = oracle.route(Lref, spec.k, layer.K, flags)
     # The logits differ from the oracle's by rounding, so the order of a token's experts can
     # differ where two of its top-k logits are that close; compare per (token, expert) pair.
     # Expert choice itself is pinned by the gap screen; capacity decisions may only differ where
@@ -281,12 +282,13 @@ def test_unsupported_and_invalid():
 @pytest.mark.parametrize("T,d,E,k,C", [(3000, 128, 64, 6, 1.0), (1000, 256, 8, 2, 1.25),
                                        (777, 64, 33, 4, 0.75), (200, 64, 16, 8, math.inf),
                                        (5000, 64, 64, 6, 0.5), (129, 64, 1, 1, 1.0)])
-def test_fused_router_matches_route(T, d, E, k, C):
+@pytest.mark.parametrize("flags", [0, 1, 3])
+def test_fused_router_matches_route(T, d, E, k, C, flags):
     moe = _moe()
     spec = inputs.LayerSpec("fused", T, d, 64, E, k, C, "bf16", router="normal",
                             router_bias=0.5)
     L = inputs.make_layer(spec, seed=E + T)
-    layer = moe.MoELayer(T, d, 64, E, k, C, "bf16")
+    layer = moe.MoELayer(T, d, 64, E, k, C, "bf16", flags=flags)
     args = [to_dev(L[n]) for n in ("x", "Wr", "br", "W1", "b1", "W2", "b2")]
     _, rt = layer.forward(*args, want_routing=True)
     r = layer.route(rt["logits_out"])
@@ -297,3 +299,92 @@ def test_fused_router_matches_route(T, d, E, k, C):
     assert torch.equal(rt["slot_out"], r["slot"])
     assert torch.equal(rt["drop_out"], r["drop"])
     assert torch.equal(rt["counts_out"], r["counts"])
+
+
+# ------------------------------------------------------------------------------------------
+# Routing-policy flags (renormalised weights, arrival-order capacity), bit for bit.
+# ------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("flags", [1, 2, 3])
+@pytest.mark.parametrize("T,E,k,C,seed", [(3000, 64, 6, 1.0, 1), (1000, 8, 2, 0.5, 2),
+                                          (777, 100, 8, 0.75, 3), (513, 32, 32, 1.0, 4),
+                                          (2048, 16, 1, 0.25, 5)])
+def test_route_flags_bit_exact(flags, T, E, k, C, seed):
+    L = inputs.random_logits(T, E, seed, 2.0)
+    _, g, ro = _route_both(L, T, E, k, C, flags=flags)
+    _assert_route_equal(g, ro, E)
+
+
+@pytest.mark.parametrize("flags", [1, 2, 3])
+def test_forward_with_flags(flags):
+    spec = inputs.LayerSpec("flags", 600, 128, 192, 8, 2, 0.75, "bf16", router="normal",
+                            router_bias=0.5, bias_std=0.05)
+    _forward_check(spec, seed=3, flags=flags)
+
+
+# ------------------------------------------------------------------------------------------
+# Small batches (T*k <= 1024) take the single-launch dispatch; same results, bit for bit.
+# ------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("flags", [0, 2, 3])
+@pytest.mark.parametrize("T,E,k,C,seed", [(128, 8, 8, 0.5, 1), (1024, 64, 1, 0.3, 2),
+                                          (100, 1024, 8, 1.0, 3), (64, 64, 8, math.inf, 4),
+                                          (512, 16, 2, 0.0, 5), (33, 3, 3, 0.4, 6)])
+def test_route_small_batches_bit_exact(flags, T, E, k, C, seed):
+    L = inputs.random_logits(T, E, seed, 1.5)
+    _, g, ro = _route_both(L, T, E, k, C, flags=flags)
+    _assert_route_equal(g, ro, E)
+
+
+def test_route_small_batch_weight_ties():
+    rng = np.random.default_rng(8)
+    proto = rng.standard_normal((3, 10)).astype(np.float32)
+    L = proto[rng.integers(0, 3, size=200)]
+    _, g, ro = _route_both(L, 200, 10, 2, 0.6)
+    _assert_route_equal(g, ro, 10)
+
+
+# ------------------------------------------------------------------------------------------
+# The whole forward replayed from a CUDA graph (no host sync or allocation inside the call).
+# ------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("spec", [inputs.LayerSpec("g1", 64, 256, 128, 16, 4, math.inf, "bf16"),
+                                  inputs.LayerSpec("g2", 2000, 128, 192, 8, 2, 1.0, "bf16",
+                                                   router="zipf", router_bias=1.1)])
+def test_forward_cuda_graph_replay(spec):
+    moe = _moe()
+    L = inputs.make_layer(spec, seed=2)
+    layer = moe.MoELayer(spec.T, spec.d_model, spec.d_ff, spec.E, spec.k, spec.C, spec.dtype)
+    args = [to_dev(L[n]) for n in ("x", "Wr", "br", "W1", "b1", "W2", "b2")]
+    eager = layer.forward(*args)
+    out = torch.empty_like(eager)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        layer.forward(*args, out=out)                 # warm-up on the capture stream type
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        layer.forward(*args, out=out)
+    out.zero_()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(layer.ws) == 0
+    assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+
+
+# ------------------------------------------------------------------------------------------
+# Failure detection: a pipeline wait that can never complete gives up, reports a timeout in the
+# status word, and leaves the GPU usable (no trap, no fault, no hang).
+# ------------------------------------------------------------------------------------------
+def test_bounded_wait_reports_timeout_and_gpu_stays_usable():
+    moe = _moe()
+    layer = moe.MoELayer(256, 64, 64, 8, 2, 1.0, "bf16")
+    moe.moe_reset_device_status(layer.ws)
+    moe.moe_selftest_wait_timeout(layer.ws, 50000)       # 50 ms
+    assert moe.moe_get_device_status(layer.ws) == moe.DEV_TIMEOUT
+    moe.moe_reset_device_status(layer.ws)
+    L = inputs.random_logits(256, 8, 1)
+    r = layer.route(to_dev(L))
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(layer.ws) == 0
+    ro = oracle.route(L, 2, layer.K)
+    assert np.array_equal(to_host(r["slot"]), ro["slot"])

@@ -382,3 +382,66 @@ def test_bf16_rounding_against_exhaustive_table():
         best = min(cands, key=lambda j: (abs(vals[j] - a), pats[j] & 1))
         expect = int(pats[best]) | (0x8000 if math.copysign(1.0, v) < 0 else 0)
         assert oracle.bf16_from_double(v) == expect, v
+
+
+# ------------------------------------------------------------------------------------------
+# Routing-policy flags: renormalised top-k weights and arrival-order capacity.
+# ------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("seed", range(4))
+def test_renormalized_weights(seed):
+    T, E, k = 300, 16, 4
+    L = inputs.random_logits(T, E, seed, 2.0)
+    K = oracle.capacity(T, E, k, 1.0)
+    plain = oracle.route(L, k, K)
+    r = oracle.route(L, k, K, oracle.RENORMALIZE)
+    assert np.array_equal(r["ids"], plain["ids"])            # same experts, same order
+    p = torch.softmax(torch.from_numpy(L.astype(np.float64)), dim=1).numpy()
+    top = np.take_along_axis(p, r["ids"].astype(np.int64), 1)
+    ref = top / top.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(r["w"], ref, rtol=2e-6, atol=0)
+    np.testing.assert_allclose(r["w"].astype(np.float64).sum(axis=1), 1.0, atol=4e-7 * k)
+    # Drop priority follows the renormalised weights.
+    for e in range(E):
+        m = r["ids"] == e
+        kept, dropped = m & (r["slot"] >= 0), m & (r["slot"] < 0)
+        if dropped.any():
+            assert r["w"][kept].min() >= r["w"][dropped].max()
+
+
+@pytest.mark.parametrize("seed", range(4))
+@pytest.mark.parametrize("T,E,k,C", [(200, 8, 2, 0.5), (64, 4, 1, 1.0), (500, 16, 4, 0.25)])
+def test_arrival_order_capacity_brute_force(seed, T, E, k, C):
+    L = inputs.random_logits(T, E, seed)
+    K = oracle.capacity(T, E, k, C)
+    r = oracle.route(L, k, K, oracle.ARRIVAL_ORDER)
+    for e in range(E):
+        cand = [(t, j) for t in range(T) for j in range(k) if r["ids"][t, j] == e]
+        for i, (t, j) in enumerate(cand):                    # ascending token order
+            if i < K:
+                assert r["slot"][t, j] == i and r["drop"][t, j] == 0
+            else:
+                assert r["slot"][t, j] == -1 and r["drop"][t, j] == 1
+
+
+def test_arrival_order_drops_the_late_token():
+    # The confidence-order example: under arrival order expert 0 keeps tokens 0 and 1 and
+    # drops token 2, although token 0 is its least confident.
+    L = np.array([[0.5, 0, 0], [3.0, 0, 0], [2.0, 0, 0], [0, 1.0, 0]], np.float32)
+    r = oracle.route(L, 1, 2, oracle.ARRIVAL_ORDER)
+    assert r["drop"][:, 0].tolist() == [0, 0, 1, 0]
+    g = _worked()
+    layer = inputs.make_layer(inputs.CONFIGS["tiny_f32"], seed=0)
+    r = oracle.route(layer["logits"], 1, g["K"], oracle.ARRIVAL_ORDER)
+    assert np.nonzero(r["drop"][:, 0])[0].tolist() == g["dropped_tokens"]   # token 4 is last
+
+
+def test_both_flags_compose():
+    T, E, k = 400, 8, 3
+    L = inputs.random_logits(T, E, 9, 1.5)
+    K = oracle.capacity(T, E, k, 0.6)
+    r = oracle.route(L, k, K, oracle.RENORMALIZE | oracle.ARRIVAL_ORDER)
+    rn = oracle.route(L, k, K, oracle.RENORMALIZE)
+    ra = oracle.route(L, k, K, oracle.ARRIVAL_ORDER)
+    assert np.array_equal(r["w"].view(np.uint32), rn["w"].view(np.uint32))
+    assert np.array_equal(r["slot"], ra["slot"])
