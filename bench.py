@@ -51,6 +51,8 @@ def parse():
                     help="warm-up lasts at least this long (clock sampler coverage)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the workload's token count (profiling of smaller cases)")
+    ap.add_argument("--gated", action="store_true",
+                    help="gated experts (SiLU(gate) * up, W1 twice as tall) on the same shapes")
     return ap.parse_args()
 
 
@@ -65,8 +67,9 @@ def peaks():
 
 def workload_desc(spec):
     C = "dropless" if math.isinf(spec.C) else "C=%g" % spec.C
-    return "%s: T=%d, d_model=%d, d_ff=%d, E=%d, top-%d, %s, %s" % (
-        spec.name, spec.T, spec.d_model, spec.d_ff, spec.E, spec.k, C, spec.dtype)
+    return "%s: T=%d, d_model=%d, d_ff=%d, E=%d, top-%d, %s, %s%s" % (
+        spec.name, spec.T, spec.d_model, spec.d_ff, spec.E, spec.k, C, spec.dtype,
+        ", gated experts" if spec.gated else "")
 
 
 # ------------------------------------------------------------------------------------------------
@@ -256,9 +259,11 @@ def run_cuda(args):
     spec = inputs.CONFIGS[args.config]
     if args.tokens:
         spec = dataclasses.replace(spec, T=args.tokens)
+    if args.gated:
+        spec = dataclasses.replace(spec, gated=True)
     L = inputs.make_layer(spec, seed=args.seed + rank)
     layer = moe.MoELayer(spec.T, spec.d_model, spec.d_ff, spec.E, spec.k, spec.C, spec.dtype,
-                         device=dev)
+                         device=dev, flags=moe.FLAG_GATED if spec.gated else 0)
     names = ("x", "Wr", "br", "W1", "b1", "W2", "b2")
     d = {n: to_dev(L[n], torch, dev) for n in names}
     out = torch.empty_like(d["x"])
@@ -377,12 +382,14 @@ def run_cuda(args):
     st_avg = stage_ms.mean(axis=0)
     names6 = moe.STAGE_NAMES
     gemm_flop_each = 2.0 * kept * dm * F
+    g1_flop = gemm_flop_each * (2 if spec.gated else 1)
     by = {
         "router_logits": dict(flop=2.0 * T * dm * E * 3, bytes=T * dm * esz + dm * E * 4 + T * E * 4),
         "route_topk": dict(bytes=T * E * 4 + T * k * 8),
         "capacity_dispatch": dict(bytes=T * k * 8 + T * k * 5 + kept * 4 + E * 16),
-        "expert_gemm1": dict(flop=gemm_flop_each,
-                             bytes=kept * dm * esz + E * F * dm * esz + kept * F * esz),
+        "expert_gemm1": dict(flop=g1_flop,
+                             bytes=kept * dm * esz + E * F * dm * esz * (2 if spec.gated else 1)
+                             + kept * F * esz),
         "expert_gemm2": dict(flop=gemm_flop_each,
                              bytes=kept * F * esz + E * dm * F * esz + kept * dm * esz),
         "combine": dict(bytes=2 * T * dm * esz + kept * dm * esz + T * k * 12 + (E + 1) * 4),
@@ -400,7 +407,7 @@ def run_cuda(args):
     dom = "expert_gemm1" if g1["ms"] >= g2["ms"] else "expert_gemm2"
     achieved = kernels[dom]["tflops"]
     gemm_ms = g1["ms"] + g2["ms"]
-    gemm_tflops = 2 * gemm_flop_each / (gemm_ms * 1e-3) / 1e12
+    gemm_tflops = (g1_flop + gemm_flop_each) / (gemm_ms * 1e-3) / 1e12
     rdc_bytes = sum(by[n]["bytes"] for n in ("route_topk", "capacity_dispatch", "combine"))
     rdc_ms = sum(kernels[n]["ms"] for n in ("route_topk", "capacity_dispatch", "combine"))
     rdc_gbs = rdc_bytes / (rdc_ms * 1e-3) / 1e9
@@ -433,7 +440,7 @@ def run_cuda(args):
                      "traffic": traffic_record(dom)},
         "expert_gemm": {"tflops": gemm_tflops, "frac_of_peak": gemm_tflops / tensor_peak,
                         "frac_of_burst_peak": gemm_tflops / pk.get("bf16_tflops", tensor_peak),
-                        "flop_per_step": 2 * gemm_flop_each},
+                        "flop_per_step": g1_flop + gemm_flop_each},
         "route_dispatch_combine": {"gbs": rdc_gbs, "frac_of_hbm": rdc_gbs / pk["hbm_gbs"],
                                    "bytes_per_step": rdc_bytes, "hbm_peak_gbs": pk["hbm_gbs"]},
         "kernels": kernels,

@@ -206,6 +206,78 @@ __global__ void __launch_bounds__(256) combine_vec_kernel(
     }
 }
 
+// Small batches: one block per token, so a token's row is spread over up to 256 threads and each
+// thread issues its x and kept-row loads at once (the warp-per-token kernel would leave most of
+// the GPU idle with few tokens).
+template <class Tr, int KMAX>
+__global__ void __launch_bounds__(256) combine_token_block_kernel(
+    const uint4* __restrict__ x, const uint4* __restrict__ Y, const float* __restrict__ w,
+    const int32_t* __restrict__ ids, const int32_t* __restrict__ slot,
+    const int32_t* __restrict__ offsets, int nv, int E, int k, uint4* __restrict__ out,
+    DeviceStatus* st) {
+    constexpr int V = Tr::kVec;
+    __shared__ int s_rows[KMAX];
+    __shared__ float s_w[KMAX];
+    __shared__ int s_nk;
+    const int t = blockIdx.x;
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int row = -1;
+        float wt = 0.0f;
+        if (lane < k) {
+            const size_t p = (size_t)t * k + lane;
+            const int s = slot[p];
+            if (s >= 0) {
+                const int e = ids[p];
+                if ((unsigned)e < (unsigned)E) {
+                    const int r = offsets[e] + s;
+                    if (r < offsets[e + 1]) { row = r; wt = w[p]; }
+                    else report(st, MOE_DEV_BAD_INDEX, 305);
+                } else {
+                    report(st, MOE_DEV_BAD_INDEX, 306);
+                }
+            }
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, row >= 0);
+        if (row >= 0) {
+            const int pos = __popc(m & ((1u << lane) - 1u));
+            s_rows[pos] = row;
+            s_w[pos] = wt;
+        }
+        if (lane == 0) s_nk = __popc(m);
+    }
+    __syncthreads();
+    const int nk = s_nk;
+    const uint4* xr = x + (size_t)t * nv;
+    uint4* orow = out + (size_t)t * nv;
+    for (int c = threadIdx.x; c < nv; c += blockDim.x) {
+        const uint4 xv4 = __ldg(xr + c);
+        if (nk == 0) { orow[c] = xv4; continue; }
+        uint4 yv4[KMAX];
+#pragma unroll
+        for (int q = 0; q < KMAX; ++q)
+            if (q < nk) yv4[q] = __ldg(Y + (size_t)s_rows[q] * nv + c);
+        float acc[V];
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] = 0.0f;
+#pragma unroll
+        for (int q = 0; q < KMAX; ++q) {
+            if (q < nk) {
+                float yv[V];
+                Tr::unpack(yv4[q], yv);
+                const float wq = s_w[q];
+#pragma unroll
+                for (int i = 0; i < V; ++i) acc[i] = __fmaf_rn(wq, yv[i], acc[i]);
+            }
+        }
+        float xv[V];
+        Tr::unpack(xv4, xv);
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] = __fadd_rn(xv[i], acc[i]);
+        orow[c] = Tr::pack(acc);
+    }
+}
+
 // ---------------------------------------------------------------------------------------------
 // fp32 expert FFN on CUDA cores (small fp32 layers): one block per kept row.
 //   h = W1[e] x + b1[e]; a = SiLU(h) = h / (1 + exp(-h)); Y = W2[e] a + b2[e]
@@ -216,7 +288,7 @@ __global__ void __launch_bounds__(256) ffn_f32_kernel(
     const int32_t* __restrict__ offsets, int E, int T, int d, int F,
     const float* __restrict__ W1, const float* __restrict__ b1, const float* __restrict__ W2,
     const float* __restrict__ b2, float* __restrict__ H, float* __restrict__ Y,
-    DeviceStatus* st) {
+    DeviceStatus* st, int gated) {
     extern __shared__ float s_mem[];
     float* xs = s_mem;          // [d]
     float* as = s_mem + d;      // [F]
@@ -237,12 +309,19 @@ __global__ void __launch_bounds__(256) ffn_f32_kernel(
     if ((unsigned)t >= (unsigned)T) { if (threadIdx.x == 0) report(st, MOE_DEV_BAD_INDEX, 401); return; }
     for (int i = threadIdx.x; i < d; i += blockDim.x) xs[i] = x[(size_t)t * d + i];
     __syncthreads();
-    const float* W1e = W1 + (size_t)e * F * d;
+    const size_t F1 = gated ? 2 * (size_t)F : (size_t)F;    // W1 rows per expert
+    const float* W1e = W1 + (size_t)e * F1 * d;
     for (int f = threadIdx.x; f < F; f += blockDim.x) {
         float h = 0.0f;
         for (int i = 0; i < d; ++i) h = __fmaf_rn(W1e[(size_t)f * d + i], xs[i], h);
-        if (b1) h += b1[(size_t)e * F + f];
-        const float a = h / (1.0f + expf(-h));
+        if (b1) h += b1[(size_t)e * F1 + f];
+        float a = h / (1.0f + expf(-h));
+        if (gated) {                                  // a = SiLU(gate) * up
+            float u = 0.0f;
+            for (int i = 0; i < d; ++i) u = __fmaf_rn(W1e[(size_t)(F + f) * d + i], xs[i], u);
+            if (b1) u += b1[(size_t)e * F1 + F + f];
+            a *= u;
+        }
         if (H) H[(size_t)r * F + f] = a;
         as[f] = a;
     }
@@ -288,6 +367,14 @@ void launch_combine(int dtype, const void* x, const void* Y, const float* w, con
     const int blocks = (T + 7) / 8;
     const bool aligned = ((uintptr_t)x % 16 == 0) && ((uintptr_t)Y % 16 == 0) &&
                          ((uintptr_t)out % 16 == 0);
+    if (dtype == MOE_BF16 && aligned && d % 8 == 0 && k <= 8 && T < 4 * 148) {
+        const int nv = d / 8;
+        const int threads = std::min(256, ((nv + 31) / 32) * 32);
+        combine_token_block_kernel<BF16Traits, 8><<<T, threads, 0, s>>>(
+            (const uint4*)x, (const uint4*)Y, w, ids, slot, offsets, nv, E, k, (uint4*)out, st);
+        *launches += 1;
+        return;
+    }
     if (dtype == MOE_BF16 && aligned && d % 8 == 0 && k <= 8) {
         combine_vec_kernel<BF16Traits, 8><<<blocks, 256, 0, s>>>(
             (const uint4*)x, (const uint4*)Y, w, ids, slot, offsets, T, d / 8, E, k, (uint4*)out,
@@ -316,11 +403,11 @@ void launch_combine(int dtype, const void* x, const void* Y, const float* w, con
 void launch_ffn_f32(const float* x, const int32_t* rowtok, const int32_t* offsets, int E, int T,
                     int d, int F, long long max_rows, const float* W1, const float* b1,
                     const float* W2, const float* b2, float* H, float* Y, DeviceStatus* st,
-                    cudaStream_t s, int* launches) {
+                    cudaStream_t s, int* launches, bool gated) {
     if (max_rows <= 0) return;
     const size_t smem = sizeof(float) * ((size_t)d + F);
     ffn_f32_kernel<<<(unsigned)max_rows, 256, smem, s>>>(x, rowtok, offsets, E, T, d, F, W1, b1,
-                                                         W2, b2, H, Y, st);
+                                                         W2, b2, H, Y, st, gated ? 1 : 0);
     *launches += 1;
 }
 

@@ -47,7 +47,9 @@ constexpr int kMaxGroups = 1024;
 
 // kEpiRouterFused: the router epilogue also forms the softmax, the top-k and the per-chunk
 // expert counts of its tokens (all E <= 64 experts of a token sit in one thread's TMEM lane).
-enum Epi { kEpiSiLU = 0, kEpiBias = 1, kEpiRouter = 2, kEpiRouterFused = 3 };
+// kEpiSwiGLU: gated experts; the tile's 256 B rows are 128 gate rows and the matching 128 up
+// rows, and the epilogue writes SiLU(gate) * up for 128 hidden features.
+enum Epi { kEpiSiLU = 0, kEpiBias = 1, kEpiRouter = 2, kEpiRouterFused = 3, kEpiSwiGLU = 4 };
 
 struct GemmArgs {
     const __nv_bfloat16* A;   // [*, lda] row-major
@@ -354,7 +356,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t ph = (it / S) & 1u;
                     if (!mbar_wait<PAIR>(empty_bar(s), ph ^ 1u, st, 1)) { ok = false; break; }
                     if (leader) mbar_arrive_expect_tx(full_bar(s), kTx);
-                    if (PAIR) {
+                    if (EPI == kEpiSwiGLU) {
+                        // gate rows [e*2F + nt*128, +128) and up rows [e*2F + F + nt*128, +128)
+                        // (a pair CTA holds one of the two 128-row halves).
+                        const int g0 = tc.e * args.b_rows_per_group + tc.nt * 128;
+                        const int u0 = g0 + args.Nout;
+                        if (PAIR) {
+                            if (!GATHER)
+                                tma_load_2d_pair(sA(s), &tmA, lead(full_bar(s)), kb * kBK, tc.row0);
+                            tma_load_2d_pair(sB(s), &tmB, lead(full_bar(s)), kb * kBK,
+                                             crank ? u0 : g0);
+                        } else {
+                            if (!GATHER) tma_load_2d(sA(s), &tmA, full_bar(s), kb * kBK, tc.row0);
+                            tma_load_2d(sB(s), &tmB, full_bar(s), kb * kBK, g0);
+                            tma_load_2d(sB(s) + 128u * 128u, &tmB, full_bar(s), kb * kBK, u0);
+                        }
+                    } else if (PAIR) {
                         const uint32_t fb = lead(full_bar(s));
                         if (!GATHER) tma_load_2d_pair(sA(s), &tmA, fb, kb * kBK, tc.row0);
                         tma_load_2d_pair(sB(s), &tmB, fb, kb * kBK, brow);
@@ -409,8 +426,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tempty_target0 = lead(tempty_bar(0));
         const uint32_t tempty_target1 = lead(tempty_bar(1));
         const uint32_t stg = base + C::kStgOff + (uint32_t)(warp - 2) * 2048u;
-        constexpr int kChunks = (BN + 31) / 32;
-        constexpr int kHalf = (kChunks + 1) / 2;
         uint32_t lt = 0;
         for (int tile = cid; tile < total; tile += ncl, ++lt) {
             const TileCoord tc = tile_coord<TM>(tile, s_mt, E, n_tiles, args, (int)crank);
@@ -530,16 +545,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                             args.r_cnt[(size_t)e * args.r_nC + chunk] = s_cnt[e];
                 }
             } else {
-                const int n0 = tc.nt * BN;
-                const float* bias = args.bias ? args.bias + (size_t)tc.e * args.Nout + n0 : nullptr;
+                // Output columns of this tile: BN (128 hidden features for gated experts).
+                constexpr int kOut = EPI == kEpiSwiGLU ? 128 : BN;
+                constexpr int kOutChunks = (kOut + 31) / 32;
+                constexpr int kOutHalf = (kOutChunks + 1) / 2;
+                const int n0 = tc.nt * kOut;
+                const float* bias = args.bias ? args.bias + (size_t)tc.e * args.b_rows_per_group + n0
+                                              : nullptr;
 #pragma unroll 1
-                for (int ci = h * kHalf; ci < kChunks && ci < (h + 1) * kHalf; ++ci) {
+                for (int ci = h * kOutHalf; ci < kOutChunks && ci < (h + 1) * kOutHalf; ++ci) {
                     const int c0 = ci * 32;
-                    const int ncol = (BN - c0) >= 32 ? 32 : 16;
+                    const int ncol = (kOut - c0) >= 32 ? 32 : 16;
                     float v[32];
+                    float u[32];
                     __syncwarp();
                     if (ncol == 32) tmem_ld32_wait(taddr + c0, v);
                     else tmem_ld16_wait(taddr + c0, v);
+                    if (EPI == kEpiSwiGLU) tmem_ld32_wait(taddr + 128 + c0, u);
                     if (n0 + c0 >= args.Nout || wrows == 0) continue;
                     const int nc = min(ncol, args.Nout - (n0 + c0));     // 16 or 32
                     if (bias) {
@@ -548,6 +570,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (i >= nc) break;
                             const float4 bv = __ldg(reinterpret_cast<const float4*>(bias + c0 + i));
                             v[i] += bv.x; v[i + 1] += bv.y; v[i + 2] += bv.z; v[i + 3] += bv.w;
+                            if (EPI == kEpiSwiGLU) {
+                                const float4 bu = __ldg(reinterpret_cast<const float4*>(
+                                    bias + args.Nout + c0 + i));
+                                u[i] += bu.x; u[i + 1] += bu.y; u[i + 2] += bu.z; u[i + 3] += bu.w;
+                            }
                         }
                     }
                     uint32_t pk[16];
@@ -555,9 +582,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < 32; i += 2) {
                         if (i >= nc) break;
                         float a0 = v[i], a1 = v[i + 1];
-                        if (EPI == kEpiSiLU) {
+                        if (EPI == kEpiSiLU || EPI == kEpiSwiGLU) {
                             a0 = __fdividef(a0, 1.0f + __expf(-a0));
                             a1 = __fdividef(a1, 1.0f + __expf(-a1));
+                        }
+                        if (EPI == kEpiSwiGLU) {
+                            a0 *= u[i];
+                            a1 *= u[i + 1];
                         }
                         pk[i >> 1] = pack_bf16x2(a0, a1);
                     }
@@ -848,6 +879,14 @@ int router_group(int E) { return E <= 16 ? 16 : (E <= 32 ? 32 : 64); }
 // Pair (2-SM) tiles when the experts' rows fill 256-row tiles well enough; 1-SM otherwise.
 int g_pair_mode = -1;      // -1 automatic, 0 never, 1 always (MOE_GEMM_PAIR in the environment)
 
+// Gated experts' first GEMM: W is [E, 2F, K] (gate rows then up rows), bias [E, 2F]; D = H [rows,
+// F] = SiLU(A W_gate^T + b_gate) * (A W_up^T + b_up).  256-wide tiles = 128 gate + 128 up rows.
+cudaError_t launch_gated_gemm(const void* A, long long lda, const int32_t* a_rows,
+                              int a_row_limit, const int32_t* offsets, int E, int K, int F,
+                              const void* W, const float* bias, void* D, long long ldd,
+                              long long max_rows, DeviceStatus* st, cudaStream_t s,
+                              int* launches);
+
 bool use_pair(long long max_rows, int E) {
     if (g_pair_mode < 0) {
         const char* v = getenv("MOE_GEMM_PAIR");
@@ -863,6 +902,10 @@ cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const in
                                const void* W, const float* bias, void* D, long long ldd,
                                long long max_rows, DeviceStatus* st, cudaStream_t s,
                                int* launches) {
+    if (which == 2) {
+        return launch_gated_gemm(A, lda, a_rows, a_row_limit, offsets, E, K, Nout, W, bias, D,
+                                 ldd, max_rows, st, s, launches);
+    }
     const int BN = pick_bn(Nout);
     // Gathered A on pairs needs the peer's rows forwarded to the leader's barrier by the copying
     // threads themselves, which measured slower than single-CTA tiles; only when forced.
@@ -907,6 +950,49 @@ cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const in
         e = which == 0 ? launch_gemm_bn<kEpiSiLU, false, false>(BN, tmA, tm, a, max_tiles, s)
                        : launch_gemm_bn<kEpiBias, false, false>(BN, tmA, tm, a, max_tiles, s);
     }
+    if (e == cudaSuccess) *launches += 1;
+    return e;
+}
+
+cudaError_t launch_gated_gemm(const void* A, long long lda, const int32_t* a_rows,
+                              int a_row_limit, const int32_t* offsets, int E, int K, int F,
+                              const void* W, const float* bias, void* D, long long ldd,
+                              long long max_rows, DeviceStatus* st, cudaStream_t s,
+                              int* launches) {
+    if (F % 128 != 0) return cudaErrorInvalidValue;
+    const bool pair = use_pair(max_rows, E) && (a_rows == nullptr || g_pair_mode == 1);
+    CUtensorMap tm;
+    if (!make_tmap(&tm, W, (long long)E * 2 * F, K, 128)) return cudaErrorInvalidValue;
+    GemmArgs a{};
+    a.A = reinterpret_cast<const __nv_bfloat16*>(A);
+    a.lda = lda;
+    a.a_rows = a_rows;
+    a.a_row_limit = a_row_limit;
+    a.offsets = offsets;
+    a.E = E;
+    a.K = K;
+    a.n_tiles = F / 128;
+    a.b_rows_per_group = 2 * F;
+    a.Nout = F;
+    a.bias = bias;
+    a.D = D;
+    a.ldd = ldd;
+    a.st = st;
+    const int tm_rows = pair ? 256 : kBM;
+    const long long max_tiles = ((max_rows + tm_rows - 1) / tm_rows + E) * a.n_tiles;
+    CUtensorMap tmA = tm;
+    const bool gather = a_rows != nullptr;
+    if (!gather && !make_tmap(&tmA, A, (long long)a_row_limit, K, kBM))
+        return cudaErrorInvalidValue;
+    cudaError_t e;
+    if (gather && pair)
+        e = launch_gemm_t<256, kEpiSwiGLU, true, true>(tmA, tm, a, max_tiles, s);
+    else if (gather)
+        e = launch_gemm_t<256, kEpiSwiGLU, true, false>(tmA, tm, a, max_tiles, s);
+    else if (pair)
+        e = launch_gemm_t<256, kEpiSwiGLU, false, true>(tmA, tm, a, max_tiles, s);
+    else
+        e = launch_gemm_t<256, kEpiSwiGLU, false, false>(tmA, tm, a, max_tiles, s);
     if (e == cudaSuccess) *launches += 1;
     return e;
 }

@@ -28,6 +28,12 @@ void launch_dispatch_small(const int32_t* ids, const float* w, int T, int E, int
                            unsigned flags, int32_t* slot, uint8_t* drop, int32_t* counts,
                            int32_t* offsets, int32_t* rowtok, DeviceStatus* st, cudaStream_t s,
                            int* launches);
+// Small batches of bf16 tokens (T <= 1024, E <= 256, d <= 12288): logits on CUDA cores and routing in one
+// launch, one block per token.  logits_out may be null.
+bool router_small_fits(int T, int E, int d);
+void launch_router_small(const void* x, const float* Wr, const float* br, int T, int d, int E,
+                         int k, float* logits_out, int32_t* ids, float* w, unsigned flags,
+                         cudaStream_t s, int* launches);
 void launch_wait_timeout_selftest(DeviceStatus* st, long long limit_ns, cudaStream_t s);
 void launch_dispatch(const int32_t* ids, const int32_t* slot, int T, int E, int k,
                      int32_t* kept_tmp, int32_t* offsets, int32_t* rowtok, DeviceStatus* st,
@@ -43,7 +49,7 @@ void launch_combine(int dtype, const void* x, const void* Y, const float* w, con
 void launch_ffn_f32(const float* x, const int32_t* rowtok, const int32_t* offsets, int E, int T,
                     int d, int F, long long max_rows, const float* W1, const float* b1,
                     const float* W2, const float* b2, float* H, float* Y, DeviceStatus* st,
-                    cudaStream_t s, int* launches);
+                    cudaStream_t s, int* launches, bool gated);
 void launch_logits_f32(const float* x, const float* Wr, const float* br, int T, int d, int E,
                        float* logits, cudaStream_t s, int* launches);
 
@@ -51,7 +57,9 @@ void launch_logits_f32(const float* x, const float* Wr, const float* br, int T, 
 int pick_bn(int nout);
 int router_group(int E);
 size_t router_split_bytes(int d, int E);
-// which = 0: D = SiLU(A W^T + bias) (GEMM1); which = 1: D = A W^T + bias (GEMM2).
+// which = 0: D = SiLU(A W^T + bias) (GEMM1); which = 1: D = A W^T + bias (GEMM2);
+// which = 2: gated GEMM1, W [E, 2*Nout, K] (gate rows, up rows), bias [E, 2*Nout],
+// D = SiLU(A W_gate^T + b_gate) * (A W_up^T + b_up) (Nout a multiple of 128).
 cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const int32_t* a_rows,
                                int a_row_limit, const int32_t* offsets, int E, int K, int Nout,
                                const void* W, const float* bias, void* D, long long ldd,

@@ -31,14 +31,17 @@ bool bad_problem(const moe_problem* p) {
     if (p->k < 1 || p->k > p->E || p->k > 32) return true;
     if (std::isnan(p->capacity_factor) || p->capacity_factor < 0.0f) return true;
     if (p->dtype != MOE_F32 && p->dtype != MOE_BF16) return true;
-    if (p->flags & ~(MOE_FLAG_RENORMALIZE | MOE_FLAG_ARRIVAL_ORDER)) return true;
+    if (p->flags & ~(MOE_FLAG_RENORMALIZE | MOE_FLAG_ARRIVAL_ORDER | MOE_FLAG_GATED)) return true;
     if ((long long)p->T * p->k > 0x7fffffffLL) return true;
     if ((long long)p->T * p->E > 0x7fffffffLL) return true;
     return false;
 }
 
 bool unsupported(const moe_problem* p) {
-    if (p->dtype == MOE_BF16) return (p->d_model % 64) != 0 || (p->d_ff % 64) != 0;
+    if (p->dtype == MOE_BF16) {
+        if ((p->d_model % 64) != 0 || (p->d_ff % 64) != 0) return true;
+        if ((p->flags & MOE_FLAG_GATED) && (p->d_ff % 128) != 0) return true;
+    }
     return false;
 }
 
@@ -148,14 +151,15 @@ moe_status ffn_steps(const moe_problem* p, const void* x, const int32_t* offsets
     moe::DeviceStatus* st = at<moe::DeviceStatus>(ws, q.status);
     const long long R = max_rows_of(p, capacity_of(p));
     if (R == 0) return MOE_OK;
+    const bool gated = (p->flags & MOE_FLAG_GATED) != 0;
     if (p->dtype == MOE_F32) {
         moe::launch_ffn_f32((const float*)x, rowtok, offsets, p->E, p->T, p->d_model, p->d_ff, R,
                             (const float*)W1, b1, (const float*)W2, b2, at<float>(ws, q.H),
-                            (float*)Y, st, s, launches);
+                            (float*)Y, st, s, launches, gated);
         return MOE_OK;
     }
     void* H = at<void>(ws, q.H);
-    if (moe::launch_expert_gemm(0, x, p->d_model, rowtok, p->T, offsets, p->E, p->d_model,
+    if (moe::launch_expert_gemm(gated ? 2 : 0, x, p->d_model, rowtok, p->T, offsets, p->E, p->d_model,
                                 p->d_ff, W1, b1, H, p->d_ff, R, st, s, launches) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (moe::launch_expert_gemm(1, H, p->d_ff, nullptr, (int)R, offsets, p->E, p->d_ff,
@@ -288,10 +292,15 @@ moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, con
     void* Y = at<void>(ws, q.Y);
 
     stage_mark(0, s);
-    // bf16 with E <= 64: the logits GEMM's epilogue also forms the softmax, top-k and per-chunk
-    // counts (one fused launch instead of logits + router + count kernels).
-    const bool fused = p->dtype == MOE_BF16 && moe::router_can_fuse(p->E);
-    if (p->dtype == MOE_BF16) {
+    // Small bf16 batches: logits on CUDA cores and routing in one launch (a 128-row tensor-core
+    // tile would leave the GPU idle).  Larger bf16 batches with E <= 64: the logits GEMM's
+    // epilogue also forms the softmax, top-k and per-chunk counts.
+    const bool small = p->dtype == MOE_BF16 && moe::router_small_fits(p->T, p->E, p->d_model);
+    const bool fused = !small && p->dtype == MOE_BF16 && moe::router_can_fuse(p->E);
+    if (small) {
+        moe::launch_router_small(x, Wr, br, p->T, p->d_model, p->E, p->k, logits_out, ids, w,
+                                 p->flags, s, &launches);
+    } else if (p->dtype == MOE_BF16) {
         moe::RouterFused rf{ids, w, at<int32_t>(ws, q.cnt), moe::chunk_count(p->T), p->k,
                             p->flags};
         if (moe::launch_router_gemm(x, p->T, p->d_model, Wr, br, p->E, at<void>(ws, q.split),
@@ -304,7 +313,7 @@ moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, con
     }
     stage_mark(1, s);
     const long long K = capacity_of(p);
-    if (!fused) {
+    if (!fused && !small) {
         moe::launch_route_topk(logits, p->T, p->E, p->k, ids, w, s, p->flags);
         launches += 1;
     }
@@ -321,7 +330,8 @@ moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, con
     const long long R = max_rows_of(p, K);
     if (R > 0 && p->dtype == MOE_BF16) {
         void* H = at<void>(ws, q.H);
-        if (moe::launch_expert_gemm(0, x, p->d_model, rowtok, p->T, offsets, p->E, p->d_model,
+        const int g1 = (p->flags & MOE_FLAG_GATED) ? 2 : 0;
+        if (moe::launch_expert_gemm(g1, x, p->d_model, rowtok, p->T, offsets, p->E, p->d_model,
                                     p->d_ff, W1, b1, H, p->d_ff, R, st, s, &launches) !=
             cudaSuccess)
             return MOE_ERR_CUDA;

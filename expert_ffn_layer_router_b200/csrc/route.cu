@@ -33,20 +33,18 @@ constexpr unsigned kFull = 0xffffffffu;
 // Router: softmax over E + top-k, one warp per token.  Lane l holds experts l, l+32, ...
 // Softmax sum order: lane partials left to right, then xor-butterfly 16, 8, 4, 2, 1.
 // ---------------------------------------------------------------------------------------------
+// One token's routing by one warp: L points at the token's E logits (global or shared).
 template <int EPL>
-__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T,
-                                                         int E, int k, int32_t* __restrict__ ids,
-                                                         float* __restrict__ w, unsigned flags) {
+__device__ __forceinline__ void route_token_warp(const float* L, int E, int k, size_t t,
+                                                 int32_t* __restrict__ ids,
+                                                 float* __restrict__ w, unsigned flags) {
     const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (t >= T) return;
-    const float* L = logits + (size_t)t * E;
     float v[EPL];
     uint32_t key[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
         const int e = lane + 32 * i;
-        v[i] = e < E ? __ldg(L + e) : 0.0f;
+        v[i] = e < E ? L[e] : 0.0f;
         key[i] = e < E ? float_key(v[i]) : 0u;
     }
     uint32_t lmax = 0;
@@ -97,9 +95,67 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
         my_w = __fdiv_rn(my_w, sum);
     }
     if (lane < k) {
-        ids[(size_t)t * k + lane] = my_id;
-        w[(size_t)t * k + lane] = my_w;
+        ids[t * k + lane] = my_id;
+        w[t * k + lane] = my_w;
     }
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T,
+                                                         int E, int k, int32_t* __restrict__ ids,
+                                                         float* __restrict__ w, unsigned flags) {
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    route_token_warp<EPL>(logits + (size_t)t * E, E, k, (size_t)t, ids, w, flags);
+}
+
+// Router for small batches of bf16 tokens: one block per token computes its E logits on CUDA
+// cores and warp 0 routes the token with the same arithmetic as route_topk_kernel.  Thread
+// (part, e) reduces d/P consecutive products with four interleaved accumulators (products
+// i = i0 + 4j + r go to accumulator r), combined as (a0 + a1) + (a2 + a3); the P parts are then
+// added in part order, plus the bias.  Fixed order, so the logits are deterministic.
+template <int EPL>
+__global__ void __launch_bounds__(1024) router_small_kernel(
+    const __nv_bfloat16* __restrict__ x, const float* __restrict__ Wr,
+    const float* __restrict__ br, int T, int d, int E, int k, float* __restrict__ logits_out,
+    int32_t* __restrict__ ids, float* __restrict__ w, unsigned flags) {
+    extern __shared__ float s_x[];                    // [d]
+    __shared__ float s_part[1024];
+    __shared__ float s_L[256];
+    const int t = blockIdx.x;
+    for (int i = threadIdx.x; i < d; i += blockDim.x)
+        s_x[i] = __bfloat162float(x[(size_t)t * d + i]);
+    __syncthreads();
+    const int P = (int)blockDim.x / E;                // parts of the reduction per expert
+    const int tid = threadIdx.x;
+    if (tid < P * E) {
+        const int e = tid % E, part = tid / E;
+        const int i0 = (int)((long long)d * part / P), i1 = (int)((long long)d * (part + 1) / P);
+        float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+        int i = i0;
+        for (; i + 3 < i1; i += 4) {
+            const float w0 = __ldg(Wr + (size_t)i * E + e);
+            const float w1 = __ldg(Wr + (size_t)(i + 1) * E + e);
+            const float w2 = __ldg(Wr + (size_t)(i + 2) * E + e);
+            const float w3 = __ldg(Wr + (size_t)(i + 3) * E + e);
+            a0 = __fmaf_rn(s_x[i], w0, a0);
+            a1 = __fmaf_rn(s_x[i + 1], w1, a1);
+            a2 = __fmaf_rn(s_x[i + 2], w2, a2);
+            a3 = __fmaf_rn(s_x[i + 3], w3, a3);
+        }
+        for (; i < i1; ++i) a0 = __fmaf_rn(s_x[i], __ldg(Wr + (size_t)i * E + e), a0);
+        s_part[part * E + e] = __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3));
+    }
+    __syncthreads();
+    if (tid < E) {
+        float L = s_part[tid];
+        for (int part = 1; part < P; ++part) L = __fadd_rn(L, s_part[part * E + tid]);
+        if (br) L = __fadd_rn(L, br[tid]);
+        s_L[tid] = L;
+        if (logits_out) logits_out[(size_t)t * E + tid] = L;
+    }
+    __syncthreads();
+    if (tid < 32) route_token_warp<EPL>(s_L, E, k, (size_t)t, ids, w, flags);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -540,6 +596,25 @@ void launch_route_topk(const float* logits, int T, int E, int k, int32_t* ids, f
 int chunk_count(int T) { return (T + kChunk - 1) / kChunk; }
 
 bool dispatch_small_fits(int T, int k) { return (long long)T * k <= kSmallPairs; }
+
+bool router_small_fits(int T, int E, int d) { return T <= 1024 && E <= 256 && d <= 12288; }
+
+void launch_router_small(const void* x, const float* Wr, const float* br, int T, int d, int E,
+                         int k, float* logits_out, int32_t* ids, float* w, unsigned flags,
+                         cudaStream_t s, int* launches) {
+    const size_t smem = sizeof(float) * (size_t)d;
+    const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+    const int epl = (E + 31) / 32;
+    if (epl <= 1)
+        router_small_kernel<1><<<T, 1024, smem, s>>>(xb, Wr, br, T, d, E, k, logits_out, ids, w, flags);
+    else if (epl <= 2)
+        router_small_kernel<2><<<T, 1024, smem, s>>>(xb, Wr, br, T, d, E, k, logits_out, ids, w, flags);
+    else if (epl <= 4)
+        router_small_kernel<4><<<T, 1024, smem, s>>>(xb, Wr, br, T, d, E, k, logits_out, ids, w, flags);
+    else
+        router_small_kernel<8><<<T, 1024, smem, s>>>(xb, Wr, br, T, d, E, k, logits_out, ids, w, flags);
+    *launches += 1;
+}
 
 namespace {
 // Failure-detection self-test: waits on an mbarrier that nothing arrives on, with the same

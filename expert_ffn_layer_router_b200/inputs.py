@@ -38,6 +38,7 @@ class LayerSpec:
     router: str = "plain"         # "plain" | "zipf" | "normal" | "given" (logits handed in)
     router_bias: float = 0.0      # zipf exponent s, or std of the normal router bias
     bias_std: float = 0.0         # std of b1/b2 (0 = zero biases)
+    gated: bool = False           # gated experts: W1 [E, 2*d_ff, d_model] (gate rows, up rows)
 
     @property
     def pairs(self) -> int:
@@ -135,10 +136,11 @@ def make_layer(spec: LayerSpec, seed: int = 0, T: int | None = None,
         br = (rng.standard_normal(E, dtype=np.float32) * np.float32(spec.router_bias)
               ).astype(np.float32)
     if weights:
-        W1 = rng.standard_normal((E, F, d), dtype=np.float32)
+        F1 = 2 * F if spec.gated else F
+        W1 = rng.standard_normal((E, F1, d), dtype=np.float32)
         W1 *= np.float32(1.0 / math.sqrt(d))
-        b1 = (rng.standard_normal((E, F), dtype=np.float32) * np.float32(spec.bias_std)
-              if spec.bias_std > 0 else np.zeros((E, F), np.float32))
+        b1 = (rng.standard_normal((E, F1), dtype=np.float32) * np.float32(spec.bias_std)
+              if spec.bias_std > 0 else np.zeros((E, F1), np.float32))
         W2 = rng.standard_normal((E, d, F), dtype=np.float32)
         W2 *= np.float32(1.0 / math.sqrt(F))
         b2 = (rng.standard_normal((E, d), dtype=np.float32) * np.float32(spec.bias_std)

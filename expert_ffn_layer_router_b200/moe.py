@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 MOE_F32, MOE_BF16 = 0, 1
-FLAG_RENORMALIZE, FLAG_ARRIVAL_ORDER = 1, 2
+FLAG_RENORMALIZE, FLAG_ARRIVAL_ORDER, FLAG_GATED = 1, 2, 4
 MOE_OK = 0
 DEV_OK, DEV_TIMEOUT, DEV_BAD_INDEX = 0, 1, 2
 

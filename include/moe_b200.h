@@ -85,6 +85,11 @@ typedef struct {
  *     the next one does not get in once the buffer is full), instead of the highest weights. */
 #define MOE_FLAG_RENORMALIZE 1u
 #define MOE_FLAG_ARRIVAL_ORDER 2u
+/* Expert variant: gated FFN, after the fused-MoE dataflow diagram (GEMM 1 writes gate and up
+ * halves, "SiLU x mul" combines them, GEMM 2 follows).  W1 is then [E, 2*d_ff, d_model] (rows
+ * [0, d_ff) the gate, [d_ff, 2*d_ff) the up projection) and b1 [E, 2*d_ff]; the expert computes
+ * a = SiLU(W1_gate x + b1_gate) * (W1_up x + b1_up), y = W2 a + b2.  bf16 needs d_ff % 128 == 0. */
+#define MOE_FLAG_GATED 4u
 
 /* Host only.  Per-expert capacity K = min(T, floor(C * T * k / E)) evaluated in double
  * (worked example, capacity paragraph; generalised to k slots per token as in "Some Tokens Do

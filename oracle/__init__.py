@@ -43,10 +43,10 @@ def lib():
         L.oracle_dispatch.argtypes = [ctypes.c_int] * 3 + [_i32p, _i32p, _i32p, _i32p]
         L.oracle_expert_rows.restype = ctypes.c_int
         L.oracle_expert_rows.argtypes = [ctypes.c_int] * 4 + [_vp] * 5 + [
-            ctypes.c_int, _i32p, _i32p, _f64p, _vp, ctypes.c_int]
+            ctypes.c_int, _i32p, _i32p, _f64p, _vp, ctypes.c_int, ctypes.c_int]
         L.oracle_combine_tokens.restype = ctypes.c_int
         L.oracle_combine_tokens.argtypes = [ctypes.c_int] * 6 + [_vp] * 5 + [
-            _i32p, _f32p, _i32p, ctypes.c_int, _i32p, _f64p, _vp, ctypes.c_int]
+            _i32p, _f32p, _i32p, ctypes.c_int, _i32p, _f64p, _vp, ctypes.c_int, ctypes.c_int]
         L.oracle_combine_given_y.restype = ctypes.c_int
         L.oracle_combine_given_y.argtypes = [ctypes.c_int] * 5 + [_vp, _vp, ctypes.c_longlong,
                                                                   _f32p, _i32p, _i32p, _i32p,
@@ -108,6 +108,7 @@ def logits(x, Wr, br=None, nthreads=0):
 
 RENORMALIZE = 1
 ARRIVAL_ORDER = 2
+GATED = 4
 
 
 def route(logits_, k, K, flags=0):
@@ -135,11 +136,12 @@ def dispatch(ids, slot, E):
     return offsets, rowtok[: int(offsets[-1])].copy()
 
 
-def expert_rows(x, W1, b1, W2, b2, row_tok, row_exp, want_h=False, nthreads=0):
+def expert_rows(x, W1, b1, W2, b2, row_tok, row_exp, want_h=False, nthreads=0, flags=0):
+    """Expert outputs per (token, expert) row.  flags & GATED: W1 is [E, 2F, d] (gate, up)."""
     x = np.ascontiguousarray(x)
     W1 = np.ascontiguousarray(W1)
     W2 = np.ascontiguousarray(W2)
-    E, F, d = W1.shape
+    E, d, F = W2.shape
     row_tok = _c(row_tok, np.int32)
     row_exp = _c(row_exp, np.int32)
     n = row_tok.size
@@ -148,13 +150,14 @@ def expert_rows(x, W1, b1, W2, b2, row_tok, row_exp, want_h=False, nthreads=0):
     b1c = None if b1 is None else _c(b1, np.float32)
     b2c = None if b2 is None else _c(b2, np.float32)
     rc = lib().oracle_expert_rows(d, F, E, _dtype_code(x), _ptr(x), _ptr(W1), _ptr(b1c),
-                                  _ptr(W2), _ptr(b2c), n, row_tok, row_exp, Y, _ptr(H), nthreads)
+                                  _ptr(W2), _ptr(b2c), n, row_tok, row_exp, Y, _ptr(H), nthreads,
+                                  int(flags))
     if rc != 0:
         raise ValueError("oracle_expert_rows rejected its arguments")
     return (Y, H) if want_h else Y
 
 
-def combine_tokens(x, W1, b1, W2, b2, route_, tokens=None, nthreads=0):
+def combine_tokens(x, W1, b1, W2, b2, route_, tokens=None, nthreads=0, flags=0):
     """Layer output for ``tokens`` (all when None) given a routing dict from :func:`route`.
 
     Returns ``(out_f64, out_x)``: the unrounded double result and the result in x's dtype."""
@@ -162,7 +165,7 @@ def combine_tokens(x, W1, b1, W2, b2, route_, tokens=None, nthreads=0):
     W1 = np.ascontiguousarray(W1)
     W2 = np.ascontiguousarray(W2)
     T, d = x.shape
-    E, F, _ = W1.shape
+    E, _, F = W2.shape
     ids, w, slot = (_c(route_["ids"], np.int32), _c(route_["w"], np.float32),
                     _c(route_["slot"], np.int32))
     k = ids.shape[1]
@@ -173,7 +176,7 @@ def combine_tokens(x, W1, b1, W2, b2, route_, tokens=None, nthreads=0):
     b2c = None if b2 is None else _c(b2, np.float32)
     rc = lib().oracle_combine_tokens(T, d, F, E, k, _dtype_code(x), _ptr(x), _ptr(W1), _ptr(b1c),
                                      _ptr(W2), _ptr(b2c), ids, w, slot, tok.size, tok, out64,
-                                     _ptr(outx), nthreads)
+                                     _ptr(outx), nthreads, int(flags))
     if rc != 0:
         raise ValueError("oracle_combine_tokens rejected its arguments")
     return out64, outx
@@ -185,8 +188,8 @@ def forward(x, Wr, br, W1, b1, W2, b2, k, C, tokens=None, logits_=None, nthreads
     E = W1.shape[0]
     L = logits(x, Wr, br, nthreads) if logits_ is None else _c(logits_, np.float32)
     K = capacity(T, E, k, C)
-    r = route(L, k, K, flags)
-    out64, outx = combine_tokens(x, W1, b1, W2, b2, r, tokens, nthreads)
+    r = route(L, k, K, flags & 3)
+    out64, outx = combine_tokens(x, W1, b1, W2, b2, r, tokens, nthreads, flags)
     return dict(logits=L, K=K, route=r, out_f64=out64, out=outx)
 
 

@@ -140,16 +140,24 @@ uint16_t bf16_from_double(double v) {
 
 // One expert FFN on one token (worked-example trace): h = W1 x + b1, a = SiLU(h) = h / (1 +
 // e^{-h}), y = W2 a + b2.  W1e is [F, d] and W2e is [d, F], row-major ("out x in").
+// gated (the fused-MoE dataflow diagram's "SiLU x mul" between GEMM 1 and GEMM 2): W1e is
+// [2F, d] and b1e [2F], rows [0, F) the gate g and rows [F, 2F) the up projection u, and
+// a = SiLU(g) * u.  h_out receives a.
 void expert_ffn(int d, int F, int dtype, const double* x, const void* W1, size_t w1_off,
                 const float* b1e, const void* W2, size_t w2_off, const float* b2e,
-                double* h_out, double* y) {
+                double* h_out, double* y, bool gated = false) {
     std::vector<double> a(F);
-    for (int f = 0; f < F; ++f) {
+    auto row_dot = [&](int row) {
         double h = 0.0;
-        for (int i = 0; i < d; ++i) h += load_elem(W1, w1_off + (size_t)f * d + i, dtype) * x[i];
-        if (b1e) h += (double)b1e[f];
-        if (h_out) h_out[f] = h;
-        a[f] = h / (1.0 + std::exp(-h));
+        for (int i = 0; i < d; ++i) h += load_elem(W1, w1_off + (size_t)row * d + i, dtype) * x[i];
+        if (b1e) h += (double)b1e[row];
+        return h;
+    };
+    for (int f = 0; f < F; ++f) {
+        const double g = row_dot(f);
+        const double silu = g / (1.0 + std::exp(-g));
+        a[f] = gated ? silu * row_dot(F + f) : silu;
+        if (h_out) h_out[f] = gated ? a[f] : g;
     }
     for (int o = 0; o < d; ++o) {
         double s = 0.0;
@@ -289,18 +297,21 @@ int oracle_dispatch(int T, int E, int k, const int32_t* ids, const int32_t* slot
 // Expert FFN outputs for a list of (token, expert) rows: Y[r] = W2e SiLU(W1e x_t + b1e) + b2e in
 // double; H[r] (optional) is the pre-activation h.  W1 is [E, F, d], W2 is [E, d, F] in x's
 // dtype; b1 [E, F], b2 [E, d] float or null.
+// flags bit 4: gated experts (W1 [E, 2F, d], b1 [E, 2F]).
 int oracle_expert_rows(int d, int F, int E, int dtype, const void* x, const void* W1,
                        const float* b1, const void* W2, const float* b2, int nrows,
                        const int32_t* row_tok, const int32_t* row_exp, double* Y, double* H,
-                       int nthreads) {
+                       int nthreads, int flags) {
     for (int r = 0; r < nrows; ++r) if (row_exp[r] < 0 || row_exp[r] >= E) return -1;
+    const bool gated = (flags & 4) != 0;
+    const size_t F1 = gated ? 2 * (size_t)F : (size_t)F;   // rows of W1 per expert
     parallel_for(nrows, nthreads, [&](int r) {
         int t = row_tok[r], e = row_exp[r];
         std::vector<double> xv(d);
         for (int i = 0; i < d; ++i) xv[i] = load_elem(x, (size_t)t * d + i, dtype);
-        expert_ffn(d, F, dtype, xv.data(), W1, (size_t)e * F * d, b1 ? b1 + (size_t)e * F : nullptr,
+        expert_ffn(d, F, dtype, xv.data(), W1, (size_t)e * F1 * d, b1 ? b1 + (size_t)e * F1 : nullptr,
                    W2, (size_t)e * d * F, b2 ? b2 + (size_t)e * d : nullptr,
-                   H ? H + (size_t)r * F : nullptr, Y + (size_t)r * d);
+                   H ? H + (size_t)r * F : nullptr, Y + (size_t)r * d, gated);
     });
     return 0;
 }
@@ -311,8 +322,11 @@ int oracle_expert_rows(int d, int F, int E, int dtype, const void* x, const void
 int oracle_combine_tokens(int T, int d, int F, int E, int k, int dtype, const void* x,
                           const void* W1, const float* b1, const void* W2, const float* b2,
                           const int32_t* ids, const float* w, const int32_t* slot, int ntok,
-                          const int32_t* tok, double* out_f64, void* out_x, int nthreads) {
+                          const int32_t* tok, double* out_f64, void* out_x, int nthreads,
+                          int flags) {
     for (int i = 0; i < ntok; ++i) if (tok[i] < 0 || tok[i] >= T) return -1;
+    const bool gated = (flags & 4) != 0;
+    const size_t F1 = gated ? 2 * (size_t)F : (size_t)F;
     parallel_for(ntok, nthreads, [&](int i) {
         int t = tok[i];
         std::vector<double> xv(d), y(d), s(d, 0.0);
@@ -322,9 +336,9 @@ int oracle_combine_tokens(int T, int d, int F, int E, int k, int dtype, const vo
             size_t pi = (size_t)t * k + j;
             if (slot[pi] < 0) continue;
             int e = ids[pi];
-            expert_ffn(d, F, dtype, xv.data(), W1, (size_t)e * F * d,
-                       b1 ? b1 + (size_t)e * F : nullptr, W2, (size_t)e * d * F,
-                       b2 ? b2 + (size_t)e * d : nullptr, nullptr, y.data());
+            expert_ffn(d, F, dtype, xv.data(), W1, (size_t)e * F1 * d,
+                       b1 ? b1 + (size_t)e * F1 : nullptr, W2, (size_t)e * d * F,
+                       b2 ? b2 + (size_t)e * d : nullptr, nullptr, y.data(), gated);
             for (int c = 0; c < d; ++c) s[c] += (double)w[pi] * y[c];
             any = true;
         }

@@ -83,10 +83,10 @@ def test_malformed_problems_rejected(moe, bad):
 
 def test_unknown_flags_rejected(moe):
     n = ctypes.c_size_t()
-    for bad in (4, 8, 0x80000000):
+    for bad in (8, 16, 0x80000000):
         p = moe.Problem(16, 64, 64, 4, 2, 1.0, 1, bad)
         assert moe.lib().moe_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 1
-    for good in (0, moe.FLAG_RENORMALIZE, moe.FLAG_ARRIVAL_ORDER, 3):
+    for good in (0, moe.FLAG_RENORMALIZE, moe.FLAG_ARRIVAL_ORDER, moe.FLAG_GATED, 7):
         p = moe.Problem(16, 64, 64, 4, 2, 1.0, 1, good)
         assert moe.lib().moe_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
 

@@ -197,7 +197,7 @@ def _forward_check(spec, seed, tokens=None, logit_rel=1e-4, flags=0):
     Lref = oracle.logits(L["x"], L["Wr"], L["br"])
     lerr = np.abs(g["logits_out"] - Lref).max()
     assert lerr <= logit_rel * max(1.0, float(np.abs(Lref).max())), lerr
-    ro = oracle.route(Lref, spec.k, layer.K, flags)
+    ro = oracle.route(Lref, spec.k, layer.K, flags & 3)
     # The logits differ from the oracle's by rounding, so the order of a token's experts can
     # differ where two of its top-k logits are that close; compare per (token, expert) pair.
     # Expert choice itself is pinned by the gap screen; capacity decisions may only differ where
@@ -223,7 +223,8 @@ def _forward_check(spec, seed, tokens=None, logit_rel=1e-4, flags=0):
     if tokens is None:
         tokens = np.arange(T, dtype=np.int32)
     tokens = np.array([t for t in tokens if agree[t]], dtype=np.int32)
-    _, ref = oracle.combine_tokens(L["x"], L["W1"], L["b1"], L["W2"], L["b2"], ro, tokens)
+    _, ref = oracle.combine_tokens(L["x"], L["W1"], L["b1"], L["W2"], L["b2"], ro, tokens,
+                                   flags=flags)
     got = to_host(out)
     assert_close(got[tokens], ref, spec.dtype, "layer output")
     none_kept = ~(ro["slot"] >= 0).any(axis=1) & agree
@@ -388,3 +389,47 @@ def test_bounded_wait_reports_timeout_and_gpu_stays_usable():
     assert moe.moe_get_device_status(layer.ws) == 0
     ro = oracle.route(L, 2, layer.K)
     assert np.array_equal(to_host(r["slot"]), ro["slot"])
+
+
+# ------------------------------------------------------------------------------------------
+# Gated experts (MOE_FLAG_GATED): H = SiLU(x W_gate^T + b_gate) * (x W_up^T + b_up).
+# ------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("T,d,F,E,k,C,dtype", [(300, 128, 256, 5, 2, 1.0, "bf16"),
+                                               (700, 256, 384, 3, 3, 0.9, "bf16"),
+                                               (40, 16, 24, 4, 2, 1.0, "f32")])
+def test_gated_expert_ffn_parity(T, d, F, E, k, C, dtype):
+    moe = _moe()
+    spec = inputs.LayerSpec("gffn", T, d, F, E, k, C, dtype, router="normal", router_bias=0.5,
+                            bias_std=0.05, gated=True)
+    L = inputs.make_layer(spec, seed=T + 1)
+    logits = oracle.logits(L["x"], L["Wr"], L["br"])
+    K = oracle.capacity(T, E, k, C)
+    ro = oracle.route(logits, k, K)
+    off_ref, rowtok_ref = oracle.dispatch(ro["ids"], ro["slot"], E)
+    n = int(off_ref[-1])
+    row_exp = np.repeat(np.arange(E, dtype=np.int32), np.diff(off_ref))
+    Yref = oracle.expert_rows(L["x"], L["W1"], L["b1"], L["W2"], L["b2"], rowtok_ref, row_exp,
+                              flags=oracle.GATED)
+    layer = moe.MoELayer(T, d, F, E, k, C, dtype, flags=moe.FLAG_GATED)
+    Y = layer.expert_ffn(to_dev(L["x"]), to_dev(off_ref), to_dev(rowtok_ref), to_dev(L["W1"]),
+                         to_dev(L["b1"]), to_dev(L["W2"]), to_dev(L["b2"]))
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(layer.ws) == 0
+    assert_close(to_host(Y)[:n], Yref, dtype, "gated expert outputs")
+
+
+@pytest.mark.parametrize("spec", [
+    inputs.LayerSpec("gf1", 1000, 256, 384, 8, 2, 1.0, "bf16", router="zipf", router_bias=1.1,
+                     bias_std=0.02, gated=True),
+    inputs.LayerSpec("gf2", 2500, 128, 128, 16, 4, 0.8, "bf16", router="normal",
+                     router_bias=0.5, gated=True)])
+def test_forward_gated(spec):
+    _forward_check(spec, seed=4, flags=4)
+
+
+def test_gated_needs_d_ff_multiple_of_128():
+    moe = _moe()
+    with pytest.raises(moe.MoeError) as ei:
+        moe.MoELayer(16, 64, 192, 4, 2, 1.0, "bf16", flags=moe.FLAG_GATED).forward(
+            *[torch.zeros(8, device="cuda")] * 7)
+    assert ei.value.status == 2

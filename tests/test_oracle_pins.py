@@ -445,3 +445,53 @@ def test_both_flags_compose():
     ra = oracle.route(L, k, K, oracle.ARRIVAL_ORDER)
     assert np.array_equal(r["w"].view(np.uint32), rn["w"].view(np.uint32))
     assert np.array_equal(r["slot"], ra["slot"])
+
+
+# ------------------------------------------------------------------------------------------
+# Gated experts (the dataflow diagram's GEMM 1 -> "SiLU x mul" -> GEMM 2): a = SiLU(g) * u.
+# ------------------------------------------------------------------------------------------
+
+def dense_gated_reference(layer, route):
+    x = torch.from_numpy(_f64(layer["x"]))
+    W1 = torch.from_numpy(_f64(layer["W1"]))
+    W2 = torch.from_numpy(_f64(layer["W2"]))
+    b1 = torch.from_numpy(layer["b1"].astype(np.float64))
+    b2 = torch.from_numpy(layer["b2"].astype(np.float64))
+    E, d, F = W2.shape
+    Y = []
+    for e in range(E):
+        h = Fnn.linear(x, W1[e], b1[e])
+        g, u = h[:, :F], h[:, F:]
+        Y.append(Fnn.linear(Fnn.silu(g) * u, W2[e], b2[e]))
+    Y = torch.stack(Y)
+    T, k = route["ids"].shape
+    out = x.clone()
+    for t in range(T):
+        for j in range(k):
+            if route["slot"][t, j] >= 0:
+                out[t] += float(route["w"][t, j]) * Y[route["ids"][t, j], t]
+    return out.numpy(), Y.numpy()
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T,d,F,E,k,C", [(24, 8, 16, 4, 1, 0.75), (40, 16, 12, 6, 2, 1.0)])
+def test_gated_forward_matches_dense_reference(dtype, T, d, F, E, k, C):
+    spec = inputs.LayerSpec("g", T, d, F, E, k, C, dtype, router="normal", router_bias=0.3,
+                            bias_std=0.1, gated=True)
+    layer = inputs.make_layer(spec, seed=T + F)
+    assert layer["W1"].shape == (E, 2 * F, d)
+    res = oracle.forward(layer["x"], layer["Wr"], layer["br"], layer["W1"], layer["b1"],
+                         layer["W2"], layer["b2"], k, C, flags=oracle.GATED)
+    ref, Y = dense_gated_reference(layer, res["route"])
+    np.testing.assert_allclose(res["out_f64"], ref, rtol=0, atol=1e-12)
+    offsets, rowtok = oracle.dispatch(res["route"]["ids"], res["route"]["slot"], E)
+    row_exp = np.repeat(np.arange(E, dtype=np.int32), np.diff(offsets))
+    Yo, Ho = oracle.expert_rows(layer["x"], layer["W1"], layer["b1"], layer["W2"], layer["b2"],
+                                rowtok, row_exp, want_h=True, flags=oracle.GATED)
+    np.testing.assert_allclose(Yo, Y[row_exp, rowtok], rtol=0, atol=1e-12)
+    # Zero up-projection -> zero expert output but the bias b2.
+    layer["W1"][:, F:, :] = 0
+    layer["b1"][:, F:] = 0
+    Yz = oracle.expert_rows(layer["x"], layer["W1"], layer["b1"], layer["W2"], layer["b2"],
+                            rowtok, row_exp, flags=oracle.GATED)
+    np.testing.assert_allclose(Yz, layer["b2"][row_exp].astype(np.float64), rtol=0, atol=0)
