@@ -56,6 +56,17 @@ def parse():
     return ap.parse_args()
 
 
+def max_over_ranks(value, dist=None, device=None):
+    """Largest per-rank value (times are taken as the slowest rank); identity on one rank."""
+    if dist is None or not dist.is_available() or not dist.is_initialized() or \
+            dist.get_world_size() == 1:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -318,11 +329,7 @@ def run_cuda(args):
         for s in range(moe.STAGE_EVENTS - 1):
             stage_ms[i, s] = evs[i][s].elapsed_time(evs[i][s + 1])
     step_ms = np.array([evs[i][0].elapsed_time(evs[i][-1]) for i in range(K)])
-    total_ms = float(step_ms.sum())
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(step_ms.sum()), dist if world > 1 else None, dev)
     ms_per_step = total_ms / K
     value = world * spec.T / (ms_per_step / 1e3)
 
@@ -365,11 +372,7 @@ def run_cuda(args):
     s_in.wait_event(d2h_done[K - 1])
     e1.record(s_in)
     e1.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
     e2e_value = world * spec.T / (e2e_ms / K / 1e3)
     # The last step's output must equal the device-timed path's output (same inputs).
     assert torch.equal(out_host[(K - 1) % 2], out.cpu()), "e2e output differs"

@@ -1,0 +1,53 @@
+"""The bench's multi-rank host path on CPU: two gloo ranks, slowest-rank timing, rank 0 prints.
+
+Each rank of ``bench.py --gpus N`` runs an independent batch (no collective on the data path);
+the only cross-rank steps are a barrier and the max over ranks of the device time.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        local = [3.0, 7.5][rank]
+        out[rank] = bench.max_over_ranks(local, dist)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_two_gloo_ranks():
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_rank_main, args=(2, 29517, out), nprocs=2, start_method="spawn")
+    assert out[0] == 7.5 and out[1] == 7.5
+
+
+def test_max_over_ranks_single_process_is_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(4.25) == 4.25
+
+
+@pytest.mark.slow
+def test_reference_arm_under_torchrun_prints_once():
+    # Rank 0 times the oracle and prints one JSON line; rank 1 exits 0 without work.
+    env = dict(os.environ)
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr", "127.0.0.1", "--master-port", "29519", "bench.py", "--impl",
+           "reference", "--gpus", "2", "--steps", "1", "--warmup", "0", "--config", "tiny_f32"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1 and '"impl": "reference"' in lines[0]
