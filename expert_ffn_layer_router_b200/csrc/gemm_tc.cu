@@ -11,13 +11,15 @@
 // Router logits: L = x . [Wr_hi | Wr_mid | Wr_lo] with Wr split exactly into three bf16 terms;
 // the epilogue adds the three fp32 partial products and the router bias.
 //
-// One persistent CTA per SM walks a static list of (expert, 128-row m-tile, BN-column n-tile)
-// tiles, n-tile fastest.  Warp roles (320 threads):
-//   warp 0      TMA producer for B (weights, K-major, 128-byte swizzle)
-//   warp 1      TMEM allocator and the single thread that issues tcgen05.mma
-//   warps 2-5   epilogue: tcgen05.ld from TMEM, bias + activation, bf16/fp32 stores
-//   warps 6-9   A producers: 16-byte cp.async of the 128 rows of the m-tile (gathered through
-//               rowtok for GEMM1) into the 128-byte-swizzled K-major layout
+// One persistent CTA per SM (or CTA pair per two SMs) walks a static list of (expert, m-tile,
+// BN-column n-tile) tiles, n-tile fastest.  Warp roles (448 threads):
+//   warp 0       TMA producer for B (weights, K-major, 128-byte swizzle), and for A when its
+//                rows are contiguous
+//   warp 1       TMEM allocator and the single thread that issues tcgen05.mma
+//   warps 2-9    epilogue: tcgen05.ld from TMEM, bias + activation, bf16 blocks staged in
+//                shared memory and written by TMA stores (fp32 stores for the router)
+//   warps 10-13  A producers when A is gathered: 16-byte cp.async of the m-tile's rows
+//                (through rowtok for GEMM1) into the 128-byte-swizzled K-major layout
 // Pipeline: STAGES shared-memory stages (full/empty mbarriers) and two TMEM accumulators
 // (tmem_full/tmem_empty) so the epilogue of tile i overlaps the main loop of tile i+1.
 // Every wait is bounded (about 2 s) and reports MOE_DEV_TIMEOUT instead of hanging.
@@ -205,6 +207,25 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
         : "memory");
 }
 
+// TMA tile store from shared memory (bulk-group completion) and its waits.
+__device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     tmap),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// The shared-memory sources of all committed stores have been read (the buffer may be reused).
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// All committed stores have completed.
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
     uint4 v;
     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
@@ -248,7 +269,8 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, const int* s_mt, int E
 template <int BN, int EPI, bool GATHER, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmD, const GemmArgs args) {
     using C = Cfg<BN, PAIR>;
     constexpr int S = C::kStages;
     constexpr int TM = C::kTileM;
@@ -288,6 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
         if (!GATHER) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
+        if (EPI == kEpiSiLU || EPI == kEpiBias || EPI == kEpiSwiGLU)
+            asm volatile("prefetch.tensormap [%0];" ::"l"(&tmD) : "memory");
     }
     if (warp == 1) {
         __syncwarp();
@@ -592,7 +616,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         pk[i >> 1] = pack_bf16x2(a0, a1);
                     }
-                    // Stage: this thread's row (= lane), nc/8 chunks of 16 bytes.
+                    // The previous block's TMA store must have read the staging buffer.
+                    if (lane == 0) bulk_wait_read_all();
+                    __syncwarp();
+                    // Stage: this thread's row (= lane), nc/8 chunks of 16 bytes.  The XOR of the
+                    // chunk index with (row / 2) % 4 is the tensor map's 64-byte swizzle.
                     const uint32_t rowp = stg + (uint32_t)lane * 64u;
                     const uint32_t sw = (uint32_t)((lane >> 1) & 3);
 #pragma unroll
@@ -600,6 +628,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (j < nc / 8)
                             st_shared_v4(rowp + ((j ^ sw) << 4), pk[4 * j], pk[4 * j + 1],
                                          pk[4 * j + 2], pk[4 * j + 3]);
+                    if (wrows == 32 && nc == 32) {
+                        // A whole 32 x 32 block of this group's rows: one TMA store.
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tmD, stg, n0 + c0, (int)wrow0);
+                            bulk_commit();
+                        }
+                        continue;
+                    }
+                    // A block that crosses the end of the group (the rows past it belong to the
+                    // next group) or a 16-column block: plain stores of the valid part.
                     __syncwarp();
                     // Copy out: lane handles chunk lane % 4 of rows lane / 4 + 8 i.
                     const int cc = lane & 3;
@@ -686,6 +726,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 
+    if (warp >= 2 && warp < 2 + kEpiWarps && lane == 0) bulk_wait_all();
     tc_fence_before();
     __syncwarp();
     if (PAIR) cluster_sync_all(); else __syncthreads();
@@ -758,6 +799,12 @@ bool make_tmap(CUtensorMap* tm, const void* ptr, long long rows, int K, int box_
     return make_tmap_2d(tm, ptr, rows, K, K, kBK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// Output map of the expert GEMMs: rows x cols bf16 (row pitch ld), 32 x 32 boxes with the
+// 64-byte swizzle of the epilogue's staging buffers.
+bool make_tmap_out(CUtensorMap* tm, const void* ptr, long long rows, int cols, long long ld) {
+    return make_tmap_2d(tm, ptr, rows, cols, ld, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
 int g_num_sms = 0;
 
 int num_sms() {
@@ -772,8 +819,8 @@ int num_sms() {
 
 // The dynamic shared-memory attribute is per device; remember which devices have it.
 template <int BN, int EPI, bool GATHER, bool PAIR>
-cudaError_t launch_gemm_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
-                          long long tiles, cudaStream_t s) {
+cudaError_t launch_gemm_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,
+                          const GemmArgs& a, long long tiles, cudaStream_t s) {
     using C = Cfg<BN, PAIR>;
     auto kern = grouped_gemm_kernel<BN, EPI, GATHER, PAIR>;
     static std::atomic<uint64_t> attr_done{0};
@@ -806,7 +853,7 @@ cudaError_t launch_gemm_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const 
     }
     if (!PAIR) {
         const int grid = (int)std::min<long long>(num_sms(), std::max<long long>(tiles, 1));
-        kern<<<grid, kThreads, C::kSmemBytes, s>>>(tmA, tmB, a);
+        kern<<<grid, kThreads, C::kSmemBytes, s>>>(tmA, tmB, tmD, a);
         return cudaGetLastError();
     }
     const int clusters =
@@ -823,17 +870,18 @@ cudaError_t launch_gemm_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const 
     cfg.stream = s;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, a);
+    return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmD, a);
 }
 
 template <int EPI, bool GATHER, bool PAIR>
 cudaError_t launch_gemm_bn(int BN, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                           const GemmArgs& a, long long tiles, cudaStream_t s) {
+                           const CUtensorMap& tmD, const GemmArgs& a, long long tiles,
+                           cudaStream_t s) {
     switch (BN) {
-        case 256: return launch_gemm_t<256, EPI, GATHER, PAIR>(tmA, tmB, a, tiles, s);
-        case 192: return launch_gemm_t<192, EPI, GATHER, PAIR>(tmA, tmB, a, tiles, s);
-        case 176: return launch_gemm_t<176, EPI, GATHER, PAIR>(tmA, tmB, a, tiles, s);
-        case 128: return launch_gemm_t<128, EPI, GATHER, PAIR>(tmA, tmB, a, tiles, s);
+        case 256: return launch_gemm_t<256, EPI, GATHER, PAIR>(tmA, tmB, tmD, a, tiles, s);
+        case 192: return launch_gemm_t<192, EPI, GATHER, PAIR>(tmA, tmB, tmD, a, tiles, s);
+        case 176: return launch_gemm_t<176, EPI, GATHER, PAIR>(tmA, tmB, tmD, a, tiles, s);
+        case 128: return launch_gemm_t<128, EPI, GATHER, PAIR>(tmA, tmB, tmD, a, tiles, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -842,9 +890,9 @@ template <int EPI>
 cudaError_t launch_router_bn(int BN, const CUtensorMap& tmA, const CUtensorMap& tmB,
                              const GemmArgs& a, long long tiles, cudaStream_t s) {
     switch (BN) {
-        case 192: return launch_gemm_t<192, EPI, false, false>(tmA, tmB, a, tiles, s);
-        case 96: return launch_gemm_t<96, EPI, false, false>(tmA, tmB, a, tiles, s);
-        case 48: return launch_gemm_t<48, EPI, false, false>(tmA, tmB, a, tiles, s);
+        case 192: return launch_gemm_t<192, EPI, false, false>(tmA, tmB, tmB, a, tiles, s);
+        case 96: return launch_gemm_t<96, EPI, false, false>(tmA, tmB, tmB, a, tiles, s);
+        case 48: return launch_gemm_t<48, EPI, false, false>(tmA, tmB, tmB, a, tiles, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -936,19 +984,21 @@ cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const in
     const bool gather = a_rows != nullptr;
     if (!gather && !make_tmap(&tmA, A, (long long)a_row_limit, K, kBM))
         return cudaErrorInvalidValue;
+    CUtensorMap tmD;
+    if (!make_tmap_out(&tmD, D, max_rows, Nout, ldd)) return cudaErrorInvalidValue;
     cudaError_t e;
     if (gather && pair) {
-        e = which == 0 ? launch_gemm_bn<kEpiSiLU, true, true>(BN, tmA, tm, a, max_tiles, s)
-                       : launch_gemm_bn<kEpiBias, true, true>(BN, tmA, tm, a, max_tiles, s);
+        e = which == 0 ? launch_gemm_bn<kEpiSiLU, true, true>(BN, tmA, tm, tmD, a, max_tiles, s)
+                       : launch_gemm_bn<kEpiBias, true, true>(BN, tmA, tm, tmD, a, max_tiles, s);
     } else if (gather) {
-        e = which == 0 ? launch_gemm_bn<kEpiSiLU, true, false>(BN, tmA, tm, a, max_tiles, s)
-                       : launch_gemm_bn<kEpiBias, true, false>(BN, tmA, tm, a, max_tiles, s);
+        e = which == 0 ? launch_gemm_bn<kEpiSiLU, true, false>(BN, tmA, tm, tmD, a, max_tiles, s)
+                       : launch_gemm_bn<kEpiBias, true, false>(BN, tmA, tm, tmD, a, max_tiles, s);
     } else if (pair) {
-        e = which == 0 ? launch_gemm_bn<kEpiSiLU, false, true>(BN, tmA, tm, a, max_tiles, s)
-                       : launch_gemm_bn<kEpiBias, false, true>(BN, tmA, tm, a, max_tiles, s);
+        e = which == 0 ? launch_gemm_bn<kEpiSiLU, false, true>(BN, tmA, tm, tmD, a, max_tiles, s)
+                       : launch_gemm_bn<kEpiBias, false, true>(BN, tmA, tm, tmD, a, max_tiles, s);
     } else {
-        e = which == 0 ? launch_gemm_bn<kEpiSiLU, false, false>(BN, tmA, tm, a, max_tiles, s)
-                       : launch_gemm_bn<kEpiBias, false, false>(BN, tmA, tm, a, max_tiles, s);
+        e = which == 0 ? launch_gemm_bn<kEpiSiLU, false, false>(BN, tmA, tm, tmD, a, max_tiles, s)
+                       : launch_gemm_bn<kEpiBias, false, false>(BN, tmA, tm, tmD, a, max_tiles, s);
     }
     if (e == cudaSuccess) *launches += 1;
     return e;
@@ -984,15 +1034,17 @@ cudaError_t launch_gated_gemm(const void* A, long long lda, const int32_t* a_row
     const bool gather = a_rows != nullptr;
     if (!gather && !make_tmap(&tmA, A, (long long)a_row_limit, K, kBM))
         return cudaErrorInvalidValue;
+    CUtensorMap tmD;
+    if (!make_tmap_out(&tmD, D, max_rows, F, ldd)) return cudaErrorInvalidValue;
     cudaError_t e;
     if (gather && pair)
-        e = launch_gemm_t<256, kEpiSwiGLU, true, true>(tmA, tm, a, max_tiles, s);
+        e = launch_gemm_t<256, kEpiSwiGLU, true, true>(tmA, tm, tmD, a, max_tiles, s);
     else if (gather)
-        e = launch_gemm_t<256, kEpiSwiGLU, true, false>(tmA, tm, a, max_tiles, s);
+        e = launch_gemm_t<256, kEpiSwiGLU, true, false>(tmA, tm, tmD, a, max_tiles, s);
     else if (pair)
-        e = launch_gemm_t<256, kEpiSwiGLU, false, true>(tmA, tm, a, max_tiles, s);
+        e = launch_gemm_t<256, kEpiSwiGLU, false, true>(tmA, tm, tmD, a, max_tiles, s);
     else
-        e = launch_gemm_t<256, kEpiSwiGLU, false, false>(tmA, tm, a, max_tiles, s);
+        e = launch_gemm_t<256, kEpiSwiGLU, false, false>(tmA, tm, tmD, a, max_tiles, s);
     if (e == cudaSuccess) *launches += 1;
     return e;
 }
