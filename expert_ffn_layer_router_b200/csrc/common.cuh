@@ -71,19 +71,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Waits for the phase of parity `parity` to complete.  Gives up after kWaitLimitNs, or as soon
-// as another thread has recorded an error, and then returns false after recording a timeout.
+// Waits for the phase of parity `parity` to complete.  Gives up after kWaitLimitNs, or once
+// another thread has recorded an error, and then returns false after recording a timeout.  The
+// status word and the clock are read only every 32nd retry, so that a waiting thread is back in
+// try_wait (not in a global load) when the phase completes.
 template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, DeviceStatus* st,
                                           int where, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait<kCluster>(bar, parity)) return true;
     const uint64_t t0 = global_ns();
-    while (true) {
+    for (uint32_t n = 1;; ++n) {
         if (mbar_try_wait<kCluster>(bar, parity)) return true;
-        if (*reinterpret_cast<volatile int32_t*>(&st->code) != 0) return false;
-        if (global_ns() - t0 > limit_ns) {
-            report(st, MOE_DEV_TIMEOUT, where);
-            return false;
+        if ((n & 31u) == 0) {
+            if (*reinterpret_cast<volatile int32_t*>(&st->code) != 0) return false;
+            if (global_ns() - t0 > limit_ns) {
+                report(st, MOE_DEV_TIMEOUT, where);
+                return false;
+            }
         }
     }
 }

@@ -283,6 +283,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
     auto tfull_bar = [&](int b) { return bar0 + 8u * (3 * S + b); };
     auto tempty_bar = [&](int b) { return bar0 + 8u * (3 * S + 2 + b); };
+    // Gathered A on pairs: the peer CTA's copies complete on its own barrier first.
+    auto pfull_bar = [&](int s) { return bar0 + 8u * (2 * S + s); };
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base_ptr + C::kBarOff + 8 * (3 * S + 4));
     int* s_mt = reinterpret_cast<int*>(base_ptr + C::kTableOff);
     auto sA = [&](int s) { return base + (uint32_t)s * C::kABytes; };
@@ -298,10 +300,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < S; ++s) {
-            // producer arrive + expected bytes; gathered rows add one arrival per A thread
-            // (of both CTAs for a pair: the leader's threads locally, the peer's remotely)
-            mbar_init(full_bar(s), GATHER ? 1 + (PAIR ? 256 : 128) : 1);
+            // producer arrive + expected bytes; gathered rows add one arrival per A thread of
+            // this CTA, and for a pair one relayed arrival for all of the peer's rows
+            mbar_init(full_bar(s), GATHER ? 1 + 128 + (PAIR ? 1 : 0) : 1);
             mbar_init(empty_bar(s), 1);
+            if (GATHER && PAIR) mbar_init(pfull_bar(s), 128);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar(b), 1);
@@ -362,6 +365,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int total = s_mt[E] * n_tiles;
     const int nkb = args.K / kBK;
     constexpr uint32_t kIdesc = idesc_bf16(TM, BN);
+    // A last column tile with at most BN/2 valid columns (d_ff = 1408 on 256-wide tiles) runs
+    // N = BN/2 MMAs: the padded half is neither multiplied nor read back.  (Not on pairs, whose
+    // CTAs each hold one half of the tile's B rows.)
+    constexpr bool kHalfOk =
+        (EPI == kEpiSiLU || EPI == kEpiBias) && !PAIR && (BN / 2) % 16 == 0;
+    constexpr uint32_t kIdescHalf = idesc_bf16(TM, kHalfOk ? BN / 2 : BN);
+    const bool last_half = kHalfOk && (n_tiles * BN - args.Nout) >= BN / 2;
     // Barriers of the pair's leader that both CTAs signal.
     auto lead = [&](uint32_t addr) { return PAIR ? map_to_cta(addr, 0) : addr; };
 
@@ -416,6 +426,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait<PAIR>(tempty_bar(b), (use & 1u) ^ 1u, st, 2)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + b * 256u;
+                const uint32_t idesc =
+                    (last_half && tile % n_tiles == n_tiles - 1) ? kIdescHalf : kIdesc;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1u;
@@ -427,16 +439,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
                         if (PAIR)
-                            tc_mma_bf16_pair(d_tmem, da + 2u * kk, db + 2u * kk, kIdesc,
+                            tc_mma_bf16_pair(d_tmem, da + 2u * kk, db + 2u * kk, idesc,
                                              (kb | kk) != 0 ? 1u : 0u);
                         else
-                            tc_mma_bf16(d_tmem, da + 2u * kk, db + 2u * kk, kIdesc,
+                            tc_mma_bf16(d_tmem, da + 2u * kk, db + 2u * kk, idesc,
                                         (kb | kk) != 0 ? 1u : 0u);
                     }
                     if (PAIR) tc_commit_pair(empty_bar(s)); else tc_commit(empty_bar(s));
                 }
                 if (!ok) break;
                 if (PAIR) tc_commit_pair(tfull_bar(b)); else tc_commit(tfull_bar(b));
+            }
+        } else if (GATHER && PAIR && lane == 0) {
+            // Relay of the peer CTA: once all of its gathered rows of a stage have landed, make
+            // them visible to the tensor cores and count them on the leader's full barrier.
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = cid; ok && tile < total; tile += ncl) {
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1u;
+                    if (!mbar_wait<false>(pfull_bar(s), ph, st, 6)) { ok = false; break; }
+                    fence_proxy_async_smem();
+                    mbar_arrive_cluster(lead(full_bar(s)));
+                }
             }
         }
     } else if (warp < 2 + kEpiWarps) {
@@ -582,11 +608,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int ncol = (kOut - c0) >= 32 ? 32 : 16;
                     float v[32];
                     float u[32];
+                    // warp-uniform: columns past the group's width (padding) or no rows
+                    if (n0 + c0 >= args.Nout || wrows == 0) continue;
                     __syncwarp();
                     if (ncol == 32) tmem_ld32_wait(taddr + c0, v);
                     else tmem_ld16_wait(taddr + c0, v);
                     if (EPI == kEpiSwiGLU) tmem_ld32_wait(taddr + 128 + c0, u);
-                    if (n0 + c0 >= args.Nout || wrows == 0) continue;
                     const int nc = min(ncol, args.Nout - (n0 + c0));     // 16 or 32
                     if (bias) {
 #pragma unroll
@@ -667,16 +694,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         // stage's full barrier when they have landed (cp.async.mbarrier.arrive.noinc), so all
         // stages can be in flight at once and no producer thread ever blocks on its own copies.
         // The MMA thread makes the landed rows visible to the tensor cores with a proxy fence.
-        // The peer CTA of a pair cannot arrive asynchronously on the leader's barrier, so each
-        // of its threads waits for its own copies with kLag stages still in flight, fences them
-        // for the tensor cores and arrives on the leader's barrier itself.
-        constexpr int kLag = S - 3 > 1 ? S - 3 : 1;
+        // The peer CTA of a pair cannot arrive asynchronously on the leader's barrier: its
+        // copies arrive on its own pfull barrier, and its relay thread forwards the stage.
         const bool remote = PAIR && !leader;
         const int at = threadIdx.x - 32 * (2 + kEpiWarps);   // 0..127
         const int chunk = at & 7;                             // 16-byte chunk of the row
         const int rbase = at >> 3;                            // rows rbase + 16 i
-        uint32_t it = 0, arrived = 0;
+        // The row indices of the CTA's next tile are loaded early in the current one, so that
+        // the first copies of the next tile do not wait on them.
+        uint32_t it = 0;
         bool ok = true;
+        bool have_next = false;
+        int nidx[8];
         for (int tile = cid; ok && tile < total; tile += ncl) {
             const TileCoord tc = tile_coord<TM>(tile, s_mt, E, n_tiles, args, (int)crank);
             const __nv_bfloat16* src[8];
@@ -686,18 +715,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 8; ++i) {
                 const int r = rbase + 16 * i;
                 valid[i] = r < tc.rows;
-                long long ar = tc.row0 + r;
+                long long ar = 0;
                 if (valid[i]) {
-                    const int g = __ldg(args.a_rows + tc.row0 + r);
+                    const int g = have_next ? nidx[i] : __ldg(args.a_rows + tc.row0 + r);
                     if ((unsigned)g >= (unsigned)args.a_row_limit) {
                         report(st, MOE_DEV_BAD_INDEX, 501);
                         valid[i] = false;
+                    } else {
+                        ar = g;
                     }
-                    ar = g;
                 }
                 src[i] = args.A + ar * args.lda + chunk * 8;
                 dst_off[i] = (uint32_t)r * 128u + (uint32_t)((chunk ^ (r & 7)) << 4);
             }
+            const int next = tile + ncl;
+            TileCoord nc{0, 0, 0, 0};
+            if (next < total) nc = tile_coord<TM>(next, s_mt, E, n_tiles, args, (int)crank);
+            have_next = false;
             for (int kb = 0; kb < nkb; ++kb, ++it) {
                 const int s = it % S;
                 const uint32_t ph = (it / S) & 1u;
@@ -706,24 +740,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
                     if (valid[i]) cp_async_16(dA + dst_off[i], src[i] + kb * kBK);
-                if (!remote) {
-                    cp_async_arrive_noinc(full_bar(s));
-                } else {
-                    cp_async_commit();
-                    if (it + 1 - arrived > (uint32_t)kLag) {
-                        cp_async_wait<kLag>();
-                        fence_proxy_async_smem();
-                        mbar_arrive_cluster(lead(full_bar(arrived % S)));
-                        ++arrived;
+                cp_async_arrive_noinc(remote ? pfull_bar(s) : full_bar(s));
+                if (kb == 0 && next < total) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int r = rbase + 16 * i;
+                        nidx[i] = r < nc.rows ? __ldg(args.a_rows + nc.row0 + r) : 0;
                     }
+                    have_next = true;
                 }
             }
         }
+        cp_async_commit();     // no copy of this thread may still be in flight at exit
         cp_async_wait<0>();
-        if (remote && ok) {
-            fence_proxy_async_smem();
-            for (; arrived < it; ++arrived) mbar_arrive_cluster(lead(full_bar(arrived % S)));
-        }
     }
 
     if (warp >= 2 && warp < 2 + kEpiWarps && lane == 0) bulk_wait_all();
