@@ -235,6 +235,16 @@ def to_dev(a, torch, dev):
     return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
 
 
+def kernel_source_hash():
+    """sha256[:16] over the GEMM kernel's sources (gemm_tc.cu, then common.cuh)."""
+    csrc = os.path.join(ROOT, "expert_ffn_layer_router_b200", "csrc")
+    h = hashlib.sha256()
+    for name in ("gemm_tc.cu", "common.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def traffic_record(kernel):
     """dram bytes per launch from the committed ncu summary, if taken on the current source."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -242,8 +252,7 @@ def traffic_record(kernel):
         return None
     with open(path) as f:
         rec = json.load(f)
-    src = os.path.join(ROOT, "expert_ffn_layer_router_b200", "csrc", "gemm_tc.cu")
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    h = kernel_source_hash()
     r = rec.get(kernel)
     if not r or r.get("source_sha256_16") != h:
         return None
