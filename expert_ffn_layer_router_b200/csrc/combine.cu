@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(256) combine_kernel(
     const int32_t* __restrict__ ids, const int32_t* __restrict__ slot,
     const int32_t* __restrict__ offsets, int T, int d, int E, int k, void* __restrict__ out,
     DeviceStatus* st) {
+    pdl_begin();
     constexpr int V = Tr::kVec;
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -143,6 +144,7 @@ __global__ void __launch_bounds__(256) combine_vec_kernel(
     const int32_t* __restrict__ ids, const int32_t* __restrict__ slot,
     const int32_t* __restrict__ offsets, int T, int nv, int E, int k, uint4* __restrict__ out,
     DeviceStatus* st) {
+    pdl_begin();
     constexpr int V = Tr::kVec;
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -215,6 +217,7 @@ __global__ void __launch_bounds__(256) combine_token_block_kernel(
     const int32_t* __restrict__ ids, const int32_t* __restrict__ slot,
     const int32_t* __restrict__ offsets, int nv, int E, int k, uint4* __restrict__ out,
     DeviceStatus* st) {
+    pdl_begin();
     constexpr int V = Tr::kVec;
     __shared__ int s_rows[KMAX];
     __shared__ float s_w[KMAX];
@@ -289,6 +292,7 @@ __global__ void __launch_bounds__(256) ffn_f32_kernel(
     const float* __restrict__ W1, const float* __restrict__ b1, const float* __restrict__ W2,
     const float* __restrict__ b2, float* __restrict__ H, float* __restrict__ Y,
     DeviceStatus* st, int gated) {
+    pdl_begin();
     extern __shared__ float s_mem[];
     float* xs = s_mem;          // [d]
     float* as = s_mem + d;      // [F]
@@ -339,6 +343,7 @@ __global__ void __launch_bounds__(256) ffn_f32_kernel(
 __global__ void logits_f32_kernel(const float* __restrict__ x, const float* __restrict__ Wr,
                                   const float* __restrict__ br, int T, int d, int E,
                                   float* __restrict__ L) {
+    pdl_begin();
     const long long n = (long long)T * E;
     for (long long q = blockIdx.x * (long long)blockDim.x + threadIdx.x; q < n;
          q += (long long)gridDim.x * blockDim.x) {
@@ -356,7 +361,7 @@ void launch_logits_f32(const float* x, const float* Wr, const float* br, int T, 
     const long long n = (long long)T * E;
     if (n == 0) return;
     const int blocks = (int)std::min<long long>((n + 255) / 256, 148 * 8);
-    logits_f32_kernel<<<blocks, 256, 0, s>>>(x, Wr, br, T, d, E, logits);
+    launch_pdl(logits_f32_kernel, dim3(blocks), dim3(256), 0, s, x, Wr, br, T, d, E, logits);
     *launches += 1;
 }
 
@@ -370,32 +375,33 @@ void launch_combine(int dtype, const void* x, const void* Y, const float* w, con
     if (dtype == MOE_BF16 && aligned && d % 8 == 0 && k <= 8 && T < 4 * 148) {
         const int nv = d / 8;
         const int threads = std::min(256, ((nv + 31) / 32) * 32);
-        combine_token_block_kernel<BF16Traits, 8><<<T, threads, 0, s>>>(
-            (const uint4*)x, (const uint4*)Y, w, ids, slot, offsets, nv, E, k, (uint4*)out, st);
+        launch_pdl(combine_token_block_kernel<BF16Traits, 8>, dim3(T), dim3(threads), 0, s,
+                   (const uint4*)x, (const uint4*)Y, w, ids, slot, offsets, nv, E, k, (uint4*)out,
+                   st);
         *launches += 1;
         return;
     }
     if (dtype == MOE_BF16 && aligned && d % 8 == 0 && k <= 8) {
-        combine_vec_kernel<BF16Traits, 8><<<blocks, 256, 0, s>>>(
-            (const uint4*)x, (const uint4*)Y, w, ids, slot, offsets, T, d / 8, E, k, (uint4*)out,
-            st);
+        launch_pdl(combine_vec_kernel<BF16Traits, 8>, dim3(blocks), dim3(256), 0, s,
+                   (const uint4*)x, (const uint4*)Y, w, ids, slot, offsets, T, d / 8, E, k,
+                   (uint4*)out, st);
         *launches += 1;
         return;
     }
     if (dtype == MOE_BF16) {
         if (aligned && d % 8 == 0)
-            combine_kernel<BF16Traits, true><<<blocks, 256, 0, s>>>(x, Y, w, ids, slot, offsets,
-                                                                    T, d, E, k, out, st);
+            launch_pdl(combine_kernel<BF16Traits, true>, dim3(blocks), dim3(256), 0, s, x, Y, w,
+                       ids, slot, offsets, T, d, E, k, out, st);
         else
-            combine_kernel<BF16Traits, false><<<blocks, 256, 0, s>>>(x, Y, w, ids, slot, offsets,
-                                                                     T, d, E, k, out, st);
+            launch_pdl(combine_kernel<BF16Traits, false>, dim3(blocks), dim3(256), 0, s, x, Y, w,
+                       ids, slot, offsets, T, d, E, k, out, st);
     } else {
         if (aligned && d % 4 == 0)
-            combine_kernel<F32Traits, true><<<blocks, 256, 0, s>>>(x, Y, w, ids, slot, offsets,
-                                                                   T, d, E, k, out, st);
+            launch_pdl(combine_kernel<F32Traits, true>, dim3(blocks), dim3(256), 0, s, x, Y, w, ids,
+                       slot, offsets, T, d, E, k, out, st);
         else
-            combine_kernel<F32Traits, false><<<blocks, 256, 0, s>>>(x, Y, w, ids, slot, offsets,
-                                                                    T, d, E, k, out, st);
+            launch_pdl(combine_kernel<F32Traits, false>, dim3(blocks), dim3(256), 0, s, x, Y, w,
+                       ids, slot, offsets, T, d, E, k, out, st);
     }
     *launches += 1;
 }
@@ -406,8 +412,8 @@ void launch_ffn_f32(const float* x, const int32_t* rowtok, const int32_t* offset
                     cudaStream_t s, int* launches, bool gated) {
     if (max_rows <= 0) return;
     const size_t smem = sizeof(float) * ((size_t)d + F);
-    ffn_f32_kernel<<<(unsigned)max_rows, 256, smem, s>>>(x, rowtok, offsets, E, T, d, F, W1, b1,
-                                                         W2, b2, H, Y, st, gated ? 1 : 0);
+    launch_pdl(ffn_f32_kernel, dim3((unsigned)max_rows), dim3(256), smem, s, x, rowtok, offsets, E,
+               T, d, F, W1, b1, W2, b2, H, Y, st, gated ? 1 : 0);
     *launches += 1;
 }
 

@@ -185,6 +185,35 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
            | ((uint32_t)(m >> 4) << 24);   // M / 16
 }
 
+// ---------------------------------------------------------------------------------------------
+// Programmatic dependent launch.  Every kernel starts with pdl_begin(): it waits until the
+// preceding grid in the stream has completed and its memory is visible (a no-op without a
+// programmatic dependency), then lets the next grid be scheduled, whose blocks in turn park in
+// their own wait.  So no kernel touches global memory before its predecessor is done, and a
+// dependent launch overlaps only its scheduling and set-up with the tail of the previous grid.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_begin() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// <<<grid, block, smem, s>>> with the programmatic-stream-serialization attribute.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);

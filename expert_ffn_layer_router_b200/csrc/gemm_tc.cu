@@ -271,6 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmD, const GemmArgs args) {
+    pdl_begin();
     using C = Cfg<BN, PAIR>;
     constexpr int S = C::kStages;
     constexpr int TM = C::kTileM;
@@ -771,6 +772,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // nt*3Eg + {0, Eg, 2Eg} + c hold the hi/mid/lo bf16 terms of Wr[:, nt*Eg + c] (zero past E).
 __global__ void router_split_kernel(const float* __restrict__ Wr, int d, int E, int Eg, int ntl,
                                     __nv_bfloat16* __restrict__ B) {
+    pdl_begin();
     const long long total = (long long)ntl * 3 * Eg * d;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
          i += (long long)gridDim.x * blockDim.x) {
@@ -882,7 +884,7 @@ cudaError_t launch_gemm_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const 
     }
     if (!PAIR) {
         const int grid = (int)std::min<long long>(num_sms(), std::max<long long>(tiles, 1));
-        kern<<<grid, kThreads, C::kSmemBytes, s>>>(tmA, tmB, tmD, a);
+        launch_pdl(kern, dim3(grid), dim3(kThreads), C::kSmemBytes, s, tmA, tmB, tmD, a);
         return cudaGetLastError();
     }
     const int clusters =
@@ -897,8 +899,11 @@ cudaError_t launch_gemm_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const 
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = s;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
+    cudaLaunchAttribute at2[2] = {at[0], {}};
+    at2[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at2[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at2;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmD, a);
 }
 
@@ -1091,8 +1096,8 @@ cudaError_t launch_router_gemm(const void* x, int T, int d, const float* Wr, con
     const int ntl = (E + Eg - 1) / Eg;
     const int BN = 3 * Eg;
     const bool fuse = fused != nullptr && ntl == 1;
-    router_split_kernel<<<148 * 4, 256, 0, s>>>(Wr, d, E, Eg, ntl,
-                                                reinterpret_cast<__nv_bfloat16*>(split_buf));
+    launch_pdl(router_split_kernel, dim3(148 * 4), dim3(256), 0, s, Wr, d, E, Eg, ntl,
+               reinterpret_cast<__nv_bfloat16*>(split_buf));
     *launches += 1;
     CUtensorMap tm;
     if (!make_tmap(&tm, split_buf, (long long)ntl * BN, d, BN)) return cudaErrorInvalidValue;

@@ -104,6 +104,7 @@ template <int EPL>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T,
                                                          int E, int k, int32_t* __restrict__ ids,
                                                          float* __restrict__ w, unsigned flags) {
+    pdl_begin();
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T) return;
     route_token_warp<EPL>(logits + (size_t)t * E, E, k, (size_t)t, ids, w, flags);
@@ -119,6 +120,7 @@ __global__ void __launch_bounds__(1024) router_small_kernel(
     const __nv_bfloat16* __restrict__ x, const float* __restrict__ Wr,
     const float* __restrict__ br, int T, int d, int E, int k, float* __restrict__ logits_out,
     int32_t* __restrict__ ids, float* __restrict__ w, unsigned flags) {
+    pdl_begin();
     extern __shared__ float s_x[];                    // [d]
     __shared__ float s_part[1024];
     __shared__ float s_L[256];
@@ -167,6 +169,7 @@ __global__ void __launch_bounds__(128) count_chunks_kernel(const int32_t* __rest
                                                            int E, int k, int nC,
                                                            int32_t* __restrict__ cnt,
                                                            DeviceStatus* st) {
+    pdl_begin();
     extern __shared__ int32_t s_cnt[];                 // [4][E]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int32_t* my = s_cnt + warp * E;
@@ -217,6 +220,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
 __global__ void __launch_bounds__(256) scan_chunks_kernel(const int32_t* __restrict__ cnt, int nC,
                                                           int32_t* __restrict__ base,
                                                           int32_t* __restrict__ nrecv) {
+    pdl_begin();
     __shared__ int s_warp[32];
     const int e = blockIdx.x;
     const int32_t* in = cnt + (size_t)e * nC;
@@ -238,6 +242,7 @@ __global__ void __launch_bounds__(128) scatter_chunks_kernel(const int32_t* __re
                                                              int T, int E, int k, int nC,
                                                              const int32_t* __restrict__ base,
                                                              int32_t* __restrict__ cand) {
+    pdl_begin();
     extern __shared__ int32_t s_run[];                 // [4][E]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x * 4 + warp;
@@ -277,6 +282,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     const float* __restrict__ w, int T, int E, int k, long long K, int32_t* __restrict__ slot,
     uint8_t* __restrict__ drop, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
     int32_t* __restrict__ rowtok, unsigned flags) {
+    pdl_begin();
     extern __shared__ uint32_t s_keys[];              // [kSelSmemKeys]
     __shared__ int s_warp[32];
     __shared__ int s_hist[256];
@@ -417,6 +423,7 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(
     long long K, unsigned flags, int32_t* __restrict__ slot, uint8_t* __restrict__ drop,
     int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ rowtok,
     DeviceStatus* st) {
+    pdl_begin();
     extern __shared__ int32_t sm[];
     __shared__ int s_warp[32];
     const int P = T * k;
@@ -517,6 +524,7 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(
 __global__ void kept_count_kernel(const int32_t* __restrict__ ids,
                                   const int32_t* __restrict__ slot, long long P, int E, int T,
                                   int32_t* __restrict__ kept, DeviceStatus* st) {
+    pdl_begin();
     for (long long p = blockIdx.x * (long long)blockDim.x + threadIdx.x; p < P;
          p += (long long)gridDim.x * blockDim.x) {
         const int s = slot[p];
@@ -529,6 +537,7 @@ __global__ void kept_count_kernel(const int32_t* __restrict__ ids,
 
 __global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict__ kept, int E,
                                                        int32_t* __restrict__ offsets) {
+    pdl_begin();
     __shared__ int s_warp[32];
     int carry = 0;
     for (int e0 = 0; e0 < E; e0 += blockDim.x) {
@@ -546,6 +555,7 @@ __global__ void rowtok_scatter_kernel(const int32_t* __restrict__ ids,
                                       const int32_t* __restrict__ slot, long long P, int E, int k,
                                       const int32_t* __restrict__ offsets,
                                       int32_t* __restrict__ rowtok, DeviceStatus* st) {
+    pdl_begin();
     for (long long p = blockIdx.x * (long long)blockDim.x + threadIdx.x; p < P;
          p += (long long)gridDim.x * blockDim.x) {
         const int s = slot[p];
@@ -563,6 +573,7 @@ template <typename V>
 __global__ void permute_rows_kernel(const V* __restrict__ x, const int32_t* __restrict__ rowtok,
                                     const int32_t* __restrict__ offsets, int E, int vpr, int T,
                                     V* __restrict__ xp, DeviceStatus* st) {
+    pdl_begin();
     const int rows = offsets[E];
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < (long long)rows * vpr;
          i += (long long)gridDim.x * blockDim.x) {
@@ -577,7 +588,8 @@ template <int EPL>
 void launch_route_t(const float* logits, int T, int E, int k, int32_t* ids, float* w,
                     cudaStream_t s, unsigned flags) {
     const int blocks = (T + 7) / 8;
-    route_topk_kernel<EPL><<<blocks, 256, 0, s>>>(logits, T, E, k, ids, w, flags);
+    launch_pdl(route_topk_kernel<EPL>, dim3(blocks), dim3(256), 0, s, logits, T, E, k, ids, w,
+               flags);
 }
 
 }  // namespace
@@ -606,13 +618,17 @@ void launch_router_small(const void* x, const float* Wr, const float* br, int T,
     const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
     const int epl = (E + 31) / 32;
     if (epl <= 1)
-        router_small_kernel<1><<<T, 1024, smem, s>>>(xb, Wr, br, T, d, E, k, logits_out, ids, w, flags);
+        launch_pdl(router_small_kernel<1>, dim3(T), dim3(1024), smem, s, xb, Wr, br, T, d, E, k,
+                   logits_out, ids, w, flags);
     else if (epl <= 2)
-        router_small_kernel<2><<<T, 1024, smem, s>>>(xb, Wr, br, T, d, E, k, logits_out, ids, w, flags);
+        launch_pdl(router_small_kernel<2>, dim3(T), dim3(1024), smem, s, xb, Wr, br, T, d, E, k,
+                   logits_out, ids, w, flags);
     else if (epl <= 4)
-        router_small_kernel<4><<<T, 1024, smem, s>>>(xb, Wr, br, T, d, E, k, logits_out, ids, w, flags);
+        launch_pdl(router_small_kernel<4>, dim3(T), dim3(1024), smem, s, xb, Wr, br, T, d, E, k,
+                   logits_out, ids, w, flags);
     else
-        router_small_kernel<8><<<T, 1024, smem, s>>>(xb, Wr, br, T, d, E, k, logits_out, ids, w, flags);
+        launch_pdl(router_small_kernel<8>, dim3(T), dim3(1024), smem, s, xb, Wr, br, T, d, E, k,
+                   logits_out, ids, w, flags);
     *launches += 1;
 }
 
@@ -620,6 +636,7 @@ namespace {
 // Failure-detection self-test: waits on an mbarrier that nothing arrives on, with the same
 // bounded wait the pipelines use; the wait gives up and records MOE_DEV_TIMEOUT.
 __global__ void wait_timeout_selftest_kernel(DeviceStatus* st, unsigned long long limit_ns) {
+    pdl_begin();
     __shared__ __align__(8) uint64_t bar;
     const uint32_t b = smem_u32(&bar);
     if (threadIdx.x == 0) mbar_init(b, 1);
@@ -630,7 +647,8 @@ __global__ void wait_timeout_selftest_kernel(DeviceStatus* st, unsigned long lon
 }  // namespace
 
 void launch_wait_timeout_selftest(DeviceStatus* st, long long limit_ns, cudaStream_t s) {
-    wait_timeout_selftest_kernel<<<1, 32, 0, s>>>(st, (unsigned long long)limit_ns);
+    launch_pdl(wait_timeout_selftest_kernel, dim3(1), dim3(32), 0, s, st,
+               (unsigned long long)limit_ns);
 }
 
 void launch_dispatch_small(const int32_t* ids, const float* w, int T, int E, int k, long long K,
@@ -639,8 +657,8 @@ void launch_dispatch_small(const int32_t* ids, const float* w, int T, int E, int
                            int* launches) {
     const int P = T * k;
     const size_t smem = sizeof(int32_t) * (4 * (size_t)E + 2 + 2 * (size_t)P) + (size_t)P;
-    dispatch_small_kernel<<<1, 1024, smem, s>>>(ids, w, T, E, k, K, flags, slot, drop, counts,
-                                               offsets, rowtok, st);
+    launch_pdl(dispatch_small_kernel, dim3(1), dim3(1024), smem, s, ids, w, T, E, k, K, flags, slot,
+               drop, counts, offsets, rowtok, st);
     *launches += 1;
 }
 
@@ -653,11 +671,13 @@ void launch_capacity_select(const int32_t* ids, const float* w, int T, int E, in
     const int blocks = (nC + 3) / 4;
     const size_t smem = (size_t)4 * E * sizeof(int32_t);
     if (!counts_ready) {
-        count_chunks_kernel<<<blocks, 128, smem, s>>>(ids, T, E, k, nC, cnt, st);
+        launch_pdl(count_chunks_kernel, dim3(blocks), dim3(128), smem, s, ids, T, E, k, nC, cnt,
+                   st);
         *launches += 1;
     }
-    scan_chunks_kernel<<<E, 256, 0, s>>>(cnt, nC, base, nrecv);
-    scatter_chunks_kernel<<<blocks, 128, smem, s>>>(ids, T, E, k, nC, base, cand);
+    launch_pdl(scan_chunks_kernel, dim3(E), dim3(256), 0, s, cnt, nC, base, nrecv);
+    launch_pdl(scatter_chunks_kernel, dim3(blocks), dim3(128), smem, s, ids, T, E, k, nC, base,
+               cand);
     static std::atomic<uint64_t> attr_done{0};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -667,8 +687,8 @@ void launch_capacity_select(const int32_t* ids, const float* w, int T, int E, in
                              kSelSmemKeys * 4);
         attr_done.fetch_or(bit);
     }
-    select_kernel<<<E, kSelThreads, kSelSmemKeys * 4, s>>>(cand, nrecv, w, T, E, k, K, slot, drop,
-                                                            counts, offsets, rowtok, flags);
+    launch_pdl(select_kernel, dim3(E), dim3(kSelThreads), kSelSmemKeys * 4, s, cand, nrecv, w, T, E,
+               k, K, slot, drop, counts, offsets, rowtok, flags);
     *launches += 3;
 }
 
@@ -678,10 +698,12 @@ void launch_dispatch(const int32_t* ids, const int32_t* slot, int T, int E, int 
     const long long P = (long long)T * k;
     const int blocks = (int)std::min<long long>((P + 255) / 256, 148 * 8);
     cudaMemsetAsync(kept_tmp, 0, sizeof(int32_t) * E, s);
-    if (P > 0) kept_count_kernel<<<blocks, 256, 0, s>>>(ids, slot, P, E, T, kept_tmp, st);
-    offsets_kernel<<<1, 1024, 0, s>>>(kept_tmp, E, offsets);
+    if (P > 0) launch_pdl(kept_count_kernel, dim3(blocks), dim3(256), 0, s, ids, slot, P, E, T,
+                          kept_tmp, st);
+    launch_pdl(offsets_kernel, dim3(1), dim3(1024), 0, s, kept_tmp, E, offsets);
     if (P > 0)
-        rowtok_scatter_kernel<<<blocks, 256, 0, s>>>(ids, slot, P, E, k, offsets, rowtok, st);
+        launch_pdl(rowtok_scatter_kernel, dim3(blocks), dim3(256), 0, s, ids, slot, P, E, k,
+                   offsets, rowtok, st);
     *launches += (P > 0) ? 3 : 1;
 }
 
@@ -690,11 +712,11 @@ void launch_permute_rows(const void* x, const int32_t* rowtok, const int32_t* of
                          cudaStream_t s, int* launches) {
     const int blocks = 148 * 8;
     if (row_bytes % 16 == 0 && ((uintptr_t)x % 16 == 0) && ((uintptr_t)xp % 16 == 0)) {
-        permute_rows_kernel<uint4><<<blocks, 256, 0, s>>>(
-            (const uint4*)x, rowtok, offsets, E, (int)(row_bytes / 16), T, (uint4*)xp, st);
+        launch_pdl(permute_rows_kernel<uint4>, dim3(blocks), dim3(256), 0, s, (const uint4*)x,
+                   rowtok, offsets, E, (int)(row_bytes / 16), T, (uint4*)xp, st);
     } else {
-        permute_rows_kernel<uint32_t><<<blocks, 256, 0, s>>>(
-            (const uint32_t*)x, rowtok, offsets, E, (int)(row_bytes / 4), T, (uint32_t*)xp, st);
+        launch_pdl(permute_rows_kernel<uint32_t>, dim3(blocks), dim3(256), 0, s, (const uint32_t*)x,
+                   rowtok, offsets, E, (int)(row_bytes / 4), T, (uint32_t*)xp, st);
     }
     (void)max_rows;
     *launches += 1;
