@@ -933,9 +933,17 @@ cudaError_t launch_router_bn(int BN, const CUtensorMap& tmA, const CUtensorMap& 
 
 }  // namespace
 
-// Column tile for an output width: least padded work, then the wider tile.  MOE_GEMM_BN in the
-// environment (256, 192, 176 or 128) overrides the choice, for tuning runs.
-int pick_bn(int nout) {
+// Column tile for an output width.  MOE_GEMM_BN in the environment (256, 192, 176 or 128)
+// overrides the choice, for tuning runs.
+//  - Groups of many rows (compute-bound): a column tile costs BN + 128, for the per-tile work
+//    that does not shrink with BN (A operand loads, pipeline turn-around), about half a 256-wide
+//    tile's MMA time.  Measured on B200 at d_ff = 1408: 256-wide tiles (with a half-width last
+//    tile) beat the exact 176-wide ones by 15%.
+//  - At most 64 rows per group on average (decode, weight streaming): a tile costs about its
+//    weight bytes, BN + 32, and the persistent grid finishes with its last partial wave, so
+//    the cost is ceil(tiles / SMs) x (BN + 32).  Measured on B200 at T = 64, E = 64, k = 8:
+//    d_model = 2048 outputs on 128-wide tiles (6.9 waves) beat 256-wide ones (3.5) by 13%.
+int pick_bn(int nout, long long max_rows, int E, int num_sm) {
     static int forced = -1;
     if (forced < 0) {
         const char* v = getenv("MOE_GEMM_BN");
@@ -943,14 +951,20 @@ int pick_bn(int nout) {
         forced = (f == 256 || f == 192 || f == 176 || f == 128) ? f : 0;
     }
     if (forced > 0) return forced;
-    // Cost of a column tile ~ BN + 128: per-tile work that does not shrink with BN (A operand
-    // loads, pipeline turn-around) is about half a 256-wide tile's MMA time.  Measured on B200
-    // at d_ff = 1408: 256-wide tiles (9% padding) beat the exact 176-wide ones by 15%.
-    const int cands[] = {256, 192, 176, 128};
+    const bool streaming = max_rows <= 64LL * E;
+    const long long m_tiles = streaming ? E : (max_rows + 127) / 128 + E;
+    // Ties go to the wider tile when compute-bound, to the narrower one (finer waves) when
+    // streaming.
+    const int wide_first[] = {256, 192, 176, 128};
+    const int narrow_first[] = {128, 176, 192, 256};
+    const int* cands = streaming ? narrow_first : wide_first;
     int best = 256;
     long long best_cost = -1;
-    for (int bn : cands) {
-        const long long cost = (long long)((nout + bn - 1) / bn) * (bn + 128);
+    for (int c = 0; c < 4; ++c) {
+        const int bn = cands[c];
+        const long long n_tiles = (nout + bn - 1) / bn;
+        const long long cost =
+            streaming ? (m_tiles * n_tiles + num_sm - 1) / num_sm * (bn + 32) : n_tiles * (bn + 128);
         if (best_cost < 0 || cost < best_cost) { best = bn; best_cost = cost; }
     }
     return best;
@@ -988,7 +1002,7 @@ cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const in
         return launch_gated_gemm(A, lda, a_rows, a_row_limit, offsets, E, K, Nout, W, bias, D,
                                  ldd, max_rows, st, s, launches);
     }
-    const int BN = pick_bn(Nout);
+    const int BN = pick_bn(Nout, max_rows, E, num_sms());
     // Gathered A on pairs needs the peer's rows forwarded to the leader's barrier by the copying
     // threads themselves, which measured slower than single-CTA tiles; only when forced.
     const bool pair = use_pair(max_rows, E) && (a_rows == nullptr || g_pair_mode == 1);

@@ -54,7 +54,7 @@ void launch_logits_f32(const float* x, const float* Wr, const float* br, int T, 
                        float* logits, cudaStream_t s, int* launches);
 
 // gemm_tc.cu
-int pick_bn(int nout);
+int pick_bn(int nout, long long max_rows, int E, int num_sm);
 int router_group(int E);
 size_t router_split_bytes(int d, int E);
 // which = 0: D = SiLU(A W^T + bias) (GEMM1); which = 1: D = A W^T + bias (GEMM2);

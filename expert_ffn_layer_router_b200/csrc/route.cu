@@ -135,6 +135,20 @@ __global__ void __launch_bounds__(1024) router_small_kernel(
         const int i0 = (int)((long long)d * part / P), i1 = (int)((long long)d * (part + 1) / P);
         float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
         int i = i0;
+        // 32 weights in flight per thread (the loads do not wait on one another), then the
+        // products in the same order as four at a time.
+        for (; i + 31 < i1; i += 32) {
+            float wv[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) wv[j] = __ldg(Wr + (size_t)(i + j) * E + e);
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                a0 = __fmaf_rn(s_x[i + j], wv[j], a0);
+                a1 = __fmaf_rn(s_x[i + j + 1], wv[j + 1], a1);
+                a2 = __fmaf_rn(s_x[i + j + 2], wv[j + 2], a2);
+                a3 = __fmaf_rn(s_x[i + j + 3], wv[j + 3], a3);
+            }
+        }
         for (; i + 3 < i1; i += 4) {
             const float w0 = __ldg(Wr + (size_t)i * E + e);
             const float w1 = __ldg(Wr + (size_t)(i + 1) * E + e);
@@ -418,13 +432,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
 // ---------------------------------------------------------------------------------------------
 constexpr int kSmallPairs = 1024;
 
-__global__ void __launch_bounds__(1024) dispatch_small_kernel(
+__device__ __forceinline__ void dispatch_small_block(
     const int32_t* __restrict__ ids, const float* __restrict__ w, int T, int E, int k,
     long long K, unsigned flags, int32_t* __restrict__ slot, uint8_t* __restrict__ drop,
     int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ rowtok,
-    DeviceStatus* st) {
-    pdl_begin();
-    extern __shared__ int32_t sm[];
+    DeviceStatus* st, int32_t* sm) {
     __shared__ int s_warp[32];
     const int P = T * k;
     int32_t* cnt = sm;                 // [E]
@@ -433,12 +445,16 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(
     int32_t* koff = run + E;           // [E + 1] kept offsets
     int32_t* list = koff + E + 1;      // [P] pair index, grouped by expert, ascending token
     int32_t* lexp = list + P;          // [P] expert of each list position
-    uint8_t* keep = reinterpret_cast<uint8_t*>(lexp + P);   // [P]
+    int32_t* s_ids = lexp + P;         // [P] the routing, read from global memory once
+    float* s_w = reinterpret_cast<float*>(s_ids + P);      // [P]
+    uint8_t* keep = reinterpret_cast<uint8_t*>(s_w + P);   // [P]
     const int tid = threadIdx.x;
     for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
     __syncthreads();
     for (int p = tid; p < P; p += blockDim.x) {
         const int e = ids[p];
+        s_ids[p] = e;
+        s_w[p] = w[p];
         if ((unsigned)e < (unsigned)E) atomicAdd(&cnt[e], 1);
         else report(st, MOE_DEV_BAD_INDEX, 111);
     }
@@ -461,7 +477,7 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(
     if (tid < 32) {                                   // stable placement, 32 pairs at a time
         for (int pb = 0; pb < P; pb += 32) {
             const int p = pb + tid;
-            int e = p < P ? ids[p] : -1;
+            int e = p < P ? s_ids[p] : -1;
             if ((unsigned)e >= (unsigned)E) e = -1;
             const unsigned peers = __match_any_sync(kFull, e);
             const int rank = __popc(peers & ((1u << tid) - 1u));
@@ -485,10 +501,10 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(
             kp = pos < K;
         } else {
             const int p = list[i];
-            const float wi = w[p];
+            const float wi = s_w[p];
             int rank = 0;
             for (int j = b0; j < b0 + n; ++j) {
-                const float wj = w[list[j]];
+                const float wj = s_w[list[j]];
                 rank += (wj > wi || (wj == wi && j < i)) ? 1 : 0;
             }
             kp = rank < K;
@@ -516,6 +532,16 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(
         if (offsets) offsets[e] = koff[e];
     }
     if (tid == 0 && offsets) offsets[E] = koff[E];
+}
+
+__global__ void __launch_bounds__(1024) dispatch_small_kernel(
+    const int32_t* __restrict__ ids, const float* __restrict__ w, int T, int E, int k,
+    long long K, unsigned flags, int32_t* __restrict__ slot, uint8_t* __restrict__ drop,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ rowtok,
+    DeviceStatus* st) {
+    pdl_begin();
+    extern __shared__ int32_t sm[];
+    dispatch_small_block(ids, w, T, E, k, K, flags, slot, drop, counts, offsets, rowtok, st, sm);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -656,7 +682,7 @@ void launch_dispatch_small(const int32_t* ids, const float* w, int T, int E, int
                            int32_t* offsets, int32_t* rowtok, DeviceStatus* st, cudaStream_t s,
                            int* launches) {
     const int P = T * k;
-    const size_t smem = sizeof(int32_t) * (4 * (size_t)E + 2 + 2 * (size_t)P) + (size_t)P;
+    const size_t smem = sizeof(int32_t) * (4 * (size_t)E + 2 + 4 * (size_t)P) + (size_t)P;
     launch_pdl(dispatch_small_kernel, dim3(1), dim3(1024), smem, s, ids, w, T, E, k, K, flags, slot,
                drop, counts, offsets, rowtok, st);
     *launches += 1;

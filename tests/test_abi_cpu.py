@@ -65,6 +65,17 @@ def test_workspace_size_covers_buffers(moe):
     assert n % 256 == 0
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_workspace_size_for_any_legal_shape(moe, dtype):
+    """Sizing is host arithmetic only; every legal shape (widths the expert GEMMs reject
+    included: moe_route and moe_combine take any width) gets a size, without a host fault."""
+    for T in (0, 1, 7, 64, 128, 1000, 1024, 1025, 4096):
+        for d in (1, 4, 8, 36, 64, 100, 192, 2112, 12288, 12352):
+            for E, k in ((1, 1), (8, 2), (64, 8), (256, 4), (1024, 1)):
+                n = moe.moe_workspace_size(moe.problem(T, d, 64, E, k, 1.25, dtype))
+                assert n >= 256 and n % 256 == 0
+
+
 @pytest.mark.parametrize("bad", [dict(k=5, E=4), dict(C=-1.0), dict(C=float("nan")),
                                  dict(E=0), dict(E=2000), dict(k=33, E=64), dict(T=-1),
                                  dict(dtype=7), dict(d=0)])
