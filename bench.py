@@ -245,8 +245,9 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def traffic_record(kernel):
-    """dram bytes per launch from the committed ncu summary, if taken on the current source."""
+def traffic_record(kernel, workload):
+    """dram bytes per launch from the committed ncu summary, if taken on the current source and
+    on this workload."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -254,7 +255,7 @@ def traffic_record(kernel):
         rec = json.load(f)
     h = kernel_source_hash()
     r = rec.get(kernel)
-    if not r or r.get("source_sha256_16") != h:
+    if not r or r.get("source_sha256_16") != h or r.get("workload") != workload:
         return None
     return r.get("bytes_per_launch")
 
@@ -313,35 +314,50 @@ def run_cuda(args):
     kept = int(counts[spec.E:].sum().item())
     received = int(counts[:spec.E].sum().item())
 
-    # Timed region: K steps, L2 flushed before each (outside the step's events).
+    # Timed region: K steps, L2 flushed before each (outside the step's events).  The headline
+    # steps carry only a start and an end event; a second, instrumented run of K steps records
+    # an event between every stage (moe_set_stage_events) for the per-kernel durations.  Stage
+    # events cost the GPU about 2.5 us each, so the headline is taken without them.
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.STAGE_EVENTS)]
-           for _ in range(K)]
-    for row in evs:                       # torch creates the CUDA event at its first record
-        for e in row:
-            e.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    for i in range(K):
-        flush.zero_()
-        moe.moe_set_stage_events(evs[i])
-        step()
-    moe.moe_set_stage_events(None)
-    torch.cuda.synchronize()
+
+    def timed_steps(instrumented):
+        n_ev = moe.STAGE_EVENTS if instrumented else 2
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(K)]
+        for row in evs:                   # torch creates the CUDA event at its first record
+            for e in row:
+                e.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(K):
+            flush.zero_()
+            if instrumented:
+                moe.moe_set_stage_events(evs[i])
+                step()
+            else:
+                evs[i][0].record(stream)
+                step()
+                evs[i][1].record(stream)
+        if instrumented:
+            moe.moe_set_stage_events(None)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        return evs
+
+    evs_plain = timed_steps(False)
+    evs = timed_steps(True)
     clocks = sampler.stop()
-    if world > 1:
-        dist.barrier()
     stage_ms = np.zeros((K, moe.STAGE_EVENTS - 1))
     for i in range(K):
         for s in range(moe.STAGE_EVENTS - 1):
             stage_ms[i, s] = evs[i][s].elapsed_time(evs[i][s + 1])
-    step_ms = np.array([evs[i][0].elapsed_time(evs[i][-1]) for i in range(K)])
+    step_ms = np.array([evs_plain[i][0].elapsed_time(evs_plain[i][1]) for i in range(K)])
+    instr_ms = np.array([evs[i][0].elapsed_time(evs[i][-1]) for i in range(K)])
     total_ms = max_over_ranks(float(step_ms.sum()), dist if world > 1 else None, dev)
     ms_per_step = total_ms / K
     value = world * spec.T / (ms_per_step / 1e3)
-
     # End to end through the C ABI with host buffers, as a serving loop runs it: every step
     # copies its x from pinned host memory to the device, runs the layer and copies its output
     # back to pinned host memory.  Copy-in, compute and copy-out run on three streams with
@@ -406,6 +422,9 @@ def run_cuda(args):
                              bytes=kept * F * esz + E * dm * F * esz + kept * dm * esz),
         "combine": dict(bytes=2 * T * dm * esz + kept * dm * esz + T * k * 12 + (E + 1) * 4),
     }
+    input_bytes = sum(int(t.numel() * t.element_size()) for t in d.values() if t is not None)
+    traffic_key = spec.name + (" gated" if spec.gated else "") + \
+        (" T=%d" % spec.T if args.tokens else "")
     kernels = {}
     for i, n in enumerate(names6):
         ms = float(st_avg[i])
@@ -431,7 +450,9 @@ def run_cuda(args):
         "config": {"workload": workload_desc(spec), "seed": args.seed + rank,
                    "per_rank_tokens": T, "parallelism": "dp%d (independent batches)" % world,
                    "l2": "flushed before every timed step (256 MiB write, outside the step's"
-                         " events); per-step inputs 805 MB also exceed the 126 MB L2",
+                         " events); per-step inputs %.0f MB" % (input_bytes / 1e6),
+                   "timing": "value: K steps with start/end events only; kernels and roofline:"
+                             " a second run of K steps with an event between stages",
                    "kept_pairs": kept, "received_pairs": received,
                    "dropped_pairs": received - kept},
         "gpu_launches": launches_per_step * K,
@@ -449,7 +470,7 @@ def run_cuda(args):
                      "frac": achieved / tensor_peak if achieved else None,
                      "peak_source": "%s bf16_tflops_sustained (kernel timed inside a long"
                                     " loop of steps)" % pk_kind,
-                     "traffic": traffic_record(dom)},
+                     "traffic": traffic_record(dom, traffic_key)},
         "expert_gemm": {"tflops": gemm_tflops, "frac_of_peak": gemm_tflops / tensor_peak,
                         "frac_of_burst_peak": gemm_tflops / pk.get("bf16_tflops", tensor_peak),
                         "flop_per_step": g1_flop + gemm_flop_each},
@@ -457,6 +478,7 @@ def run_cuda(args):
                                    "bytes_per_step": rdc_bytes, "hbm_peak_gbs": pk["hbm_gbs"]},
         "kernels": kernels,
         "step_ms_min": float(step_ms.min()), "step_ms_median": float(np.median(step_ms)),
+        "instrumented_ms_per_step": float(instr_ms.mean()),
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         cores = cpu_cores()
