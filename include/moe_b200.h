@@ -25,7 +25,10 @@
  *     from the caller's workspace `ws` of `ws_bytes` bytes (size from moe_workspace_size,
  *     256-byte aligned).
  *   - Every compute call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
- *     stream) and performs no host synchronisation.
+ *     stream) and performs no host synchronisation.  Kernels are launched with programmatic
+ *     stream serialization: a kernel may be scheduled while the preceding work on `stream`
+ *     drains, but it waits for that work to complete (griddepcontrol.wait) before it reads or
+ *     writes any memory, so stream order is kept for every input and output.
  *   - Host-checkable errors (bad shapes, k > E, negative or NaN capacity factor, null or
  *     misaligned pointers, workspace too small, unsupported shape) return a non-zero status
  *     BEFORE anything is launched; outputs are then untouched.

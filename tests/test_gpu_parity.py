@@ -373,6 +373,35 @@ def test_forward_cuda_graph_replay(spec):
 
 
 # ------------------------------------------------------------------------------------------
+# Stream order with programmatic dependent launch: the first kernel of a call may be scheduled
+# while the caller's preceding work drains, but must not read x before that work has written
+# it.  x is produced on the same stream right before the call (a copy from pinned host memory,
+# then an in-place update by a torch kernel), in a loop, and every output must match.
+# ------------------------------------------------------------------------------------------
+def test_forward_reads_inputs_written_just_before_on_the_stream():
+    moe = _moe()
+    spec = inputs.LayerSpec("s1", 3000, 256, 128, 8, 2, 1.0, "bf16")
+    L = inputs.make_layer(spec, seed=5)
+    layer = moe.MoELayer(spec.T, spec.d_model, spec.d_ff, spec.E, spec.k, spec.C, spec.dtype)
+    args = [to_dev(L[n]) for n in ("x", "Wr", "br", "W1", "b1", "W2", "b2")]
+    x_host = args[0].cpu().pin_memory()
+    refs = []
+    for scale in (1.0, -1.0, 0.5):
+        xs = (args[0].float() * scale).to(torch.bfloat16)
+        refs.append(layer.forward(xs, *args[1:]).clone())
+    torch.cuda.synchronize()
+    xd = torch.empty_like(args[0])
+    out = torch.empty_like(refs[0])
+    for rep in range(3):
+        for scale, ref in zip((1.0, -1.0, 0.5), refs):
+            xd.copy_(x_host, non_blocking=True)       # same stream, no host sync in between
+            xd.mul_(scale)                           # exact in bf16 for these scales
+            layer.forward(xd, *args[1:], out=out)
+            torch.cuda.synchronize()
+            assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), (rep, scale)
+
+
+# ------------------------------------------------------------------------------------------
 # Failure detection: a pipeline wait that can never complete gives up, reports a timeout in the
 # status word, and leaves the GPU usable (no trap, no fault, no hang).
 # ------------------------------------------------------------------------------------------
