@@ -266,22 +266,31 @@ __global__ void __launch_bounds__(128) scatter_chunks_kernel(const int32_t* __re
     __syncwarp();
     const long long p0 = (long long)c * kChunk * k;
     const long long p1 = (long long)min(T, (c + 1) * kChunk) * k;
-    for (long long pb = p0; pb < p1; pb += 32) {
-        const long long p = pb + lane;
-        const bool act = p < p1;
-        const unsigned amask = __ballot_sync(kFull, act);
-        int e = act ? ids[p] : -1;
-        if ((unsigned)e >= (unsigned)E) e = -1;        // bad ids were reported by the count pass
-        const unsigned peers = __match_any_sync(kFull, e);
-        const int rank = __popc(peers & ((1u << lane) - 1u));
-        const int pos = (e >= 0) ? run[e] + rank : 0;
-        __syncwarp();
-        if (act && e >= 0) {
-            cand[(size_t)e * T + pos] = (int32_t)p;
-            if (lane == __ffs(peers) - 1) run[e] = pos + __popc(peers);
+    // The chunk's ids are loaded 8 rounds of 32 at a time (independent loads in flight), then
+    // placed round by round in pair order.
+    for (long long pg = p0; pg < p1; pg += 8 * 32) {
+        int ev[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const long long p = pg + 32 * r + lane;
+            ev[r] = p < p1 ? ids[p] : -1;
         }
-        __syncwarp();
-        (void)amask;
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const long long p = pg + 32 * r + lane;
+            if (pg + 32 * r >= p1) break;               // warp-uniform
+            int e = ev[r];
+            if ((unsigned)e >= (unsigned)E) e = -1;    // bad ids were reported by the count pass
+            const unsigned peers = __match_any_sync(kFull, e);
+            const int rank = __popc(peers & ((1u << lane) - 1u));
+            const int pos = (e >= 0) ? run[e] + rank : 0;
+            __syncwarp();
+            if (p < p1 && e >= 0) {
+                cand[(size_t)e * T + pos] = (int32_t)p;
+                if (lane == __ffs(peers) - 1) run[e] = pos + __popc(peers);
+            }
+            __syncwarp();
+        }
     }
 }
 
@@ -289,7 +298,7 @@ __global__ void __launch_bounds__(128) scatter_chunks_kernel(const int32_t* __re
 // Capacity selection: one block per expert.
 // ---------------------------------------------------------------------------------------------
 constexpr int kSelThreads = 1024;
-constexpr int kSelSmemKeys = 32768;   // weight keys of one expert's candidates kept on chip
+constexpr int kSelSmemKeys = 16384;   // candidates of one expert whose list and keys stay on chip
 
 __global__ void __launch_bounds__(kSelThreads) select_kernel(
     const int32_t* __restrict__ cand, const int32_t* __restrict__ nrecv,
@@ -297,7 +306,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     uint8_t* __restrict__ drop, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
     int32_t* __restrict__ rowtok, unsigned flags) {
     pdl_begin();
-    extern __shared__ uint32_t s_keys[];              // [kSelSmemKeys]
+    extern __shared__ uint32_t s_keys[];              // [kSelSmemKeys] keys, then the list
+    int32_t* s_list = reinterpret_cast<int32_t*>(s_keys + kSelSmemKeys);
     __shared__ int s_warp[32];
     __shared__ int s_hist[256];
     __shared__ uint32_t s_prefix;
@@ -346,7 +356,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     // values), gathered once into shared memory when they fit.
     const bool on_chip = n <= kSelSmemKeys;
     if (on_chip)
-        for (int i = tid; i < n; i += blockDim.x) s_keys[i] = __float_as_uint(w[list[i]]);
+        for (int i = tid; i < n; i += blockDim.x) {
+            const int p = list[i];
+            s_list[i] = p;
+            s_keys[i] = __float_as_uint(w[p]);
+        }
     __syncthreads();
     auto key_of = [&](int i) -> uint32_t {
         return on_chip ? s_keys[i] : __float_as_uint(w[list[i]]);
@@ -400,17 +414,22 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     }
     const uint32_t tau = prefix;        // K-th largest weight bits
     const int need_eq = remaining;      // how many weights equal to tau are kept (lowest t first)
+    // After the last pass s_hist[tau & 255] counts the keys equal to tau.  When all of them are
+    // kept (no tie straddles the capacity boundary, the usual case) keep = (key >= tau) and the
+    // tie ranks are not needed.
+    const bool all_eq_kept = s_hist[tau & 255u] == need_eq;
 
     int eq_carry = 0, keep_carry = 0;
     for (int i0 = 0; i0 < n; i0 += blockDim.x) {
         const int i = i0 + tid;
         int p = 0;
         uint32_t key = 0;
-        if (i < n) { p = list[i]; key = key_of(i); }
+        if (i < n) { p = on_chip ? s_list[i] : list[i]; key = key_of(i); }
         const int is_eq = (i < n && key == tau) ? 1 : 0;
-        int eq_tot;
-        const int eq_rank = eq_carry + block_exclusive_scan(is_eq, s_warp, &eq_tot);
-        const int keep = (i < n) && (key > tau || (is_eq && eq_rank < need_eq)) ? 1 : 0;
+        int eq_tot = 0, eq_rank = 0;
+        if (!all_eq_kept) eq_rank = eq_carry + block_exclusive_scan(is_eq, s_warp, &eq_tot);
+        const int keep =
+            (i < n) && (key > tau || (is_eq && (all_eq_kept || eq_rank < need_eq))) ? 1 : 0;
         int keep_tot;
         const int s = keep_carry + block_exclusive_scan(keep, s_warp, &keep_tot);
         if (i < n) {
@@ -710,10 +729,10 @@ void launch_capacity_select(const int32_t* ids, const float* w, int T, int E, in
     const uint64_t bit = 1ull << (dev & 63);
     if (!(attr_done.load() & bit)) {
         cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSelSmemKeys * 4);
+                             kSelSmemKeys * 8);
         attr_done.fetch_or(bit);
     }
-    launch_pdl(select_kernel, dim3(E), dim3(kSelThreads), kSelSmemKeys * 4, s, cand, nrecv, w, T, E,
+    launch_pdl(select_kernel, dim3(E), dim3(kSelThreads), kSelSmemKeys * 8, s, cand, nrecv, w, T, E,
                k, K, slot, drop, counts, offsets, rowtok, flags);
     *launches += 3;
 }
