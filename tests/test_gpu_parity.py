@@ -402,6 +402,67 @@ def test_forward_reads_inputs_written_just_before_on_the_stream():
 
 
 # ------------------------------------------------------------------------------------------
+# Canaries: every byte the forward writes lies inside its outputs and its workspace.  Each
+# buffer sits between 4 KB guard regions filled with a pattern, which must survive the call.
+# ------------------------------------------------------------------------------------------
+def _guarded(n_elems, dtype, fill_byte=0x5A, guard_bytes=4096):
+    esz = torch.empty((), dtype=dtype).element_size()
+    g = guard_bytes // esz
+    raw = torch.full(((2 * guard_bytes + n_elems * esz),), fill_byte, dtype=torch.uint8,
+                     device="cuda")
+    view = raw[guard_bytes:guard_bytes + n_elems * esz].view(dtype)
+    return raw, view, g * esz
+
+
+def _guards_intact(raw, guard_bytes, fill_byte=0x5A):
+    head = raw[:guard_bytes]
+    tail = raw[raw.numel() - guard_bytes:]
+    return bool((head == fill_byte).all().item()) and bool((tail == fill_byte).all().item())
+
+
+@pytest.mark.parametrize("spec", [
+    inputs.LayerSpec("c1", 64, 256, 128, 16, 8, math.inf, "bf16"),
+    inputs.LayerSpec("c2", 3000, 128, 192, 8, 2, 1.0, "bf16", router="zipf", router_bias=1.1),
+    inputs.LayerSpec("c3", 1500, 128, 256, 8, 2, 0.7, "bf16", gated=True),
+    inputs.LayerSpec("c4", 300, 16, 24, 6, 2, 1.0, "f32"),
+])
+def test_forward_writes_stay_inside_outputs_and_workspace(spec):
+    moe = _moe()
+    L = inputs.make_layer(spec, seed=9)
+    flags = moe.FLAG_GATED if spec.gated else 0
+    p = moe.problem(spec.T, spec.d_model, spec.d_ff, spec.E, spec.k, spec.C, spec.dtype,
+                    flags=flags)
+    args = [to_dev(L[n]) for n in ("x", "Wr", "br", "W1", "b1", "W2", "b2")]
+    x = args[0]
+    T, E, k = spec.T, spec.E, spec.k
+    bufs = {}
+    bufs["ws"] = _guarded(moe.moe_workspace_size(p), torch.uint8)
+    bufs["out"] = _guarded(x.numel(), x.dtype)
+    bufs["logits"] = _guarded(T * E, torch.float32)
+    bufs["ids"] = _guarded(T * k, torch.int32)
+    bufs["w"] = _guarded(T * k, torch.float32)
+    bufs["slot"] = _guarded(T * k, torch.int32)
+    bufs["drop"] = _guarded(T * k, torch.uint8)
+    bufs["counts"] = _guarded(2 * E, torch.int32)
+    out = bufs["out"][1].view(x.shape)
+    moe.moe_forward(p, *args, out, bufs["ws"][1], logits_out=bufs["logits"][1],
+                    ids_out=bufs["ids"][1], w_out=bufs["w"][1], slot_out=bufs["slot"][1],
+                    drop_out=bufs["drop"][1], counts_out=bufs["counts"][1])
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(bufs["ws"][1]) == 0
+    for name, (raw, _, gb) in bufs.items():
+        assert _guards_intact(raw, gb), name
+    layer = moe.MoELayer(spec.T, spec.d_model, spec.d_ff, spec.E, spec.k, spec.C, spec.dtype,
+                         flags=flags)
+    ref = layer.forward(*args)
+    torch.cuda.synchronize()
+    if x.dtype == torch.bfloat16:
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    else:
+        assert torch.equal(out, ref)
+
+
+# ------------------------------------------------------------------------------------------
 # Failure detection: a pipeline wait that can never complete gives up, reports a timeout in the
 # status word, and leaves the GPU usable (no trap, no fault, no hang).
 # ------------------------------------------------------------------------------------------
