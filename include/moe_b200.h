@@ -34,6 +34,8 @@
  *     BEFORE anything is launched; outputs are then untouched.
  *   - Errors the device detects (a pipeline wait that ran out, an index out of range) are
  *     recorded in a status word at the start of `ws`; read it with moe_get_device_status.
+ *     The calls never clear it (the first error stays), so clear it once with
+ *     moe_reset_device_status after allocating a workspace, and again after handling an error.
  *   - Layouts are row-major and dense.  Pair p = t * k + j addresses the j-th expert of token
  *     t (j = 0 is the largest logit).  W1 is [E, d_ff, d_model] and W2 is [E, d_model, d_ff]
  *     ("out x in", so h = W1 x).  b1 is [E, d_ff] and b2 is [E, d_model], float32 always.

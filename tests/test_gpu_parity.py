@@ -445,6 +445,7 @@ def test_forward_writes_stay_inside_outputs_and_workspace(spec):
     bufs["drop"] = _guarded(T * k, torch.uint8)
     bufs["counts"] = _guarded(2 * E, torch.int32)
     out = bufs["out"][1].view(x.shape)
+    moe.moe_reset_device_status(bufs["ws"][1])       # the status word is the caller's to clear
     moe.moe_forward(p, *args, out, bufs["ws"][1], logits_out=bufs["logits"][1],
                     ids_out=bufs["ids"][1], w_out=bufs["w"][1], slot_out=bufs["slot"][1],
                     drop_out=bufs["drop"][1], counts_out=bufs["counts"][1])
