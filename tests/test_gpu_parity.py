@@ -125,8 +125,8 @@ def test_dispatch_bit_exact(T, E, k, C, dtype):
 # ------------------------------------------------------------------------------------------
 @pytest.mark.parametrize("T,d,F,E,k,C,dtype,bias", [
     (300, 128, 192, 5, 2, 1.0, "bf16", 0.05),      # ragged experts, one column tile
-    (1000, 256, 1408, 4, 1, 1.25, "bf16", 0.02),   # d_ff = 11 x 128: 176-wide tiles
-    (700, 512, 320, 3, 3, 0.9, "bf16", 0.0),       # several m-tiles per expert, 128-wide tiles
+    (1000, 256, 1408, 4, 1, 1.25, "bf16", 0.02),   # d_ff = 1408: 256-wide tiles, the last half full
+    (700, 512, 320, 3, 3, 0.9, "bf16", 0.0),       # several m-tiles per expert, a ragged column tile
     (129, 64, 64, 2, 1, math.inf, "bf16", 0.1),    # 129 rows: one full tile + one row
     (40, 16, 24, 4, 2, 1.0, "f32", 0.1),
     (8, 4, 8, 4, 1, 1.25, "f32", 0.1)])
