@@ -166,7 +166,10 @@ def run_reference(args):
                              "unit": "tokens/s"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0},
-            "measured_seconds_per_step": statistics.mean(meas)}
+            "measured_seconds_per_step": statistics.mean(meas),
+            "sample_tokens_per_step": sample,
+            "timing_note": "ms_per_step extrapolates each step's timed sample to all T tokens;"
+                           " measured_seconds_per_step is the time actually spent per step"}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -411,12 +414,20 @@ def run_cuda(args):
     names6 = moe.STAGE_NAMES
     gemm_flop_each = 2.0 * kept * dm * F
     g1_flop = gemm_flop_each * (2 if spec.gated else 1)
+    # Algorithmic work per stage (the method's, not the implementation's): the router's flops
+    # are 2 T d E; bytes count every input read once and every output written once.  With the
+    # routing fused into the logits GEMM (bf16, E <= 64, T > 1024) the router stage reads x and
+    # Wr and writes ids, weights and per-chunk counts, and the separate top-k stage is empty;
+    # otherwise the logits round-trip through HBM between the two stages.
+    n_chunks = (T + 31) // 32
+    fused = spec.dtype == "bf16" and E <= 64 and T > 1024
+    router_out = T * k * 8 + E * n_chunks * 4 if fused else T * E * 4
     by = {
-        "router_logits": dict(flop=2.0 * T * dm * E * 3, bytes=T * dm * esz + dm * E * 4 + T * E * 4),
-        "route_topk": dict(bytes=T * E * 4 + T * k * 8),
+        "router_logits": dict(flop=2.0 * T * dm * E, bytes=T * dm * esz + dm * E * 4 + router_out),
+        "route_topk": dict(bytes=0 if fused else T * E * 4 + T * k * 8),
         "capacity_dispatch": dict(bytes=T * k * 8 + T * k * 5 + kept * 4 + E * 16),
         "expert_gemm1": dict(flop=g1_flop,
-                             bytes=kept * dm * esz + E * F * dm * esz * (2 if spec.gated else 1)
+                             bytes=T * dm * esz + E * F * dm * esz * (2 if spec.gated else 1)
                              + kept * F * esz),
         "expert_gemm2": dict(flop=gemm_flop_each,
                              bytes=kept * F * esz + E * dm * F * esz + kept * dm * esz),
@@ -439,8 +450,9 @@ def run_cuda(args):
     achieved = kernels[dom]["tflops"]
     gemm_ms = g1["ms"] + g2["ms"]
     gemm_tflops = (g1_flop + gemm_flop_each) / (gemm_ms * 1e-3) / 1e12
-    rdc_bytes = sum(by[n]["bytes"] for n in ("route_topk", "capacity_dispatch", "combine"))
-    rdc_ms = sum(kernels[n]["ms"] for n in ("route_topk", "capacity_dispatch", "combine"))
+    rdc_stages = ("router_logits", "route_topk", "capacity_dispatch", "combine")
+    rdc_bytes = sum(by[n]["bytes"] for n in rdc_stages)
+    rdc_ms = sum(kernels[n]["ms"] for n in rdc_stages)
     rdc_gbs = rdc_bytes / (rdc_ms * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
@@ -475,7 +487,9 @@ def run_cuda(args):
                         "frac_of_burst_peak": gemm_tflops / pk.get("bf16_tflops", tensor_peak),
                         "flop_per_step": g1_flop + gemm_flop_each},
         "route_dispatch_combine": {"gbs": rdc_gbs, "frac_of_hbm": rdc_gbs / pk["hbm_gbs"],
-                                   "bytes_per_step": rdc_bytes, "hbm_peak_gbs": pk["hbm_gbs"]},
+                                   "bytes_per_step": rdc_bytes, "hbm_peak_gbs": pk["hbm_gbs"],
+                                   "stages": list(rdc_stages),
+                                   "router_fused": fused},
         "kernels": kernels,
         "step_ms_min": float(step_ms.min()), "step_ms_median": float(np.median(step_ms)),
         "instrumented_ms_per_step": float(instr_ms.mean()),

@@ -59,8 +59,8 @@ template <class Tr, bool kVector>
 __global__ void __launch_bounds__(256) combine_kernel(
     const void* __restrict__ x, const void* __restrict__ Y, const float* __restrict__ w,
     const int32_t* __restrict__ ids, const int32_t* __restrict__ slot,
-    const int32_t* __restrict__ offsets, int T, int d, int E, int k, void* __restrict__ out,
-    DeviceStatus* st) {
+    const int32_t* __restrict__ offsets, int T, int d, int E, int k, long long max_rows,
+    void* __restrict__ out, DeviceStatus* st) {
     pdl_begin();
     constexpr int V = Tr::kVec;
     const int lane = threadIdx.x & 31;
@@ -75,8 +75,8 @@ __global__ void __launch_bounds__(256) combine_kernel(
         if (s >= 0) {
             const int e = ids[p];
             if ((unsigned)e < (unsigned)E) {
-                const int r = offsets[e] + s;
-                if (r < offsets[e + 1]) { row = r; wt = w[p]; }
+                const long long r = (long long)offsets[e] + s;
+                if (r >= 0 && r < offsets[e + 1] && r < max_rows) { row = (int)r; wt = w[p]; }
                 else report(st, MOE_DEV_BAD_INDEX, 301);
             } else {
                 report(st, MOE_DEV_BAD_INDEX, 302);
@@ -142,8 +142,8 @@ template <class Tr, int KMAX>
 __global__ void __launch_bounds__(256) combine_vec_kernel(
     const uint4* __restrict__ x, const uint4* __restrict__ Y, const float* __restrict__ w,
     const int32_t* __restrict__ ids, const int32_t* __restrict__ slot,
-    const int32_t* __restrict__ offsets, int T, int nv, int E, int k, uint4* __restrict__ out,
-    DeviceStatus* st) {
+    const int32_t* __restrict__ offsets, int T, int nv, int E, int k, long long max_rows,
+    uint4* __restrict__ out, DeviceStatus* st) {
     pdl_begin();
     constexpr int V = Tr::kVec;
     const int lane = threadIdx.x & 31;
@@ -157,8 +157,8 @@ __global__ void __launch_bounds__(256) combine_vec_kernel(
         if (s >= 0) {
             const int e = ids[p];
             if ((unsigned)e < (unsigned)E) {
-                const int r = offsets[e] + s;
-                if (r < offsets[e + 1]) { row = r; wt = w[p]; }
+                const long long r = (long long)offsets[e] + s;
+                if (r >= 0 && r < offsets[e + 1] && r < max_rows) { row = (int)r; wt = w[p]; }
                 else report(st, MOE_DEV_BAD_INDEX, 303);
             } else {
                 report(st, MOE_DEV_BAD_INDEX, 304);
@@ -215,8 +215,8 @@ template <class Tr, int KMAX>
 __global__ void __launch_bounds__(256) combine_token_block_kernel(
     const uint4* __restrict__ x, const uint4* __restrict__ Y, const float* __restrict__ w,
     const int32_t* __restrict__ ids, const int32_t* __restrict__ slot,
-    const int32_t* __restrict__ offsets, int nv, int E, int k, uint4* __restrict__ out,
-    DeviceStatus* st) {
+    const int32_t* __restrict__ offsets, int nv, int E, int k, long long max_rows,
+    uint4* __restrict__ out, DeviceStatus* st) {
     pdl_begin();
     constexpr int V = Tr::kVec;
     __shared__ int s_rows[KMAX];
@@ -233,8 +233,8 @@ __global__ void __launch_bounds__(256) combine_token_block_kernel(
             if (s >= 0) {
                 const int e = ids[p];
                 if ((unsigned)e < (unsigned)E) {
-                    const int r = offsets[e] + s;
-                    if (r < offsets[e + 1]) { row = r; wt = w[p]; }
+                    const long long r = (long long)offsets[e] + s;
+                    if (r >= 0 && r < offsets[e + 1] && r < max_rows) { row = (int)r; wt = w[p]; }
                     else report(st, MOE_DEV_BAD_INDEX, 305);
                 } else {
                     report(st, MOE_DEV_BAD_INDEX, 306);
@@ -298,6 +298,15 @@ __global__ void __launch_bounds__(256) ffn_f32_kernel(
     float* as = s_mem + d;      // [F]
     __shared__ int s_e;
     const int r = blockIdx.x;
+    // Row ranges given by the caller: offsets[0] = 0, non-decreasing, offsets[E] <= the rows of H
+    // and Y (the grid).  Bad offsets: nothing is stored, MOE_DEV_BAD_INDEX is recorded.
+    int bad = 0;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) bad |= offsets[e + 1] < offsets[e];
+    if (threadIdx.x == 0) bad |= offsets[0] != 0 || offsets[E] > (long long)gridDim.x;
+    if (__syncthreads_or(bad)) {
+        if (r == 0 && threadIdx.x == 0) report(st, MOE_DEV_BAD_INDEX, 402);
+        return;
+    }
     if (r >= offsets[E]) return;
     if (threadIdx.x == 0) {
         int lo = 0, hi = E - 1;                  // expert e with offsets[e] <= r < offsets[e+1]
@@ -367,7 +376,8 @@ void launch_logits_f32(const float* x, const float* Wr, const float* br, int T, 
 
 void launch_combine(int dtype, const void* x, const void* Y, const float* w, const int32_t* ids,
                     const int32_t* slot, const int32_t* offsets, int T, int d, int E, int k,
-                    void* out, DeviceStatus* st, cudaStream_t s, int* launches) {
+                    long long max_rows, void* out, DeviceStatus* st, cudaStream_t s,
+                    int* launches) {
     if (T == 0) return;
     const int blocks = (T + 7) / 8;
     const bool aligned = ((uintptr_t)x % 16 == 0) && ((uintptr_t)Y % 16 == 0) &&
@@ -376,32 +386,32 @@ void launch_combine(int dtype, const void* x, const void* Y, const float* w, con
         const int nv = d / 8;
         const int threads = std::min(256, ((nv + 31) / 32) * 32);
         launch_pdl(combine_token_block_kernel<BF16Traits, 8>, dim3(T), dim3(threads), 0, s,
-                   (const uint4*)x, (const uint4*)Y, w, ids, slot, offsets, nv, E, k, (uint4*)out,
-                   st);
+                   (const uint4*)x, (const uint4*)Y, w, ids, slot, offsets, nv, E, k, max_rows,
+                   (uint4*)out, st);
         *launches += 1;
         return;
     }
     if (dtype == MOE_BF16 && aligned && d % 8 == 0 && k <= 8) {
         launch_pdl(combine_vec_kernel<BF16Traits, 8>, dim3(blocks), dim3(256), 0, s,
                    (const uint4*)x, (const uint4*)Y, w, ids, slot, offsets, T, d / 8, E, k,
-                   (uint4*)out, st);
+                   max_rows, (uint4*)out, st);
         *launches += 1;
         return;
     }
     if (dtype == MOE_BF16) {
         if (aligned && d % 8 == 0)
             launch_pdl(combine_kernel<BF16Traits, true>, dim3(blocks), dim3(256), 0, s, x, Y, w,
-                       ids, slot, offsets, T, d, E, k, out, st);
+                       ids, slot, offsets, T, d, E, k, max_rows, out, st);
         else
             launch_pdl(combine_kernel<BF16Traits, false>, dim3(blocks), dim3(256), 0, s, x, Y, w,
-                       ids, slot, offsets, T, d, E, k, out, st);
+                       ids, slot, offsets, T, d, E, k, max_rows, out, st);
     } else {
         if (aligned && d % 4 == 0)
             launch_pdl(combine_kernel<F32Traits, true>, dim3(blocks), dim3(256), 0, s, x, Y, w, ids,
-                       slot, offsets, T, d, E, k, out, st);
+                       slot, offsets, T, d, E, k, max_rows, out, st);
         else
             launch_pdl(combine_kernel<F32Traits, false>, dim3(blocks), dim3(256), 0, s, x, Y, w,
-                       ids, slot, offsets, T, d, E, k, out, st);
+                       ids, slot, offsets, T, d, E, k, max_rows, out, st);
     }
     *launches += 1;
 }

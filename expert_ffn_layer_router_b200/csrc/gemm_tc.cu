@@ -60,6 +60,7 @@ struct GemmArgs {
     int a_row_limit;          // rows of A (bound for gathered indices)
     const int32_t* offsets;   // [E+1] row ranges of the groups; null = one group of rows0 rows
     int rows0;
+    int max_rows;             // rows of D (and of a contiguous A): offsets[E] must not exceed it
     int E;                    // groups
     int K;                    // reduction length, multiple of 64
     int n_tiles;              // column tiles per group
@@ -328,17 +329,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     if (warp == 2) {
-        // Tile prefix over groups: lane l sums groups [l*per, (l+1)*per).
+        // Tile prefix over groups: lane l sums groups [l*per, (l+1)*per).  Row ranges given by
+        // the caller are checked first: offsets[0] = 0, non-decreasing, offsets[E] <= max_rows,
+        // so every row of every tile lies inside D.  Bad offsets: no tile runs, nothing is
+        // stored, MOE_DEV_BAD_INDEX is recorded.
         const int per = (E + 31) / 32;
         int loc = 0;
+        bool bad = false;
         for (int q = 0; q < per; ++q) {
             const int e = lane * per + q;
             if (e < E) {
                 const int n = args.offsets ? __ldg(args.offsets + e + 1) - __ldg(args.offsets + e)
                                            : args.rows0;
+                bad |= n < 0;
                 loc += (max(n, 0) + TM - 1) / TM;
             }
         }
+        if (args.offsets && lane == 0)
+            bad |= __ldg(args.offsets) != 0 || __ldg(args.offsets + E) > args.max_rows;
+        bad = __any_sync(0xffffffffu, bad);
+        if (bad && lane == 0) report(st, MOE_DEV_BAD_INDEX, 510);
         int inc = loc;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -355,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 run += (max(n, 0) + TM - 1) / TM;
             }
         }
-        if (lane == 31) s_mt[E] = inc;
+        if (lane == 31) s_mt[E] = bad ? 0 : inc;
     }
     tc_fence_before();
     __syncwarp();
@@ -1015,6 +1025,7 @@ cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const in
     a.a_row_limit = a_row_limit;
     a.offsets = offsets;
     a.rows0 = 0;
+    a.max_rows = (int)max_rows;
     a.E = E;
     a.K = K;
     a.n_tiles = (Nout + BN - 1) / BN;
@@ -1067,6 +1078,7 @@ cudaError_t launch_gated_gemm(const void* A, long long lda, const int32_t* a_row
     a.a_rows = a_rows;
     a.a_row_limit = a_row_limit;
     a.offsets = offsets;
+    a.max_rows = (int)max_rows;
     a.E = E;
     a.K = K;
     a.n_tiles = F / 128;
@@ -1122,6 +1134,7 @@ cudaError_t launch_router_gemm(const void* x, int T, int d, const float* Wr, con
     a.a_row_limit = T;
     a.offsets = nullptr;
     a.rows0 = T;
+    a.max_rows = T;
     a.E = 1;
     a.K = d;
     a.n_tiles = ntl;

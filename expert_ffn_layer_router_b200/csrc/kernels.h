@@ -43,9 +43,12 @@ void launch_permute_rows(const void* x, const int32_t* rowtok, const int32_t* of
                          cudaStream_t s, int* launches);
 
 // combine.cu
+// max_rows: rows of Y; a kept pair whose row falls outside [0, max_rows) or outside its
+// expert's range is skipped and recorded as MOE_DEV_BAD_INDEX (st may be null).
 void launch_combine(int dtype, const void* x, const void* Y, const float* w, const int32_t* ids,
                     const int32_t* slot, const int32_t* offsets, int T, int d, int E, int k,
-                    void* out, DeviceStatus* st, cudaStream_t s, int* launches);
+                    long long max_rows, void* out, DeviceStatus* st, cudaStream_t s,
+                    int* launches);
 void launch_ffn_f32(const float* x, const int32_t* rowtok, const int32_t* offsets, int E, int T,
                     int d, int F, long long max_rows, const float* W1, const float* b1,
                     const float* W2, const float* b2, float* H, float* Y, DeviceStatus* st,

@@ -169,6 +169,98 @@ moe_status ffn_steps(const moe_problem* p, const void* x, const int32_t* offsets
     return MOE_OK;
 }
 
+// ------------------------------------------------------------------------------------------------
+// moe_route_static: moe_route for callers that cannot allocate device memory.
+//
+// Some callers have no way to hand the library a workspace: plug-ins inside an inference engine
+// that owns all device memory and gives its plug-ins no allocator, and latency-bound serving
+// loops whose policy forbids cudaMalloc/cudaFree on the request path (an allocation can
+// synchronise the device and stall every stream).  This entry point runs the same router and
+// capacity kernels as moe_route, with their scratch (per-chunk counts and prefixes, per-expert
+// candidate lists, the status word) placed in one file-scope __device__ array below.
+//
+// The array is a fixed kRouteStaticBytes per GPU, held by every GPU that loads the library until
+// the process exits.  Host code only sees a stand-in for it, so the device address is fetched
+// with cudaGetSymbolAddress on the first call in each CUDA context (the first call on a device,
+// for callers of the runtime's primary context) and cached per context.  The call allocates
+// nothing and calls no allocating routine.
+// ------------------------------------------------------------------------------------------------
+constexpr size_t kRouteStaticBytes = 8u << 20;   // 8 MiB per device
+constexpr int kStaticSlots = 64;      // cached (context, address) pairs
+
+__device__ __align__(256) unsigned char g_route_static_scratch[kRouteStaticBytes];
+
+struct StaticSlot {
+    std::atomic<void*> ctx{nullptr};
+    std::atomic<void*> ptr{nullptr};
+};
+StaticSlot g_static_slots[kStaticSlots];
+std::mutex g_static_mu;
+
+using CtxGetCurrentFn = int (*)(void**);     // cuCtxGetCurrent(CUcontext*)
+CtxGetCurrentFn g_ctx_get = nullptr;
+std::once_flag g_ctx_once;
+
+// The CUDA context current on this thread (null if none is bound yet).  The array has one
+// device address per context that loaded the library's module.
+void* current_context() {
+    std::call_once(g_ctx_once, []() {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_get = reinterpret_cast<CtxGetCurrentFn>(fn);
+    });
+    void* ctx = nullptr;
+    if (!g_ctx_get || g_ctx_get(&ctx) != 0) return nullptr;
+    return ctx;
+}
+
+// Scratch layout of moe_route inside the static array; returns the bytes it needs.
+size_t route_static_layout(const moe_problem* p, size_t* cnt, size_t* base, size_t* nrecv,
+                           size_t* cand) {
+    const size_t nC = (size_t)moe::chunk_count(p->T);
+    size_t off = align_up(sizeof(moe::DeviceStatus));
+    *cnt = off;
+    off = align_up(off + (size_t)p->E * nC * 4);
+    *base = off;
+    off = align_up(off + (size_t)p->E * nC * 4);
+    *nrecv = off;
+    off = align_up(off + (size_t)p->E * 4);
+    *cand = off;
+    off = align_up(off + (size_t)p->E * p->T * 4);
+    return off;
+}
+
+// Device address of the static array in the current context: the cached one, else looked up
+// (cudaGetSymbolAddress, which binds the device's primary context if none is current) and
+// cached.  With every slot taken the address is looked up on each call, uncached.
+void* static_scratch_for_current_context(cudaError_t* err) {
+    *err = cudaSuccess;
+    void* ctx = current_context();
+    if (ctx)
+        for (int i = 0; i < kStaticSlots; ++i)
+            if (g_static_slots[i].ctx.load(std::memory_order_acquire) == ctx)
+                return g_static_slots[i].ptr.load(std::memory_order_acquire);
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    void* ptr = nullptr;
+    *err = cudaGetSymbolAddress(&ptr, g_route_static_scratch);
+    if (*err != cudaSuccess) return nullptr;
+    ctx = current_context();
+    if (!ctx) return ptr;
+    for (int i = 0; i < kStaticSlots; ++i) {
+        void* c = g_static_slots[i].ctx.load(std::memory_order_relaxed);
+        if (c == ctx) return g_static_slots[i].ptr.load(std::memory_order_relaxed);
+        if (c == nullptr) {
+            g_static_slots[i].ptr.store(ptr, std::memory_order_relaxed);
+            g_static_slots[i].ctx.store(ctx, std::memory_order_release);
+            return ptr;
+        }
+    }
+    return ptr;
+}
+
 }  // namespace
 
 extern "C" {
@@ -247,15 +339,18 @@ moe_status moe_expert_ffn(const moe_problem* p, const void* x, const int32_t* of
 
 moe_status moe_combine(const moe_problem* p, const void* x, const void* Y, const float* w,
                        const int32_t* ids, const int32_t* slot, const int32_t* offsets,
-                       void* out, void* stream) {
+                       void* out, void* ws, size_t ws_bytes, void* stream) {
     moe_status r = pre(p, false);
     if (r != MOE_OK) return r;
     if (p->T > 0 && (!x || !Y || !w || !ids || !slot || !offsets || !out))
         return MOE_ERR_INVALID_ARG;
     if (out && (out == x || out == Y)) return MOE_ERR_INVALID_ARG;
+    if (ws && (ws_bytes < kAlign || misaligned(ws, kAlign))) return MOE_ERR_WORKSPACE;
     int launches = 0;
     moe::launch_combine(p->dtype, x, Y, w, ids, slot, offsets, p->T, p->d_model, p->E, p->k,
-                        out, nullptr, (cudaStream_t)stream, &launches);
+                        max_rows_of(p, capacity_of(p)), out,
+                        ws ? at<moe::DeviceStatus>(ws, 0) : nullptr, (cudaStream_t)stream,
+                        &launches);
     return finish(launches);
 }
 
@@ -347,14 +442,22 @@ moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, con
         stage_mark(4, s);
         stage_mark(5, s);
     }
-    moe::launch_combine(p->dtype, x, Y, w, ids, slot, offsets, p->T, p->d_model, p->E, p->k, out,
-                        st, s, &launches);
+    moe::launch_combine(p->dtype, x, Y, w, ids, slot, offsets, p->T, p->d_model, p->E, p->k, R,
+                        out, st, s, &launches);
     stage_mark(6, s);
     return finish(launches);
 }
 
 moe_status moe_get_device_status(const void* ws, size_t ws_bytes, void* stream, int32_t* code) {
-    if (!ws || !code || ws_bytes < sizeof(moe::DeviceStatus)) return MOE_ERR_INVALID_ARG;
+    if (!code) return MOE_ERR_INVALID_ARG;
+    if (!ws) {
+        // The status word of moe_route_static's scratch on the current device.
+        cudaError_t err;
+        ws = static_scratch_for_current_context(&err);
+        if (!ws) return MOE_ERR_CUDA;
+        ws_bytes = sizeof(moe::DeviceStatus);
+    }
+    if (ws_bytes < sizeof(moe::DeviceStatus)) return MOE_ERR_INVALID_ARG;
     moe::DeviceStatus h{};
     if (cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, (cudaStream_t)stream) !=
             cudaSuccess ||
@@ -365,7 +468,13 @@ moe_status moe_get_device_status(const void* ws, size_t ws_bytes, void* stream, 
 }
 
 moe_status moe_reset_device_status(void* ws, size_t ws_bytes, void* stream) {
-    if (!ws || ws_bytes < sizeof(moe::DeviceStatus)) return MOE_ERR_INVALID_ARG;
+    if (!ws) {
+        cudaError_t err;
+        ws = static_scratch_for_current_context(&err);
+        if (!ws) return MOE_ERR_CUDA;
+        ws_bytes = sizeof(moe::DeviceStatus);
+    }
+    if (ws_bytes < sizeof(moe::DeviceStatus)) return MOE_ERR_INVALID_ARG;
     if (cudaMemsetAsync(ws, 0, sizeof(moe::DeviceStatus), (cudaStream_t)stream) != cudaSuccess)
         return MOE_ERR_CUDA;
     return MOE_OK;
@@ -410,69 +519,6 @@ const char* moe_status_string(moe_status s) {
 
 }  // extern "C"
 
-// ------------------------------------------------------------------------------------------------
-// moe_route_static: moe_route for callers that cannot allocate device memory.
-//
-// Some callers have no way to hand the library a workspace: plug-ins inside an inference engine
-// that owns all device memory and gives its plug-ins no allocator, and latency-bound serving
-// loops whose policy forbids cudaMalloc/cudaFree on the request path (an allocation can
-// synchronise the device and stall every stream).  This entry point runs the same router and
-// capacity kernels as moe_route, with their scratch (per-chunk counts and prefixes, per-expert
-// candidate lists, the status word) placed in one file-scope __device__ array below.
-//
-// The array is a fixed kRouteStaticBytes per GPU, held by every GPU that loads the library until
-// the process exits.  Host code only sees a stand-in for it, so the device address is fetched
-// with cudaGetSymbolAddress once per device (first call on that device, with it current) and
-// cached.  The call allocates nothing and calls no allocating routine.
-// ------------------------------------------------------------------------------------------------
-namespace {
-
-constexpr size_t kRouteStaticBytes = 8u << 20;   // 8 MiB per device
-constexpr int kMaxStaticDevices = 64;
-
-__device__ __align__(256) unsigned char g_route_static_scratch[kRouteStaticBytes];
-
-std::mutex g_static_mu;
-std::atomic<void*> g_static_ptr[kMaxStaticDevices];
-
-// Scratch layout of moe_route inside the static array; returns the bytes it needs.
-size_t route_static_layout(const moe_problem* p, size_t* cnt, size_t* base, size_t* nrecv,
-                           size_t* cand) {
-    const size_t nC = (size_t)moe::chunk_count(p->T);
-    size_t off = align_up(sizeof(moe::DeviceStatus));
-    *cnt = off;
-    off = align_up(off + (size_t)p->E * nC * 4);
-    *base = off;
-    off = align_up(off + (size_t)p->E * nC * 4);
-    *nrecv = off;
-    off = align_up(off + (size_t)p->E * 4);
-    *cand = off;
-    off = align_up(off + (size_t)p->E * p->T * 4);
-    return off;
-}
-
-void* static_scratch_for_current_device(cudaError_t* err) {
-    int dev = 0;
-    *err = cudaGetDevice(&dev);
-    if (*err != cudaSuccess) return nullptr;
-    if (dev < 0 || dev >= kMaxStaticDevices) {
-        *err = cudaErrorInvalidDevice;
-        return nullptr;
-    }
-    void* ptr = g_static_ptr[dev].load(std::memory_order_acquire);
-    if (ptr) return ptr;
-    std::lock_guard<std::mutex> lock(g_static_mu);
-    ptr = g_static_ptr[dev].load(std::memory_order_relaxed);
-    if (!ptr) {
-        *err = cudaGetSymbolAddress(&ptr, g_route_static_scratch);
-        if (*err != cudaSuccess) return nullptr;
-        g_static_ptr[dev].store(ptr, std::memory_order_release);
-    }
-    return ptr;
-}
-
-}  // namespace
-
 extern "C" moe_status moe_route_static(const moe_problem* p, const float* logits, int32_t* ids,
                                        float* w, int32_t* slot, uint8_t* drop, int32_t* counts,
                                        void* stream) {
@@ -484,7 +530,7 @@ extern "C" moe_status moe_route_static(const moe_problem* p, const float* logits
     if (route_static_layout(p, &o_cnt, &o_base, &o_nrecv, &o_cand) > kRouteStaticBytes)
         return MOE_ERR_WORKSPACE;
     cudaError_t err;
-    void* scratch = static_scratch_for_current_device(&err);
+    void* scratch = static_scratch_for_current_context(&err);
     if (!scratch) return MOE_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
     if (p->T == 0) {

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 MOE_F32, MOE_BF16 = 0, 1
 FLAG_RENORMALIZE, FLAG_ARRIVAL_ORDER, FLAG_GATED = 1, 2, 4
 MOE_OK = 0
+MOE_ERR_DEVICE = 5       # the status word holds an error (moe_get_device_status)
 DEV_OK, DEV_TIMEOUT, DEV_BAD_INDEX = 0, 1, 2
 
 
@@ -48,7 +49,7 @@ def _load():
         "moe_route": [P, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "moe_dispatch": [P, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "moe_expert_ffn": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
-        "moe_combine": [P, vp, vp, vp, vp, vp, vp, vp, vp],
+        "moe_combine": [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "moe_forward": [P] + [vp] * 15 + [sz, vp],
         "moe_get_device_status": [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)],
         "moe_reset_device_status": [vp, sz, vp],
@@ -146,9 +147,11 @@ def moe_expert_ffn(p, x, offsets, rowtok, W1, b1, W2, b2, Y, ws, stream=None):
            "moe_expert_ffn")
 
 
-def moe_combine(p, x, Y, w, ids, slot, offsets, out, stream=None):
+def moe_combine(p, x, Y, w, ids, slot, offsets, out, ws=None, stream=None):
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check(_lib.moe_combine(ctypes.byref(p), _ptr(x), _ptr(Y), _ptr(w), _ptr(ids), _ptr(slot),
-                            _ptr(offsets), _ptr(out), _stream(stream)), "moe_combine")
+                            _ptr(offsets), _ptr(out), _ptr(ws), nbytes, _stream(stream)),
+           "moe_combine")
 
 
 def moe_forward(p, x, Wr, br, W1, b1, W2, b2, out, ws, logits_out=None, ids_out=None,
@@ -161,15 +164,19 @@ def moe_forward(p, x, Wr, br, W1, b1, W2, b2, out, ws, logits_out=None, ids_out=
 
 
 def moe_get_device_status(ws, stream=None) -> int:
+    """Status word of ``ws``; ``ws=None``: that of moe_route_static on the current device."""
     code = ctypes.c_int32()
-    _lib.moe_get_device_status(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream),
-                               ctypes.byref(code))
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    rc = _lib.moe_get_device_status(_ptr(ws), nbytes, _stream(stream), ctypes.byref(code))
+    if rc not in (MOE_OK, MOE_ERR_DEVICE):
+        raise MoeError(rc, "moe_get_device_status")
     return code.value
 
 
 def moe_reset_device_status(ws, stream=None):
-    _check(_lib.moe_reset_device_status(_ptr(ws), ws.numel() * ws.element_size(),
-                                        _stream(stream)), "moe_reset_device_status")
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_lib.moe_reset_device_status(_ptr(ws), nbytes, _stream(stream)),
+           "moe_reset_device_status")
 
 
 def moe_selftest_wait_timeout(ws, limit_us, stream=None):
@@ -255,5 +262,5 @@ class MoELayer:
 
     def combine(self, x, Y, w, ids, slot, offsets, stream=None):
         out = torch.empty_like(x)
-        moe_combine(self.p, x, Y, w, ids, slot, offsets, out, stream)
+        moe_combine(self.p, x, Y, w, ids, slot, offsets, out, self.ws, stream)
         return out

@@ -131,7 +131,10 @@ moe_status moe_dispatch(const moe_problem* p, const int32_t* ids, const int32_t*
  * [offsets[e], offsets[e+1]): Y[r] = W2[e] SiLU(W1[e] x[rowtok[r]] + b1[e]) + b2[e].
  * The token gather is folded into the first GEMM's operand load; nothing is materialised but
  * the hidden activations (in ws, x's dtype).  Y is [min(T*k, E*K), d_model] in x's dtype.
- * b1, b2 may be NULL (zero bias). */
+ * b1, b2 may be NULL (zero bias).
+ * The kernels check offsets on the device: offsets[0] = 0, non-decreasing, offsets[E] <=
+ * min(T*k, E*K).  If not, nothing is written to Y or H and MOE_DEV_BAD_INDEX is recorded.  A
+ * rowtok entry outside [0, T) is recorded the same way and its row is computed from zeros. */
 moe_status moe_expert_ffn(const moe_problem* p, const void* x, const int32_t* offsets,
                           const int32_t* rowtok, const void* W1, const float* b1,
                           const void* W2, const float* b2, void* Y, void* ws, size_t ws_bytes,
@@ -139,10 +142,14 @@ moe_status moe_expert_ffn(const moe_problem* p, const void* x, const int32_t* of
 
 /* Combine (step 4): out[t] = x[t] + sum over kept j (ascending) of w[t*k+j] * Y[offsets[id]
  * + slot], accumulated in float32 and rounded once; out[t] = x[t] bit for bit when no pair of
- * t is kept.  out must not alias x or Y. */
+ * t is kept.  out must not alias x or Y.  Y has min(T*k, E*K) rows.
+ *   ws (nullable, 256-byte aligned, ws_bytes >= 256): only its status word is used.  A kept
+ *   pair whose expert id is out of range, or whose row offsets[id] + slot lies outside
+ *   [offsets[id], offsets[id+1]) or outside Y, is skipped (its term is left out) and recorded
+ *   as MOE_DEV_BAD_INDEX in ws's status word; with ws = NULL it is skipped silently. */
 moe_status moe_combine(const moe_problem* p, const void* x, const void* Y, const float* w,
                        const int32_t* ids, const int32_t* slot, const int32_t* offsets,
-                       void* out, void* stream);
+                       void* out, void* ws, size_t ws_bytes, void* stream);
 
 /* The whole layer: logits = x Wr + br (Wr [d_model, E] float32, br [E] float32 or NULL), then
  * the four steps.  out [T, d_model] in x's dtype.  Optional outputs (NULL = keep in ws):
@@ -173,8 +180,13 @@ moe_status moe_set_stage_events(void* const* events, int32_t n);
  *   16 + 8*E*ceil(T/32) + 4*E + 4*E*T bytes (each part rounded up to 256); larger problems get
  *   MOE_ERR_WORKSPACE before anything is launched (T=16384 with E=64 fits; T=65536 with E=128
  *   does not).
- *   The first call on a device looks up the array's device address (with that device current)
- *   and caches it; make that first call before any stream capture.
+ *   The first call in a CUDA context (for runtime-API callers: the first call on a device) looks
+ *   up the array's device address in that context and caches it; make that first call before
+ *   any stream capture.  The cached address dies with its context: do not call it across a
+ *   cudaDeviceReset of that device.
+ *   The status word lives in the array too: each call clears it when it starts, and
+ *   moe_get_device_status(NULL, 0, stream, &code) reads it (MOE_DEV_BAD_INDEX for an id out of
+ *   range).
  *   Every call on a device shares the one array: calls that overlap on the GPU (other streams,
  *   other host threads) race and corrupt each other's results; serialise them.  Nothing is
  *   allocated, and no allocating routine is called. */
@@ -188,10 +200,13 @@ moe_status moe_route_static(const moe_problem* p, const float* logits, int32_t* 
  * read the result with moe_get_device_status. */
 moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, int32_t limit_us, void* stream);
 
-/* Reads the device status word of `ws` (synchronises `stream`). */
+/* Reads the device status word of `ws` (synchronises `stream`).  ws = NULL reads the status word
+ * of moe_route_static's fixed scratch on the current device, which that call clears when it
+ * starts: it holds the result of the latest moe_route_static call there. */
 moe_status moe_get_device_status(const void* ws, size_t ws_bytes, void* stream, int32_t* code);
 
-/* Clears the device status word of `ws` (asynchronous on `stream`). */
+/* Clears the device status word of `ws` (asynchronous on `stream`); ws = NULL: the status word of
+ * moe_route_static's scratch on the current device. */
 moe_status moe_reset_device_status(void* ws, size_t ws_bytes, void* stream);
 
 /* Kernel launches made by the most recent successful compute call on this host thread. */

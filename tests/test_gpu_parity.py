@@ -184,7 +184,28 @@ def test_combine_parity(T, d, E, k, C, dtype):
 # ------------------------------------------------------------------------------------------
 # The fused forward against the oracle's whole layer.
 # ------------------------------------------------------------------------------------------
+def _assert_forward_route_equal(g, ro, E):
+    """The forward's exported routing against the oracle's routing of the same fp32 logits."""
+    assert np.array_equal(g["ids_out"], ro["ids"]), "expert ids differ"
+    assert np.array_equal(g["w_out"].view(np.uint32), ro["w"].view(np.uint32)), "weights differ"
+    assert np.array_equal(g["slot_out"], ro["slot"]), "slot map differs"
+    assert np.array_equal(g["drop_out"], ro["drop"]), "drop mask differs"
+    assert np.array_equal(g["counts_out"][:E], ro["received"]), "received counts differ"
+    assert np.array_equal(g["counts_out"][E:], ro["kept"]), "kept counts differ"
+
+
 def _forward_check(spec, seed, tokens=None, logit_rel=1e-4, flags=0):
+    """The whole forward against the oracle.
+
+    1. logits_out within logit_rel * max(1, max|L|) of the oracle's float64 x Wr + br;
+    2. routing (ids, weight bits, slots, drop mask, counts) bit for bit equal to the oracle's
+       routing of the forward's own exported fp32 logits (routing is a function of the logits);
+    3. outputs of ``tokens`` (all by default) within the dtype's tolerance of the oracle's
+       layer given that routing; tokens with no kept pair bit for bit equal to x;
+    4. against the oracle's routing of its own logits: the same expert sets, and capacity
+       decisions that differ only where the oracle's weights tie within the logit error at an
+       expert's capacity boundary (the logits differ by rounding).
+    """
     moe = _moe()
     L = inputs.make_layer(spec, seed=seed)
     layer = moe.MoELayer(spec.T, spec.d_model, spec.d_ff, spec.E, spec.k, spec.C, spec.dtype,
@@ -197,11 +218,20 @@ def _forward_check(spec, seed, tokens=None, logit_rel=1e-4, flags=0):
     Lref = oracle.logits(L["x"], L["Wr"], L["br"])
     lerr = np.abs(g["logits_out"] - Lref).max()
     assert lerr <= logit_rel * max(1.0, float(np.abs(Lref).max())), lerr
+    rg = oracle.route(g["logits_out"], spec.k, layer.K, flags & 3)
+    _assert_forward_route_equal(g, rg, spec.E)
+    T = spec.T
+    if tokens is None:
+        tokens = np.arange(T, dtype=np.int32)
+    tokens = np.asarray(tokens, dtype=np.int32)
+    _, ref = oracle.combine_tokens(L["x"], L["W1"], L["b1"], L["W2"], L["b2"], rg, tokens,
+                                   flags=flags)
+    got = to_host(out)
+    assert_close(got[tokens], ref, spec.dtype, "layer output")
+    none_kept = ~(rg["slot"] >= 0).any(axis=1)
+    assert got[none_kept].tobytes() == L["x"][none_kept].tobytes()
+    # Against the routing of the oracle's own logits.
     ro = oracle.route(Lref, spec.k, layer.K, flags & 3)
-    # The logits differ from the oracle's by rounding, so the order of a token's experts can
-    # differ where two of its top-k logits are that close; compare per (token, expert) pair.
-    # Expert choice itself is pinned by the gap screen; capacity decisions may only differ where
-    # the oracle's own weights tie within the logit error at an expert's capacity boundary.
     og = np.argsort(g["ids_out"], axis=1, kind="stable")
     oo = np.argsort(ro["ids"], axis=1, kind="stable")
     gi, gw, gs = (np.take_along_axis(g[n], og, 1) for n in ("ids_out", "w_out", "slot_out"))
@@ -217,19 +247,8 @@ def _forward_check(spec, seed, tokens=None, logit_rel=1e-4, flags=0):
         drop_w = ow[same_e & (os_ < 0)]
         boundary = (kept_w.min() + drop_w.max()) / 2
         assert abs(float(ow[t, j]) - boundary) <= 8 * dw.max() + 1e-7, "not a near-tie"
-    agree = ((gs >= 0) == (os_ >= 0)).all(axis=1)
-    assert agree.mean() >= 0.99
-    T = spec.T
-    if tokens is None:
-        tokens = np.arange(T, dtype=np.int32)
-    tokens = np.array([t for t in tokens if agree[t]], dtype=np.int32)
-    _, ref = oracle.combine_tokens(L["x"], L["W1"], L["b1"], L["W2"], L["b2"], ro, tokens,
-                                   flags=flags)
-    got = to_host(out)
-    assert_close(got[tokens], ref, spec.dtype, "layer output")
-    none_kept = ~(ro["slot"] >= 0).any(axis=1) & agree
-    assert got[none_kept].tobytes() == L["x"][none_kept].tobytes()
-    return g, ro
+    assert ((gs >= 0) == (os_ >= 0)).all(axis=1).mean() >= 0.99
+    return g, rg
 
 
 @pytest.mark.parametrize("spec", [
@@ -276,9 +295,8 @@ def test_unsupported_and_invalid():
 
 # ------------------------------------------------------------------------------------------
 # Fused router: with bf16 and E <= 64 the logits GEMM's epilogue also forms the softmax, the
-# top-k and the per-chunk counts.  Its routing must equal moe_route's on the same logits bit for
-# bit (moe_route itself is bit-exact against the oracle above), so the chain reaches the oracle
-# without feeding it anything computed on the GPU.
+# top-k and the per-chunk counts.  Its routing must equal, bit for bit, both moe_route's and the
+# oracle's routing of the logits the forward exported.
 # ------------------------------------------------------------------------------------------
 @pytest.mark.parametrize("T,d,E,k,C", [(3000, 128, 64, 6, 1.0), (1000, 256, 8, 2, 1.25),
                                        (777, 64, 33, 4, 0.75), (200, 64, 16, 8, math.inf),
@@ -300,6 +318,9 @@ def test_fused_router_matches_route(T, d, E, k, C, flags):
     assert torch.equal(rt["slot_out"], r["slot"])
     assert torch.equal(rt["drop_out"], r["drop"])
     assert torch.equal(rt["counts_out"], r["counts"])
+    g = {k_: to_host(v) for k_, v in rt.items()}
+    ro = oracle.route(g["logits_out"], k, layer.K, flags & 3)
+    _assert_forward_route_equal(g, ro, E)
 
 
 # ------------------------------------------------------------------------------------------
@@ -461,6 +482,86 @@ def test_forward_writes_stay_inside_outputs_and_workspace(spec):
         assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
     else:
         assert torch.equal(out, ref)
+
+
+# ------------------------------------------------------------------------------------------
+# Caller-supplied dispatch data is checked on the device.  moe_expert_ffn with offsets whose
+# total exceeds the row count by one row, or that decrease, stores nothing: the guard regions
+# around Y and the workspace (each larger than one 128-row output tile) survive, Y keeps its
+# fill pattern, and the status word says MOE_DEV_BAD_INDEX.  Good offsets then run normally.
+# ------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("defect", ["one_row_too_many", "decreasing", "nonzero_start"])
+def test_expert_ffn_rejects_bad_offsets(dtype, defect):
+    moe = _moe()
+    T, d, F, E, k = 300, 128, 192, 5, 2
+    spec = inputs.LayerSpec("bad", T, d, F, E, k, math.inf, dtype, router="normal",
+                            router_bias=0.5, bias_std=0.05)
+    L = inputs.make_layer(spec, seed=1)
+    ro = oracle.route(oracle.logits(L["x"], L["Wr"], L["br"]), k, T)
+    off, rowtok = oracle.dispatch(ro["ids"], ro["slot"], E)
+    R = T * k
+    assert int(off[-1]) == R                          # dropless: every row of Y is used
+    bad = off.copy()
+    if defect == "one_row_too_many":
+        bad[-1] = R + 1
+    elif defect == "decreasing":
+        bad[2], bad[3] = bad[3], bad[2]
+    else:
+        bad[0] = 1
+    p = moe.problem(T, d, F, E, k, math.inf, dtype)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    guard = 128 * d * 4 * 2                           # bytes: more than one output tile
+    ws_raw, ws, gb = _guarded(moe.moe_workspace_size(p), torch.uint8, guard_bytes=guard)
+    y_raw, Y, gy = _guarded(R * d, tdt, guard_bytes=guard)
+    y_before = y_raw.clone()
+    args = [to_dev(L[n]) for n in ("x", "W1", "b1", "W2", "b2")]
+    moe.moe_reset_device_status(ws)
+    moe.moe_expert_ffn(p, args[0], to_dev(bad), to_dev(rowtok), args[1], args[2], args[3],
+                       args[4], Y, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == moe.DEV_BAD_INDEX
+    assert _guards_intact(ws_raw, gb) and _guards_intact(y_raw, gy)
+    assert torch.equal(y_raw, y_before), "nothing may be stored with bad offsets"
+    moe.moe_reset_device_status(ws)
+    moe.moe_expert_ffn(p, args[0], to_dev(off), to_dev(rowtok), args[1], args[2], args[3],
+                       args[4], Y, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == 0
+    row_exp = np.repeat(np.arange(E, dtype=np.int32), np.diff(off))
+    Yref = oracle.expert_rows(L["x"], L["W1"], L["b1"], L["W2"], L["b2"], rowtok, row_exp)
+    assert_close(to_host(Y.view(R, d)), Yref, dtype, "expert outputs after bad offsets")
+
+
+def test_combine_reports_rows_outside_y():
+    # The last expert's range is moved so that some of its rows fall past the end of Y: those
+    # terms are skipped and reported in the workspace's status word; tokens routed elsewhere
+    # are unaffected.
+    moe = _moe()
+    T, d, E, k, C = 400, 64, 6, 2, 0.8
+    L = inputs.random_logits(T, E, 21)
+    K = oracle.capacity(T, E, k, C)
+    ro = oracle.route(L, k, K)
+    off, _ = oracle.dispatch(ro["ids"], ro["slot"], E)
+    R = min(T * k, E * K)
+    rng = np.random.default_rng(4)
+    x = inputs.f32_to_bf16_bits(rng.standard_normal((T, d)).astype(np.float32))
+    Y = inputs.f32_to_bf16_bits(rng.standard_normal((R, d)).astype(np.float32))
+    layer = moe.MoELayer(T, d, 64, E, k, C, "bf16")
+    args = [to_dev(a) for a in (x, Y, ro["w"], ro["ids"], ro["slot"])]
+    good = layer.combine(*args, to_dev(off))
+    bad = off.copy()
+    last_kept = int(off[E] - off[E - 1])
+    assert last_kept >= 2
+    bad[E - 1] = R - 1                                 # slot s of expert E-1 -> row R - 1 + s
+    bad[E] = R + 1000
+    moe.moe_reset_device_status(layer.ws)
+    out = layer.combine(*args, to_dev(bad))
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(layer.ws) == moe.DEV_BAD_INDEX
+    elsewhere = ~((ro["ids"] == E - 1) & (ro["slot"] >= 0)).any(axis=1)
+    assert torch.equal(out[torch.from_numpy(elsewhere).cuda()].view(torch.int16),
+                       good[torch.from_numpy(elsewhere).cuda()].view(torch.int16))
 
 
 # ------------------------------------------------------------------------------------------

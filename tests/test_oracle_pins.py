@@ -356,6 +356,120 @@ def test_capacity_zero_is_identity():
 
 
 # ------------------------------------------------------------------------------------------
+# Combine from given expert outputs (the checker of the standalone combine kernel).
+# Definition (worked example, token-0 trace "x0 + w0 * y0" and the dropped token 4; the
+# dataflow diagram's moe_sum for top_k > 1): out[t] = x[t] + sum over kept j, ascending, of
+# w[t, j] * Y[offsets[ids[t, j]] + slot[t, j]], in float64, rounded once; a token with no kept
+# pair is x[t] bit for bit.  The reference below is numpy fancy indexing in float64, written
+# from that definition and sharing nothing with the oracle's loops.
+# ------------------------------------------------------------------------------------------
+
+def _combine_reference(x64, Y64, route, offsets):
+    ids, w, slot = route["ids"], route["w"], route["slot"]
+    T, k = ids.shape
+    kept = slot >= 0
+    rows = np.where(kept, offsets[ids] + slot, 0)
+    s = np.zeros_like(x64)
+    for j in range(k):                                   # j ascending, as the definition
+        s = s + np.where(kept[:, j, None], w[:, j, None].astype(np.float64) * Y64[rows[:, j]],
+                         0.0)
+    return x64 + s, kept.any(axis=1)
+
+
+def _bf16_of_f64(v):
+    return np.array([oracle.bf16_from_double(float(a)) for a in v.reshape(-1)],
+                    dtype=np.uint16).reshape(v.shape)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T,d,E,k,C,seed", [(60, 12, 5, 3, 0.5, 0), (40, 8, 4, 1, 0.75, 1),
+                                             (33, 16, 8, 8, 0.4, 2), (20, 4, 3, 2, 0.0, 3)])
+def test_combine_given_y_matches_definition(dtype, T, d, E, k, C, seed):
+    L = inputs.random_logits(T, E, seed + 40, 2.0)
+    K = oracle.capacity(T, E, k, C)
+    r = oracle.route(L, k, K)
+    off, _ = oracle.dispatch(r["ids"], r["slot"], E)
+    n = int(off[-1])
+    rng = np.random.default_rng(seed)
+    x32 = rng.standard_normal((T, d)).astype(np.float32)
+    # Large expert outputs against a unit residual: a float32 accumulation of the k terms
+    # would round away low bits that the float64 sum keeps, and change the rounded output.
+    Y32 = (rng.standard_normal((max(n, 1), d)) * 1e4).astype(np.float32)
+    none_kept = ~(r["slot"] >= 0).any(axis=1)
+    if dtype == "bf16":
+        x, Y = inputs.f32_to_bf16_bits(x32), inputs.f32_to_bf16_bits(Y32)
+        if none_kept.any():
+            x[np.nonzero(none_kept)[0][0], 0] = 0x8000           # -0.0
+    else:
+        x, Y = x32, Y32
+        if none_kept.any():
+            x[np.nonzero(none_kept)[0][0], 0] = np.float32(-0.0)
+    out64, out = oracle.combine_given_y(x, Y, r, off)
+    ref64, any_kept = _combine_reference(_f64(x), _f64(Y), r, off)
+    # Same float64 operations in the same order: identical to the last bit.
+    assert np.array_equal(out64, ref64)
+    if dtype == "f32":
+        assert np.array_equal(out[any_kept], ref64[any_kept].astype(np.float32))
+    else:
+        assert np.array_equal(out[any_kept], _bf16_of_f64(ref64[any_kept]))
+    assert out[none_kept].tobytes() == x[none_kept].tobytes()
+    if C == 0.0:
+        assert none_kept.all()
+    elif k > 1:
+        partly = (r["slot"] >= 0).any(axis=1) & (r["slot"] < 0).any(axis=1)
+        assert partly.any(), "the case must hold partially dropped tokens"
+
+
+def test_combine_given_y_detects_float_accumulation():
+    # w = 0.1f times Y = 2^24 - 1 and -(2^24 - 2): both products are exact in float64 and their
+    # sum is exactly w, but each product rounds to a multiple of 1/8 in float32, so a float32
+    # accumulation gives 0 or 0.125 instead of 0.1f.  Pins the float64 accumulation.
+    w32 = np.float32(0.1)
+    x = np.zeros((1, 1), np.float32)
+    Y = np.array([[16777215.0], [-16777214.0]], np.float32)
+    route = dict(ids=np.array([[0, 1]], np.int32), w=np.array([[w32, w32]], np.float32),
+                 slot=np.array([[0, 0]], np.int32))
+    off = np.array([0, 1, 2], np.int32)
+    out64, out = oracle.combine_given_y(x, Y, route, off)
+    f32_sum = np.float32(np.float32(w32 * Y[0, 0]) + np.float32(w32 * Y[1, 0]))
+    assert f32_sum != w32
+    assert out64[0, 0] == float(w32) and out[0, 0] == w32
+
+
+def test_combine_given_y_agrees_with_combine_tokens():
+    # Expert outputs from the oracle's own FFN rows (pinned against torch float64 above), then
+    # the standalone combine: the same layer output as the fused oracle path.
+    spec = inputs.LayerSpec("cg", 48, 16, 24, 6, 2, 0.6, "f32", router="normal",
+                            router_bias=0.3, bias_std=0.1)
+    layer = inputs.make_layer(spec, seed=3)
+    res = oracle.forward(layer["x"], layer["Wr"], layer["br"], layer["W1"], layer["b1"],
+                         layer["W2"], layer["b2"], 2, 0.6)
+    off, rowtok = oracle.dispatch(res["route"]["ids"], res["route"]["slot"], 6)
+    row_exp = np.repeat(np.arange(6, dtype=np.int32), np.diff(off))
+    Y = oracle.expert_rows(layer["x"], layer["W1"], layer["b1"], layer["W2"], layer["b2"],
+                           rowtok, row_exp).astype(np.float32)
+    out64, out = oracle.combine_given_y(layer["x"], Y, res["route"], off)
+    np.testing.assert_allclose(out64, res["out_f64"], rtol=0, atol=1e-5)
+    dropped = (res["route"]["slot"] < 0).any(axis=1)
+    assert dropped.any()
+
+
+def test_worked_example_combine_given_y():
+    # Token 0 keeps its expert: out0 = x0 + w0 * y0 with y0 the row at offsets[0] + slot; token
+    # 4 is dropped and comes back unchanged.
+    layer = inputs.make_layer(inputs.CONFIGS["tiny_f32"], seed=0)
+    r = oracle.route(layer["logits"], 1, 2)
+    off, rowtok = oracle.dispatch(r["ids"], r["slot"], 4)
+    Y = np.arange(int(off[-1]) * 4, dtype=np.float32).reshape(-1, 4) / 8.0
+    out64, out = oracle.combine_given_y(layer["x"], Y, r, off)
+    row0 = int(off[r["ids"][0, 0]] + r["slot"][0, 0])
+    assert rowtok[row0] == 0
+    np.testing.assert_array_equal(
+        out64[0], layer["x"][0].astype(np.float64) + float(r["w"][0, 0]) * Y[row0].astype(np.float64))
+    assert out[4].tobytes() == layer["x"][4].tobytes()
+
+
+# ------------------------------------------------------------------------------------------
 # Logits and bfloat16 rounding
 # ------------------------------------------------------------------------------------------
 

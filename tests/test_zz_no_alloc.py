@@ -7,6 +7,7 @@ a row (the array keeps the previous call's contents), whether this file runs alo
 process or after every other test.  This file is named to be collected last.
 """
 import ctypes
+import math
 
 import numpy as np
 import pytest
@@ -37,14 +38,15 @@ def _call_static(moe, p, logits, o):
                                       vp(o["counts"].data_ptr()), vp(s))
 
 
-def _check_pair(moe, spec_T, E, k, C, logits_np):
+def _check_pair(moe, spec_T, E, k, C, logits_np, flags=0):
     dev = torch.device("cuda:0")
-    layer = moe.MoELayer(spec_T, 64, 64, E, k, C, "bf16", device=dev)
+    layer = moe.MoELayer(spec_T, 64, 64, E, k, C, "bf16", device=dev, flags=flags)
     logits = to_dev(logits_np)
     ref = layer.route(logits)                                   # the workspace entry point
     got = _outputs(layer.p, dev)
     assert _call_static(moe, layer.p, logits, got) == 0
     torch.cuda.synchronize()
+    assert moe.moe_get_device_status(None) == 0                 # the static status word
     for name in ("ids", "slot", "drop", "counts"):
         assert torch.equal(got[name], ref[name]), name
     assert torch.equal(got["w"].view(torch.int32), ref["w"].view(torch.int32))
@@ -72,3 +74,25 @@ def test_static_route_rejects_problems_beyond_its_scratch():
     o = _outputs(moe.problem(1, 64, 64, 128, 8, 1.5, "bf16"), torch.device("cuda:0"))
     x = torch.zeros(1, device="cuda:0")
     assert _call_static(moe, p, x, o) == 3                       # MOE_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("T,E,k,C,flags", [
+    (64, 64, 8, math.inf, 0),       # decode shape: moe_route takes its single-block dispatch
+    (8, 4, 1, 1.25, 0),             # the worked example's shape (token 4 is dropped)
+    (100, 16, 4, 0.5, 0),           # small batch with drops
+    (3000, 20, 3, 0.8, 1),          # renormalised weights
+    (3000, 20, 3, 0.8, 2),          # arrival-order capacity
+    (120, 10, 3, 0.6, 3),           # both flags, small batch
+])
+def test_static_route_matches_workspace_route_small_batches_and_flags(T, E, k, C, flags):
+    from expert_ffn_layer_router_b200 import moe
+    if (T, E) == (8, 4):
+        L = inputs.make_layer(inputs.CONFIGS["tiny_f32"], seed=0)["logits"]
+    else:
+        L = inputs.random_logits(T, E, T + E + flags, 2.0)
+    g = _check_pair(moe, T, E, k, C, L, flags=flags)
+    ro = oracle.route(L, k, oracle.capacity(T, E, k, C), flags)
+    assert np.array_equal(g["slot"], ro["slot"])
+    assert np.array_equal(g["w"].view(np.uint32), ro["w"].view(np.uint32))
+    if (T, E) == (8, 4):
+        assert g["drop"][:, 0].tolist() == [0, 0, 0, 0, 1, 0, 0, 0]
