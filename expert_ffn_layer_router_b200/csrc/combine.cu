@@ -351,8 +351,10 @@ __global__ void __launch_bounds__(256) ffn_f32_kernel(
 // fp32 router logits on CUDA cores: L[t, e] = sum_i x[t, i] Wr[i, e] + br[e], i ascending.
 __global__ void logits_f32_kernel(const float* __restrict__ x, const float* __restrict__ Wr,
                                   const float* __restrict__ br, int T, int d, int E,
-                                  float* __restrict__ L) {
+                                  float* __restrict__ L, int32_t* __restrict__ zero, int zero_n) {
     pdl_begin();
+    if (zero && blockIdx.x == 0)
+        for (int i = threadIdx.x; i < zero_n; i += blockDim.x) zero[i] = 0;
     const long long n = (long long)T * E;
     for (long long q = blockIdx.x * (long long)blockDim.x + threadIdx.x; q < n;
          q += (long long)gridDim.x * blockDim.x) {
@@ -366,11 +368,12 @@ __global__ void logits_f32_kernel(const float* __restrict__ x, const float* __re
 }  // namespace
 
 void launch_logits_f32(const float* x, const float* Wr, const float* br, int T, int d, int E,
-                       float* logits, cudaStream_t s, int* launches) {
+                       float* logits, int32_t* zero, int zero_n, cudaStream_t s, int* launches) {
     const long long n = (long long)T * E;
     if (n == 0) return;
     const int blocks = (int)std::min<long long>((n + 255) / 256, 148 * 8);
-    launch_pdl(logits_f32_kernel, dim3(blocks), dim3(256), 0, s, x, Wr, br, T, d, E, logits);
+    launch_pdl(logits_f32_kernel, dim3(blocks), dim3(256), 0, s, x, Wr, br, T, d, E, logits, zero,
+               zero_n);
     *launches += 1;
 }
 

@@ -8,8 +8,9 @@
 //          into the A-operand load (the fused-MoE dataflow diagram's "GEMM 1 reads row p //
 //          top_k" idea, here indexed by expert-sorted row rather than pair order);
 //   GEMM2: Y[r, :] = H[r] . W2[e]^T + b2[e].
-// Router logits: L = x . [Wr_hi | Wr_mid | Wr_lo] with Wr split exactly into three bf16 terms;
-// the epilogue adds the three fp32 partial products and the router bias.
+// Router logits: L = x . (Wr_hi + Wr_mid) with the fp32 Wr split into two bf16 terms (hi =
+// bf16(Wr), mid = bf16(Wr - hi); the rest is below 2^-18 |Wr|) by router_split_kernel; the
+// epilogue adds the two fp32 partial products and the router bias.
 //
 // One persistent CTA per SM (or CTA pair per two SMs) walks a static list of (expert, m-tile,
 // BN-column n-tile) tiles, n-tile fastest.  Warp roles (448 threads):
@@ -28,7 +29,6 @@
 
 #include <cstdint>
 #include <cstdio>
-#include <cstdlib>
 #include <atomic>
 #include <mutex>
 
@@ -47,11 +47,10 @@ constexpr int kEpiWarps = 8;        // two per TMEM lane quadrant, each half of 
 constexpr int kTmemCols = 512;      // two accumulators at column 0 and 256
 constexpr int kMaxGroups = 1024;
 
-// kEpiRouterFused: the router epilogue also forms the softmax, the top-k and the per-chunk
-// expert counts of its tokens (all E <= 64 experts of a token sit in one thread's TMEM lane).
+// kEpiRouter: fp32 logits hi + mid (+ bias), staged in shared memory and written row by row.
 // kEpiSwiGLU: gated experts; the tile's 256 B rows are 128 gate rows and the matching 128 up
 // rows, and the epilogue writes SiLU(gate) * up for 128 hidden features.
-enum Epi { kEpiSiLU = 0, kEpiBias = 1, kEpiRouter = 2, kEpiRouterFused = 3, kEpiSwiGLU = 4 };
+enum Epi { kEpiSiLU = 0, kEpiBias = 1, kEpiRouter = 2, kEpiSwiGLU = 4 };
 
 struct GemmArgs {
     const __nv_bfloat16* A;   // [*, lda] row-major
@@ -70,27 +69,28 @@ struct GemmArgs {
     void* D;                  // output
     long long ldd;            // elements
     int router_E;             // router epilogue: number of experts (columns of D)
-    int32_t* r_ids;           // fused router: [T*k] expert ids
-    float* r_w;               // fused router: [T*k] softmax weights
-    int32_t* r_cnt;           // fused router: [E][r_nC] pairs per expert and 32-token chunk
-    int r_nC;
-    int r_k;
-    unsigned r_flags;
     DeviceStatus* st;
 };
 
 // PAIR: two CTAs of a cluster share one 256-row tile; each holds its 128 A rows and half of the
 // BN B rows in shared memory, the pair's tensor cores compute the 256 x BN product together.
-template <int BN, bool PAIR>
+// The router epilogue (BN = 2 Eg: hi and mid columns of Eg experts) stages the tile's logits in a
+// padded [128][Eg + 1] fp32 array instead of the bf16 staging buffers.
+template <int BN, bool PAIR, int EPI>
 struct Cfg {
+    static constexpr bool kRouter = EPI == kEpiRouter;
+    static constexpr int kEg = BN / 2;
+    static constexpr int kLStride = kEg + 1;                      // floats per staged logits row
     static constexpr int kTileM = PAIR ? 256 : 128;
     static constexpr int kBRows = PAIR ? BN / 2 : BN;          // B rows held by this CTA
     static constexpr int kABytes = kBM * kBK * 2;                // 16 KB
     static constexpr int kBBytes = kBRows * kBK * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kStages = (200 * 1024) / kStageBytes > 8 ? 8 : (200 * 1024) / kStageBytes;
-    static constexpr int kStgOff = kStages * kStageBytes;        // epilogue staging, 2 KB a warp
-    static constexpr int kStgBytes = kEpiWarps * 2048;
+    static constexpr int kStageBudget = (kRouter ? 168 : 200) * 1024;
+    static constexpr int kStages = kStageBudget / kStageBytes > 8 ? 8 : kStageBudget / kStageBytes;
+    static constexpr int kStgOff = kStages * kStageBytes;        // epilogue staging
+    static constexpr int kStgBytes =
+        kRouter ? kBM * kLStride * 4 : kEpiWarps * 2048;
     static constexpr int kBarOff = kStgOff + kStgBytes;
     static constexpr int kTableOff = kBarOff + 512;
     static constexpr int kSmemBytes = 1024 + kTableOff + (kMaxGroups + 1) * 4;
@@ -99,6 +99,7 @@ struct Cfg {
     static_assert(kBBytes % 1024 == 0, "B stage must stay 1024-byte aligned");
     static_assert(8 * (3 * kStages + 4) + 4 <= 512, "barrier area");
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+    static_assert(kStgBytes % 8 == 0, "barriers stay 8-byte aligned");
 };
 
 __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c,
@@ -267,13 +268,39 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, const int* s_mt, int E
     return c;
 }
 
+// Writers of the router GEMM's logits: the 8 epilogue warps (index 0-7) and warps 10-13 (index
+// 8-11).  Per tile: barrier 1 (the staged logits are complete), then warp r writes rows r, r + 12,
+// ... (coalesced along the experts); barrier 2 (the staging array may be refilled).  Every writer
+// warp meets both barriers for every tile; wr = -1 only meets them (an epilogue warp whose
+// pipeline wait failed).
+constexpr int kRouteWarps = kEpiWarps + 4;
+
+__device__ __forceinline__ void named_bar(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ void router_tile(const float* sL, int LS, int Eg, const TileCoord& tc,
+                                            const GemmArgs& a, int wr) {
+    const int lane = threadIdx.x & 31;
+    named_bar(1, kRouteWarps * 32);
+    if (wr >= 0) {
+        const int e0 = tc.nt * Eg;                         // first expert of this column tile
+        const int ne = min(Eg, a.router_E - e0);
+        for (int r = wr; r < tc.rows; r += kRouteWarps) {
+            float* out = reinterpret_cast<float*>(a.D) + ((long long)tc.row0 + r) * a.ldd + e0;
+            for (int e = lane; e < ne; e += 32) out[e] = sL[r * LS + e];
+        }
+    }
+    named_bar(2, kRouteWarps * 32);
+}
+
 template <int BN, int EPI, bool GATHER, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmD, const GemmArgs args) {
     pdl_begin();
-    using C = Cfg<BN, PAIR>;
+    using C = Cfg<BN, PAIR, EPI>;
     constexpr int S = C::kStages;
     constexpr int TM = C::kTileM;
     extern __shared__ uint8_t smem_raw[];
@@ -285,13 +312,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
     auto tfull_bar = [&](int b) { return bar0 + 8u * (3 * S + b); };
     auto tempty_bar = [&](int b) { return bar0 + 8u * (3 * S + 2 + b); };
-    // Gathered A on pairs: the peer CTA's copies complete on its own barrier first.
-    auto pfull_bar = [&](int s) { return bar0 + 8u * (2 * S + s); };
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base_ptr + C::kBarOff + 8 * (3 * S + 4));
     int* s_mt = reinterpret_cast<int*>(base_ptr + C::kTableOff);
     auto sA = [&](int s) { return base + (uint32_t)s * C::kABytes; };
     auto sB = [&](int s) { return base + (uint32_t)S * C::kABytes + (uint32_t)s * C::kBBytes; };
 
+    // Gathered rows run on single-CTA tiles: the pipeline is limited by the rows in flight, not
+    // by the weight traffic that pairs would halve (measured on B200: pairs with a relay of the
+    // peer's gathered stages were 4% slower).
+    static_assert(!(GATHER && PAIR), "gathered A uses single-CTA tiles");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = args.E;
     DeviceStatus* st = args.st;
@@ -302,11 +331,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < S; ++s) {
-            // producer arrive + expected bytes; gathered rows add one arrival per A thread of
-            // this CTA, and for a pair one relayed arrival for all of the peer's rows
-            mbar_init(full_bar(s), GATHER ? 1 + 128 + (PAIR ? 1 : 0) : 1);
+            // producer arrive + expected bytes; gathered rows add one arrival per A thread
+            mbar_init(full_bar(s), GATHER ? 1 + 128 : 1);
             mbar_init(empty_bar(s), 1);
-            if (GATHER && PAIR) mbar_init(pfull_bar(s), 128);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar(b), 1);
@@ -377,10 +404,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nkb = args.K / kBK;
     constexpr uint32_t kIdesc = idesc_bf16(TM, BN);
     // A last column tile with at most BN/2 valid columns (d_ff = 1408 on 256-wide tiles) runs
-    // N = BN/2 MMAs: the padded half is neither multiplied nor read back.  (Not on pairs, whose
-    // CTAs each hold one half of the tile's B rows.)
-    constexpr bool kHalfOk =
-        (EPI == kEpiSiLU || EPI == kEpiBias) && !PAIR && (BN / 2) % 16 == 0;
+    // N = BN/2 MMAs: the padded half is neither multiplied nor read back.  On pairs each CTA then
+    // supplies BN/4 of the tile's weight rows (the first BN/4 rows of its B stage).
+    constexpr bool kHalfOk = (EPI == kEpiSiLU || EPI == kEpiBias) && (BN / 2) % 16 == 0;
     constexpr uint32_t kIdescHalf = idesc_bf16(TM, kHalfOk ? BN / 2 : BN);
     const bool last_half = kHalfOk && (n_tiles * BN - args.Nout) >= BN / 2;
     // Barriers of the pair's leader that both CTAs signal.
@@ -395,7 +421,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int tile = cid; ok && tile < total; tile += ncl) {
                 const TileCoord tc = tile_coord<TM>(tile, s_mt, E, n_tiles, args, (int)crank);
-                const int brow = tc.e * args.b_rows_per_group + tc.nt * BN + (int)crank * C::kBRows;
+                const bool half = last_half && tc.nt == n_tiles - 1;
+                const int brow = tc.e * args.b_rows_per_group + tc.nt * BN +
+                                 (int)crank * (half ? BN / 4 : C::kBRows);
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1u;
@@ -461,20 +489,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 if (PAIR) tc_commit_pair(tfull_bar(b)); else tc_commit(tfull_bar(b));
             }
-        } else if (GATHER && PAIR && lane == 0) {
-            // Relay of the peer CTA: once all of its gathered rows of a stage have landed, make
-            // them visible to the tensor cores and count them on the leader's full barrier.
-            uint32_t it = 0;
-            bool ok = true;
-            for (int tile = cid; ok && tile < total; tile += ncl) {
-                for (int kb = 0; kb < nkb; ++kb, ++it) {
-                    const int s = it % S;
-                    const uint32_t ph = (it / S) & 1u;
-                    if (!mbar_wait<false>(pfull_bar(s), ph, st, 6)) { ok = false; break; }
-                    fence_proxy_async_smem();
-                    mbar_arrive_cluster(lead(full_bar(s)));
-                }
-            }
         }
     } else if (warp < 2 + kEpiWarps) {
         // ---------------- epilogue (this CTA's 128 rows) ----------------
@@ -491,120 +505,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int tile = cid; tile < total; tile += ncl, ++lt) {
             const TileCoord tc = tile_coord<TM>(tile, s_mt, E, n_tiles, args, (int)crank);
             const uint32_t b = lt & 1u, use = lt >> 1;
-            if (!mbar_wait<PAIR>(tfull_bar(b), use & 1u, st, 4)) break;
+            if (!mbar_wait<PAIR>(tfull_bar(b), use & 1u, st, 4)) {
+                // The router's routing warps meet two barriers per tile: keep meeting them.
+                if (EPI == kEpiRouter) {
+                    router_tile(nullptr, 0, 0, tc, args, -1);
+                    continue;
+                }
+                break;
+            }
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + b * 256u;
             const int wrows = min(32, max(0, tc.rows - q * 32));      // valid rows of the warp
             const long long wrow0 = (long long)tc.row0 + q * 32;
             if (EPI == kEpiRouter) {
-                constexpr int Eg = BN / 3;
-                if (h == 0) {
+                // Logits of this warp's 32 rows, hi + mid (+ bias), into the staging array; a
+                // warp pair splits the tile's experts.  Then the TMEM buffer is released and the
+                // writer warps store the tile (router_tile).
+                constexpr int Eg = C::kEg, LS = C::kLStride;
+                constexpr int kCols = Eg >= 32 ? Eg / 2 : Eg;
+                float* sL = reinterpret_cast<float*>(base_ptr + C::kStgOff);
+                if (Eg >= 32 || h == 0) {
 #pragma unroll 1
-                    for (int c0 = 0; c0 < Eg; c0 += 16) {
-                        float hi[16], mi[16], lo[16];
+                    for (int c0 = h * kCols; c0 < (h + 1) * kCols; c0 += 16) {
+                        float hi[16], mi[16];
                         __syncwarp();
                         tmem_ld16_wait(taddr + c0, hi);
                         tmem_ld16_wait(taddr + Eg + c0, mi);
-                        tmem_ld16_wait(taddr + 2 * Eg + c0, lo);
-                        const int e0 = tc.nt * Eg + c0;
-                        if (lane < wrows) {
-                            float* out = reinterpret_cast<float*>(args.D) + (wrow0 + lane) * args.ldd;
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                const int e = e0 + i;
-                                if (e < args.router_E) {
-                                    float v = __fadd_rn(hi[i], __fadd_rn(mi[i], lo[i]));
-                                    if (args.bias) v = __fadd_rn(v, __ldg(args.bias + e));
-                                    out[e] = v;
-                                }
-                            }
-                        }
-                    }
-                }
-            } else if (EPI == kEpiRouterFused) {
-                // One thread = one token: logits of all E experts from TMEM, then the softmax in
-                // the warp router's order (lane partials of experts l, l+32, then the pairwise
-                // tree 16, 8, 4, 2, 1), the top-k by (logit desc, expert asc) and this warp's
-                // 32-token chunk histogram.
-                constexpr int Eg = BN / 3;
-                if (h == 0) {
-                    const int Er = args.router_E;
-                    int* s_cnt = reinterpret_cast<int*>(base_ptr + C::kStgOff) + (warp - 2) * 512;
-                    for (int e = lane; e < Er; e += 32) s_cnt[e] = 0;
-                    float L[Eg];
-#pragma unroll
-                    for (int c0 = 0; c0 < Eg; c0 += 16) {
-                        float hi[16], mi[16], lo[16];
-                        __syncwarp();
-                        tmem_ld16_wait(taddr + c0, hi);
-                        tmem_ld16_wait(taddr + Eg + c0, mi);
-                        tmem_ld16_wait(taddr + 2 * Eg + c0, lo);
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
-                            float v = __fadd_rn(hi[i], __fadd_rn(mi[i], lo[i]));
-                            if (args.bias && c0 + i < Er) v = __fadd_rn(v, __ldg(args.bias + c0 + i));
-                            L[c0 + i] = v;
+                            const int e = tc.nt * Eg + c0 + i;
+                            float v = __fadd_rn(hi[i], mi[i]);
+                            if (args.bias && e < args.router_E) v = __fadd_rn(v, __ldg(args.bias + e));
+                            sL[(q * 32 + lane) * LS + c0 + i] = v;
                         }
                     }
-                    __syncwarp();
-                    if (lane < wrows) {
-                        const long long t = wrow0 + lane;
-                        if (args.D) {
-                            float* out = reinterpret_cast<float*>(args.D) + t * args.ldd;
-#pragma unroll
-                            for (int e = 0; e < Eg; ++e)
-                                if (e < Er) out[e] = L[e];
-                        }
-                        float m = L[0];
-#pragma unroll
-                        for (int e = 1; e < Eg; ++e)
-                            if (e < Er && L[e] > m) m = L[e];
-                        float part[32];
-#pragma unroll
-                        for (int l = 0; l < 32; ++l) {
-                            float acc = 0.0f;
-#pragma unroll
-                            for (int e = l; e < Eg; e += 32)
-                                if (e < Er) acc = __fadd_rn(acc, exp_cody_waite(__fsub_rn(L[e], m)));
-                            part[l] = acc;
-                        }
-#pragma unroll
-                        for (int hh = 16; hh >= 1; hh >>= 1)
-#pragma unroll
-                            for (int l = 0; l < hh; ++l) part[l] = __fadd_rn(part[l], part[l + hh]);
-                        const float S = part[0];
-                        uint64_t taken = 0;
-                        float wsum = 0.0f;
-                        for (int j = 0; j < args.r_k; ++j) {
-                            int best = -1;
-                            float bl = 0.0f;
-#pragma unroll
-                            for (int e = 0; e < Eg; ++e) {
-                                if (e < Er && !((taken >> e) & 1ull) && (best < 0 || L[e] > bl)) {
-                                    best = e;
-                                    bl = L[e];
-                                }
-                            }
-                            taken |= 1ull << best;
-                            const size_t pj = (size_t)t * args.r_k + j;
-                            const float wj = __fdiv_rn(exp_cody_waite(__fsub_rn(bl, m)), S);
-                            args.r_ids[pj] = best;
-                            args.r_w[pj] = wj;
-                            wsum = __fadd_rn(wsum, wj);
-                            atomicAdd(&s_cnt[best], 1);
-                        }
-                        if (args.r_flags & MOE_FLAG_RENORMALIZE)
-                            for (int j = 0; j < args.r_k; ++j) {
-                                const size_t pj = (size_t)t * args.r_k + j;
-                                args.r_w[pj] = __fdiv_rn(args.r_w[pj], wsum);
-                            }
-                    }
-                    __syncwarp();
-                    const int chunk = (int)(wrow0 >> 5);
-                    if (chunk < args.r_nC)
-                        for (int e = lane; e < Er; e += 32)
-                            args.r_cnt[(size_t)e * args.r_nC + chunk] = s_cnt[e];
                 }
+                __syncwarp();
+                tc_fence_before();
+                mbar_arrive(tempty_bar(b));
+                router_tile(sL, LS, Eg, tc, args, warp - 2);
+                continue;
             } else {
                 // Output columns of this tile: BN (128 hidden features for gated experts).
                 constexpr int kOut = EPI == kEpiSwiGLU ? 128 : BN;
@@ -705,9 +645,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // stage's full barrier when they have landed (cp.async.mbarrier.arrive.noinc), so all
         // stages can be in flight at once and no producer thread ever blocks on its own copies.
         // The MMA thread makes the landed rows visible to the tensor cores with a proxy fence.
-        // The peer CTA of a pair cannot arrive asynchronously on the leader's barrier: its
-        // copies arrive on its own pfull barrier, and its relay thread forwards the stage.
-        const bool remote = PAIR && !leader;
         const int at = threadIdx.x - 32 * (2 + kEpiWarps);   // 0..127
         const int chunk = at & 7;                             // 16-byte chunk of the row
         const int rbase = at >> 3;                            // rows rbase + 16 i
@@ -751,7 +688,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
                     if (valid[i]) cp_async_16(dA + dst_off[i], src[i] + kb * kBK);
-                cp_async_arrive_noinc(remote ? pfull_bar(s) : full_bar(s));
+                cp_async_arrive_noinc(full_bar(s));
                 if (kb == 0 && next < total) {
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
@@ -764,6 +701,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         cp_async_commit();     // no copy of this thread may still be in flight at exit
         cp_async_wait<0>();
+    } else if (EPI == kEpiRouter) {
+        // ---------------- router: warps 10-13 help write each tile's logits ----------------
+        float* sL = reinterpret_cast<float*>(base_ptr + C::kStgOff);
+        for (int tile = cid; tile < total; tile += ncl) {
+            const TileCoord tc = tile_coord<TM>(tile, s_mt, E, n_tiles, args, 0);
+            router_tile(sL, C::kLStride, C::kEg, tc, args, warp - 2);
+        }
     }
 
     if (warp >= 2 && warp < 2 + kEpiWarps && lane == 0) bulk_wait_all();
@@ -778,28 +722,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// Wr [d, E] fp32 -> B rows for the router GEMM: for column tile nt, rows
-// nt*3Eg + {0, Eg, 2Eg} + c hold the hi/mid/lo bf16 terms of Wr[:, nt*Eg + c] (zero past E).
-__global__ void router_split_kernel(const float* __restrict__ Wr, int d, int E, int Eg, int ntl,
-                                    __nv_bfloat16* __restrict__ B) {
+// Wr [d, E] fp32 -> B [ntl * 2Eg, d] bf16, the router GEMM's weight rows; also clears zero[0,
+// zero_n).  For column tile nt, row
+// nt*2Eg + c holds hi = bf16(Wr[:, nt*Eg + c]) and row nt*2Eg + Eg + c holds mid = bf16(Wr - hi)
+// (Wr - hi is exact in fp32); experts past E are zero.  One block per 16 x Eg piece of Wr: every
+// thread issues its (at most 4) coalesced loads before using any, the piece is transposed through
+// shared memory, and each of the first 2 Eg threads writes 16 consecutive k of one hi or mid row.
+constexpr int kSplitK = 16;
+
+template <int Eg>
+__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ Wr, int d,
+                                                           int E, __nv_bfloat16* __restrict__ B,
+                                                           int32_t* __restrict__ zero,
+                                                           int zero_n) {
     pdl_begin();
-    const long long total = (long long)ntl * 3 * Eg * d;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-         i += (long long)gridDim.x * blockDim.x) {
-        const int col = (int)(i % d);
-        const int row = (int)(i / d);
-        const int nt = row / (3 * Eg), part = (row / Eg) % 3, c = row % Eg;
-        const int e = nt * Eg + c;
-        float v = 0.0f;
-        if (e < E) {
-            const float w = Wr[(size_t)col * E + e];
-            const float hi = __bfloat162float(__float2bfloat16_rn(w));
-            const float r1 = __fsub_rn(w, hi);
-            const float mid = __bfloat162float(__float2bfloat16_rn(r1));
-            const float r2 = __fsub_rn(r1, mid);
-            v = part == 0 ? hi : (part == 1 ? mid : r2);
+    // The dispatch counters of this call start at zero (the routing kernel after the logits GEMM
+    // adds to them).
+    if (zero && blockIdx.x == 0 && blockIdx.y == 0)
+        for (int i = threadIdx.x; i < zero_n; i += blockDim.x) zero[i] = 0;
+    constexpr int kPer = (kSplitK * Eg + 255) / 256;
+    __shared__ float s_w[kSplitK][Eg + 1];
+    const int k0 = blockIdx.x * kSplitK, nt = blockIdx.y;
+    float v[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        const int i = threadIdx.x + 256 * j, kk = i / Eg, c = i % Eg, e = nt * Eg + c;
+        v[j] = (i < kSplitK * Eg && e < E) ? __ldg(Wr + (size_t)(k0 + kk) * E + e) : 0.0f;
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        const int i = threadIdx.x + 256 * j;
+        if (i < kSplitK * Eg) s_w[i / Eg][i % Eg] = v[j];
+    }
+    __syncthreads();
+    if (threadIdx.x < 2 * Eg) {
+        const int c = threadIdx.x % Eg, t = threadIdx.x / Eg;
+        uint32_t pk[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float a = s_w[2 * q][c], b = s_w[2 * q + 1][c];
+            const uint32_t h = pack_bf16x2(a, b);
+            pk[q] = t == 0 ? h
+                           : pack_bf16x2(__fsub_rn(a, __uint_as_float(h << 16)),
+                                         __fsub_rn(b, __uint_as_float(h & 0xffff0000u)));
         }
-        B[i] = __float2bfloat16_rn(v);
+        uint4* dst =
+            reinterpret_cast<uint4*>(B + ((size_t)nt * 2 * Eg + t * Eg + c) * d + k0);
+        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
     }
 }
 
@@ -862,7 +832,7 @@ int num_sms() {
 template <int BN, int EPI, bool GATHER, bool PAIR>
 cudaError_t launch_gemm_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,
                           const GemmArgs& a, long long tiles, cudaStream_t s) {
-    using C = Cfg<BN, PAIR>;
+    using C = Cfg<BN, PAIR, EPI>;
     auto kern = grouped_gemm_kernel<BN, EPI, GATHER, PAIR>;
     static std::atomic<uint64_t> attr_done{0};
     static std::atomic<int> pair_slots[64];
@@ -934,17 +904,16 @@ template <int EPI>
 cudaError_t launch_router_bn(int BN, const CUtensorMap& tmA, const CUtensorMap& tmB,
                              const GemmArgs& a, long long tiles, cudaStream_t s) {
     switch (BN) {
-        case 192: return launch_gemm_t<192, EPI, false, false>(tmA, tmB, tmB, a, tiles, s);
-        case 96: return launch_gemm_t<96, EPI, false, false>(tmA, tmB, tmB, a, tiles, s);
-        case 48: return launch_gemm_t<48, EPI, false, false>(tmA, tmB, tmB, a, tiles, s);
+        case 128: return launch_gemm_t<128, EPI, false, false>(tmA, tmB, tmB, a, tiles, s);
+        case 64: return launch_gemm_t<64, EPI, false, false>(tmA, tmB, tmB, a, tiles, s);
+        case 32: return launch_gemm_t<32, EPI, false, false>(tmA, tmB, tmB, a, tiles, s);
         default: return cudaErrorInvalidValue;
     }
 }
 
 }  // namespace
 
-// Column tile for an output width.  MOE_GEMM_BN in the environment (256, 192, 176 or 128)
-// overrides the choice, for tuning runs.
+// Column tile for an output width.
 //  - Groups of many rows (compute-bound): a column tile costs BN + 128, for the per-tile work
 //    that does not shrink with BN (A operand loads, pipeline turn-around), about half a 256-wide
 //    tile's MMA time.  Measured on B200 at d_ff = 1408: 256-wide tiles (with a half-width last
@@ -954,13 +923,6 @@ cudaError_t launch_router_bn(int BN, const CUtensorMap& tmA, const CUtensorMap& 
 //    the cost is ceil(tiles / SMs) x (BN + 32).  Measured on B200 at T = 64, E = 64, k = 8:
 //    d_model = 2048 outputs on 128-wide tiles (6.9 waves) beat 256-wide ones (3.5) by 13%.
 int pick_bn(int nout, long long max_rows, int E, int num_sm) {
-    static int forced = -1;
-    if (forced < 0) {
-        const char* v = getenv("MOE_GEMM_BN");
-        const int f = v ? atoi(v) : 0;
-        forced = (f == 256 || f == 192 || f == 176 || f == 128) ? f : 0;
-    }
-    if (forced > 0) return forced;
     const bool streaming = max_rows <= 64LL * E;
     const long long m_tiles = streaming ? E : (max_rows + 127) / 128 + E;
     // Ties go to the wider tile when compute-bound, to the narrower one (finer waves) when
@@ -982,8 +944,6 @@ int pick_bn(int nout, long long max_rows, int E, int num_sm) {
 
 int router_group(int E) { return E <= 16 ? 16 : (E <= 32 ? 32 : 64); }
 
-// Pair (2-SM) tiles when the experts' rows fill 256-row tiles well enough; 1-SM otherwise.
-int g_pair_mode = -1;      // -1 automatic, 0 never, 1 always (MOE_GEMM_PAIR in the environment)
 
 // Gated experts' first GEMM: W is [E, 2F, K] (gate rows then up rows), bias [E, 2F]; D = H [rows,
 // F] = SiLU(A W_gate^T + b_gate) * (A W_up^T + b_up).  256-wide tiles = 128 gate + 128 up rows.
@@ -993,15 +953,11 @@ cudaError_t launch_gated_gemm(const void* A, long long lda, const int32_t* a_row
                               long long max_rows, DeviceStatus* st, cudaStream_t s,
                               int* launches);
 
-bool use_pair(long long max_rows, int E) {
-    if (g_pair_mode < 0) {
-        const char* v = getenv("MOE_GEMM_PAIR");
-        g_pair_mode = v ? (v[0] == '1' ? 1 : (v[0] == '0' ? 0 : 2)) : 2;
-    }
-    if (g_pair_mode == 0) return false;
-    if (g_pair_mode == 1) return true;
-    return max_rows >= 256LL * E;
-}
+// Pair (2-SM, M = 256) tiles when the experts' rows fill 256-row tiles well enough; 1-SM
+// otherwise.  A 128 x 256 single-CTA tile moves about 96 KB through shared memory per 512 tensor
+// cycles (its operand fills plus the MMA's operand reads), above what shared memory delivers; a
+// pair's 256 x 256 tile holds half of the weight rows in each CTA and needs about 64 KB per SM.
+bool use_pair(long long max_rows, int E) { return max_rows >= 256LL * E; }
 
 cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const int32_t* a_rows,
                                int a_row_limit, const int32_t* offsets, int E, int K, int Nout,
@@ -1013,9 +969,7 @@ cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const in
                                  ldd, max_rows, st, s, launches);
     }
     const int BN = pick_bn(Nout, max_rows, E, num_sms());
-    // Gathered A on pairs needs the peer's rows forwarded to the leader's barrier by the copying
-    // threads themselves, which measured slower than single-CTA tiles; only when forced.
-    const bool pair = use_pair(max_rows, E) && (a_rows == nullptr || g_pair_mode == 1);
+    const bool pair = use_pair(max_rows, E) && a_rows == nullptr;
     CUtensorMap tm;
     if (!make_tmap(&tm, W, (long long)E * Nout, K, pair ? BN / 2 : BN)) return cudaErrorInvalidValue;
     GemmArgs a{};
@@ -1046,10 +1000,7 @@ cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const in
     CUtensorMap tmD;
     if (!make_tmap_out(&tmD, D, max_rows, Nout, ldd)) return cudaErrorInvalidValue;
     cudaError_t e;
-    if (gather && pair) {
-        e = which == 0 ? launch_gemm_bn<kEpiSiLU, true, true>(BN, tmA, tm, tmD, a, max_tiles, s)
-                       : launch_gemm_bn<kEpiBias, true, true>(BN, tmA, tm, tmD, a, max_tiles, s);
-    } else if (gather) {
+    if (gather) {
         e = which == 0 ? launch_gemm_bn<kEpiSiLU, true, false>(BN, tmA, tm, tmD, a, max_tiles, s)
                        : launch_gemm_bn<kEpiBias, true, false>(BN, tmA, tm, tmD, a, max_tiles, s);
     } else if (pair) {
@@ -1069,7 +1020,7 @@ cudaError_t launch_gated_gemm(const void* A, long long lda, const int32_t* a_row
                               long long max_rows, DeviceStatus* st, cudaStream_t s,
                               int* launches) {
     if (F % 128 != 0) return cudaErrorInvalidValue;
-    const bool pair = use_pair(max_rows, E) && (a_rows == nullptr || g_pair_mode == 1);
+    const bool pair = use_pair(max_rows, E) && a_rows == nullptr;
     CUtensorMap tm;
     if (!make_tmap(&tm, W, (long long)E * 2 * F, K, 128)) return cudaErrorInvalidValue;
     GemmArgs a{};
@@ -1097,9 +1048,7 @@ cudaError_t launch_gated_gemm(const void* A, long long lda, const int32_t* a_row
     CUtensorMap tmD;
     if (!make_tmap_out(&tmD, D, max_rows, F, ldd)) return cudaErrorInvalidValue;
     cudaError_t e;
-    if (gather && pair)
-        e = launch_gemm_t<256, kEpiSwiGLU, true, true>(tmA, tm, tmD, a, max_tiles, s);
-    else if (gather)
+    if (gather)
         e = launch_gemm_t<256, kEpiSwiGLU, true, false>(tmA, tm, tmD, a, max_tiles, s);
     else if (pair)
         e = launch_gemm_t<256, kEpiSwiGLU, false, true>(tmA, tm, tmD, a, max_tiles, s);
@@ -1112,18 +1061,23 @@ cudaError_t launch_gated_gemm(const void* A, long long lda, const int32_t* a_row
 size_t router_split_bytes(int d, int E) {
     const int Eg = router_group(E);
     const int ntl = (E + Eg - 1) / Eg;
-    return (size_t)ntl * 3 * Eg * d * 2;
+    return (size_t)ntl * 2 * Eg * d * 2;
 }
 
 cudaError_t launch_router_gemm(const void* x, int T, int d, const float* Wr, const float* br,
-                               int E, void* split_buf, float* logits, DeviceStatus* st,
-                               cudaStream_t s, int* launches, const RouterFused* fused) {
+                               int E, void* split_buf, float* logits, int32_t* zero, int zero_n,
+                               DeviceStatus* st, cudaStream_t s, int* launches) {
     const int Eg = router_group(E);
     const int ntl = (E + Eg - 1) / Eg;
-    const int BN = 3 * Eg;
-    const bool fuse = fused != nullptr && ntl == 1;
-    launch_pdl(router_split_kernel, dim3(148 * 4), dim3(256), 0, s, Wr, d, E, Eg, ntl,
-               reinterpret_cast<__nv_bfloat16*>(split_buf));
+    const int BN = 2 * Eg;
+    const dim3 sg(d / kSplitK, ntl);
+    __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(split_buf);
+    if (Eg == 16)
+        launch_pdl(router_split_kernel<16>, sg, dim3(256), 0, s, Wr, d, E, sb, zero, zero_n);
+    else if (Eg == 32)
+        launch_pdl(router_split_kernel<32>, sg, dim3(256), 0, s, Wr, d, E, sb, zero, zero_n);
+    else
+        launch_pdl(router_split_kernel<64>, sg, dim3(256), 0, s, Wr, d, E, sb, zero, zero_n);
     *launches += 1;
     CUtensorMap tm;
     if (!make_tmap(&tm, split_buf, (long long)ntl * BN, d, BN)) return cudaErrorInvalidValue;
@@ -1145,23 +1099,13 @@ cudaError_t launch_router_gemm(const void* x, int T, int d, const float* Wr, con
     a.ldd = E;
     a.router_E = E;
     a.st = st;
-    if (fuse) {
-        a.r_ids = fused->ids;
-        a.r_w = fused->w;
-        a.r_cnt = fused->cnt;
-        a.r_nC = fused->nC;
-        a.r_k = fused->k;
-        a.r_flags = fused->flags;
-    }
     const long long tiles = (long long)((T + kBM - 1) / kBM) * ntl;
     CUtensorMap tmA;
     if (!make_tmap(&tmA, x, (long long)T, d, kBM)) return cudaErrorInvalidValue;
-    cudaError_t e = fuse ? launch_router_bn<kEpiRouterFused>(BN, tmA, tm, a, tiles, s)
-                         : launch_router_bn<kEpiRouter>(BN, tmA, tm, a, tiles, s);
+    cudaError_t e = launch_router_bn<kEpiRouter>(BN, tmA, tm, a, tiles, s);
     if (e == cudaSuccess) *launches += 1;
     return e;
 }
 
-bool router_can_fuse(int E) { return E <= 64; }
 
 }  // namespace moe

@@ -14,14 +14,21 @@ struct DeviceStatus;
 // flags: MOE_FLAG_RENORMALIZE divides each token's k weights by their sum.
 void launch_route_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
                        cudaStream_t s, unsigned flags);
-int chunk_count(int T);
-// counts_ready: cnt already holds the per-chunk counts (fused router), skip the count pass.
-// flags: MOE_FLAG_ARRIVAL_ORDER keeps an overflowing expert's first K pairs in token order.
-void launch_capacity_select(const int32_t* ids, const float* w, int T, int E, int k, long long K,
-                            int32_t* cnt, int32_t* base, int32_t* nrecv, int32_t* cand,
-                            int32_t* slot, uint8_t* drop, int32_t* counts, int32_t* offsets,
-                            int32_t* rowtok, DeviceStatus* st, cudaStream_t s, int* launches,
-                            bool counts_ready, unsigned flags);
+// Routing of T tokens from their logits (ids, w) that also appends every pair p = t*k + j to its
+// expert's candidate list cand[e][.] ([E][T]) and counts it in gcnt[e]; gcnt must be zero at
+// entry.  A group of route_group_lanes(E, k) lanes per token when that is not 0, else a warp.
+int route_group_lanes(int E, int k);
+void launch_route_place(const float* logits, int T, int E, int k, unsigned flags, int32_t* ids,
+                        float* w, int32_t* gcnt, int32_t* cand, DeviceStatus* st, cudaStream_t s,
+                        int* launches);
+// Capacity selection from the candidate lists: slot, drop, counts (nullable), offsets and rowtok
+// (nullable).  flags: MOE_FLAG_ARRIVAL_ORDER keeps an overflowing expert's first K pairs in token
+// order.  gbits: select_bits_bytes(T, E) bytes of scratch (unused and nullable when that is 0).
+size_t select_bits_bytes(int T, int E);
+void launch_select(const int32_t* cand, const int32_t* gcnt, const float* w, int T, int E, int k,
+                   long long K, unsigned flags, uint32_t* gbits, int32_t* slot, uint8_t* drop,
+                   int32_t* counts, int32_t* offsets, int32_t* rowtok, DeviceStatus* st,
+                   cudaStream_t s, int* launches);
 // Small batches (T*k <= 1024): the whole capacity selection in one single-block launch.
 bool dispatch_small_fits(int T, int k);
 void launch_dispatch_small(const int32_t* ids, const float* w, int T, int E, int k, long long K,
@@ -53,8 +60,9 @@ void launch_ffn_f32(const float* x, const int32_t* rowtok, const int32_t* offset
                     int d, int F, long long max_rows, const float* W1, const float* b1,
                     const float* W2, const float* b2, float* H, float* Y, DeviceStatus* st,
                     cudaStream_t s, int* launches, bool gated);
+// Also clears zero[0, zero_n) (the dispatch counters).
 void launch_logits_f32(const float* x, const float* Wr, const float* br, int T, int d, int E,
-                       float* logits, cudaStream_t s, int* launches);
+                       float* logits, int32_t* zero, int zero_n, cudaStream_t s, int* launches);
 
 // gemm_tc.cu
 int pick_bn(int nout, long long max_rows, int E, int num_sm);
@@ -68,19 +76,10 @@ cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const in
                                const void* W, const float* bias, void* D, long long ldd,
                                long long max_rows, DeviceStatus* st, cudaStream_t s,
                                int* launches);
-// Outputs of the fused router epilogue (softmax, top-k and per-chunk counts of each token).
-struct RouterFused {
-    int32_t* ids;
-    float* w;
-    int32_t* cnt;     // [E][nC]
-    int nC;
-    int k;
-    unsigned flags;   // MOE_FLAG_RENORMALIZE honoured
-};
-bool router_can_fuse(int E);
-// logits may be null when fused (logits are then not stored).  fused == null: logits only.
+// Router logits L = x Wr + br [T, E] on the tensor cores (Wr split into two bf16 terms in
+// split_buf, router_split_bytes); also clears zero[0, zero_n) (the dispatch counters).
 cudaError_t launch_router_gemm(const void* x, int T, int d, const float* Wr, const float* br,
-                               int E, void* split_buf, float* logits, DeviceStatus* st,
-                               cudaStream_t s, int* launches, const RouterFused* fused);
+                               int E, void* split_buf, float* logits, int32_t* zero, int zero_n,
+                               DeviceStatus* st, cudaStream_t s, int* launches);
 
 }  // namespace moe

@@ -60,7 +60,7 @@ long long max_rows_of(const moe_problem* p, long long K) {
 }
 
 struct Plan {
-    size_t status, logits, ids, w, slot, drop, counts, cnt, base, nrecv, cand, offsets, rowtok,
+    size_t status, gcnt, logits, ids, w, slot, drop, counts, cand, bits, offsets, rowtok,
         kept_tmp, H, Y, split, total;
 };
 
@@ -68,7 +68,6 @@ Plan make_plan(const moe_problem* p) {
     const long long K = capacity_of(p);
     const size_t P = (size_t)p->T * p->k;
     const size_t R = (size_t)max_rows_of(p, K);
-    const size_t nC = (size_t)moe::chunk_count(p->T);
     Plan q{};
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -77,16 +76,15 @@ Plan make_plan(const moe_problem* p) {
         return at;
     };
     q.status = take(sizeof(moe::DeviceStatus));
+    q.gcnt = take((size_t)p->E * 4);
     q.logits = take((size_t)p->T * p->E * 4);
     q.ids = take(P * 4);
     q.w = take(P * 4);
     q.slot = take(P * 4);
     q.drop = take(P);
     q.counts = take((size_t)2 * p->E * 4);
-    q.cnt = take((size_t)p->E * nC * 4);
-    q.base = take((size_t)p->E * nC * 4);
-    q.nrecv = take((size_t)p->E * 4);
     q.cand = take((size_t)p->E * p->T * 4);
+    q.bits = take(moe::select_bits_bytes(p->T, p->E));
     q.offsets = take((size_t)(p->E + 1) * 4);
     q.rowtok = take(R * 4);
     q.kept_tmp = take((size_t)p->E * 4);
@@ -126,22 +124,39 @@ moe_status pre(const moe_problem* p, bool needs_ffn) {
     return MOE_OK;
 }
 
-// Steps 1-2 on device data.  rowtok/offsets may be null (moe_route), counts always written.
+// Scratch of the routing and capacity selection (the workspace's, or the static array's).
+struct RouteScratch {
+    moe::DeviceStatus* st;
+    int32_t* gcnt;      // [E] pairs received per expert, zero at entry of the route kernel
+    int32_t* cand;      // [E][T] candidate lists
+    uint32_t* bits;     // select_bits_bytes(T, E) bytes, or null when that is 0
+};
+
+// Steps 1-2 on device data from given logits.  rowtok/offsets may be null (moe_route); counts is
+// always written.  Small batches: the warp router, then the single-block dispatch.  Otherwise:
+// the dispatch counters are cleared, the router places every pair in its expert's candidate
+// list, and the capacity selection runs per expert.
 void route_steps(const moe_problem* p, const float* logits, int32_t* ids, float* w,
                  int32_t* slot, uint8_t* drop, int32_t* counts, int32_t* offsets,
-                 int32_t* rowtok, void* ws, const Plan& q, cudaStream_t s, int* launches) {
-    moe::DeviceStatus* st = at<moe::DeviceStatus>(ws, q.status);
+                 int32_t* rowtok, const RouteScratch& rs, cudaStream_t s, int* launches) {
     const long long K = capacity_of(p);
-    moe::launch_route_topk(logits, p->T, p->E, p->k, ids, w, s, p->flags);
-    *launches += 1;
-    if (moe::dispatch_small_fits(p->T, p->k))
+    if (moe::dispatch_small_fits(p->T, p->k)) {
+        moe::launch_route_topk(logits, p->T, p->E, p->k, ids, w, s, p->flags);
+        *launches += 1;
         moe::launch_dispatch_small(ids, w, p->T, p->E, p->k, K, p->flags, slot, drop, counts,
-                                   offsets, rowtok, st, s, launches);
-    else
-        moe::launch_capacity_select(ids, w, p->T, p->E, p->k, K, at<int32_t>(ws, q.cnt),
-                                    at<int32_t>(ws, q.base), at<int32_t>(ws, q.nrecv),
-                                    at<int32_t>(ws, q.cand), slot, drop, counts, offsets, rowtok,
-                                    st, s, launches, false, p->flags);
+                                   offsets, rowtok, rs.st, s, launches);
+        return;
+    }
+    cudaMemsetAsync(rs.gcnt, 0, sizeof(int32_t) * p->E, s);
+    moe::launch_route_place(logits, p->T, p->E, p->k, p->flags, ids, w, rs.gcnt, rs.cand, rs.st,
+                            s, launches);
+    moe::launch_select(rs.cand, rs.gcnt, w, p->T, p->E, p->k, K, p->flags, rs.bits, slot, drop,
+                       counts, offsets, rowtok, rs.st, s, launches);
+}
+
+RouteScratch scratch_of(void* ws, const Plan& q) {
+    return RouteScratch{at<moe::DeviceStatus>(ws, q.status), at<int32_t>(ws, q.gcnt),
+                        at<int32_t>(ws, q.cand), q.bits ? at<uint32_t>(ws, q.bits) : nullptr};
 }
 
 moe_status ffn_steps(const moe_problem* p, const void* x, const int32_t* offsets,
@@ -218,18 +233,14 @@ void* current_context() {
 }
 
 // Scratch layout of moe_route inside the static array; returns the bytes it needs.
-size_t route_static_layout(const moe_problem* p, size_t* cnt, size_t* base, size_t* nrecv,
-                           size_t* cand) {
-    const size_t nC = (size_t)moe::chunk_count(p->T);
+size_t route_static_layout(const moe_problem* p, size_t* gcnt, size_t* cand, size_t* bits) {
     size_t off = align_up(sizeof(moe::DeviceStatus));
-    *cnt = off;
-    off = align_up(off + (size_t)p->E * nC * 4);
-    *base = off;
-    off = align_up(off + (size_t)p->E * nC * 4);
-    *nrecv = off;
+    *gcnt = off;
     off = align_up(off + (size_t)p->E * 4);
     *cand = off;
     off = align_up(off + (size_t)p->E * p->T * 4);
+    *bits = off;
+    off = align_up(off + moe::select_bits_bytes(p->T, p->E));
     return off;
 }
 
@@ -292,7 +303,8 @@ moe_status moe_route(const moe_problem* p, const float* logits, int32_t* ids, fl
         cudaMemsetAsync(counts, 0, sizeof(int32_t) * 2 * p->E, s);
         return finish(0);
     }
-    route_steps(p, logits, ids, w, slot, drop, counts, nullptr, nullptr, ws, q, s, &launches);
+    route_steps(p, logits, ids, w, slot, drop, counts, nullptr, nullptr, scratch_of(ws, q), s,
+                &launches);
     return finish(launches);
 }
 
@@ -388,39 +400,48 @@ moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, con
 
     stage_mark(0, s);
     // Small bf16 batches: logits on CUDA cores and routing in one launch (a 128-row tensor-core
-    // tile would leave the GPU idle).  Larger bf16 batches with E <= 64: the logits GEMM's
-    // epilogue also forms the softmax, top-k and per-chunk counts.
+    // tile would leave the GPU idle), then the single-block dispatch.  Larger batches: logits
+    // from the tensor cores (bf16) or CUDA cores (fp32), whose launch also clears the dispatch
+    // counters; then the router that places each pair in its expert's candidate list, and the
+    // per-expert capacity selection.
     const bool small = p->dtype == MOE_BF16 && moe::router_small_fits(p->T, p->E, p->d_model);
-    const bool fused = !small && p->dtype == MOE_BF16 && moe::router_can_fuse(p->E);
+    const bool small_dispatch = moe::dispatch_small_fits(p->T, p->k);
+    int32_t* gcnt = small_dispatch ? nullptr : at<int32_t>(ws, q.gcnt);
+    const int zero_n = small_dispatch ? 0 : p->E;
     if (small) {
-        moe::launch_router_small(x, Wr, br, p->T, p->d_model, p->E, p->k, logits_out, ids, w,
-                                 p->flags, s, &launches);
+        // The large dispatch re-reads the logits: keep them (in the workspace if not asked for).
+        moe::launch_router_small(x, Wr, br, p->T, p->d_model, p->E, p->k,
+                                 small_dispatch ? logits_out : logits, ids, w, p->flags, s,
+                                 &launches);
+        if (!small_dispatch) cudaMemsetAsync(gcnt, 0, sizeof(int32_t) * p->E, s);
     } else if (p->dtype == MOE_BF16) {
-        moe::RouterFused rf{ids, w, at<int32_t>(ws, q.cnt), moe::chunk_count(p->T), p->k,
-                            p->flags};
         if (moe::launch_router_gemm(x, p->T, p->d_model, Wr, br, p->E, at<void>(ws, q.split),
-                                    fused ? logits_out : logits, st, s, &launches,
-                                    fused ? &rf : nullptr) != cudaSuccess)
+                                    logits, gcnt, zero_n, st, s, &launches) != cudaSuccess)
             return MOE_ERR_CUDA;
     } else {
-        moe::launch_logits_f32((const float*)x, Wr, br, p->T, p->d_model, p->E, logits, s,
-                               &launches);
+        moe::launch_logits_f32((const float*)x, Wr, br, p->T, p->d_model, p->E, logits, gcnt,
+                               zero_n, s, &launches);
     }
     stage_mark(1, s);
     const long long K = capacity_of(p);
-    if (!fused && !small) {
-        moe::launch_route_topk(logits, p->T, p->E, p->k, ids, w, s, p->flags);
-        launches += 1;
-    }
-    stage_mark(2, s);
-    if (moe::dispatch_small_fits(p->T, p->k))
+    if (small_dispatch) {
+        if (!small) {
+            moe::launch_route_topk(logits, p->T, p->E, p->k, ids, w, s, p->flags);
+            launches += 1;
+        }
+        stage_mark(2, s);
         moe::launch_dispatch_small(ids, w, p->T, p->E, p->k, K, p->flags, slot, drop, counts,
                                    offsets, rowtok, st, s, &launches);
-    else
-        moe::launch_capacity_select(ids, w, p->T, p->E, p->k, K, at<int32_t>(ws, q.cnt),
-                                    at<int32_t>(ws, q.base), at<int32_t>(ws, q.nrecv),
-                                    at<int32_t>(ws, q.cand), slot, drop, counts, offsets, rowtok,
-                                    st, s, &launches, fused, p->flags);
+    } else {
+        const RouteScratch rs = scratch_of(ws, q);
+        // (After the small router this routes the T <= 1024 tokens a second time, with the
+        // same arithmetic, to place the pairs.)
+        moe::launch_route_place(logits, p->T, p->E, p->k, p->flags, ids, w, gcnt, rs.cand, st,
+                                s, &launches);
+        stage_mark(2, s);
+        moe::launch_select(rs.cand, gcnt, w, p->T, p->E, p->k, K, p->flags, rs.bits, slot, drop,
+                           counts, offsets, rowtok, st, s, &launches);
+    }
     stage_mark(3, s);
     const long long R = max_rows_of(p, K);
     if (R > 0 && p->dtype == MOE_BF16) {
@@ -526,8 +547,8 @@ extern "C" moe_status moe_route_static(const moe_problem* p, const float* logits
     if (r != MOE_OK) return r;
     if (!counts || (p->T > 0 && (!logits || !ids || !w || !slot || !drop)))
         return MOE_ERR_INVALID_ARG;
-    size_t o_cnt, o_base, o_nrecv, o_cand;
-    if (route_static_layout(p, &o_cnt, &o_base, &o_nrecv, &o_cand) > kRouteStaticBytes)
+    size_t o_gcnt, o_cand, o_bits;
+    if (route_static_layout(p, &o_gcnt, &o_cand, &o_bits) > kRouteStaticBytes)
         return MOE_ERR_WORKSPACE;
     cudaError_t err;
     void* scratch = static_scratch_for_current_context(&err);
@@ -537,17 +558,15 @@ extern "C" moe_status moe_route_static(const moe_problem* p, const float* logits
         cudaMemsetAsync(counts, 0, sizeof(int32_t) * 2 * p->E, s);
         return finish(0);
     }
-    // The array keeps the previous call's contents: the status word must start at zero; every
-    // other region is fully written by this call before it is read.
+    // The array keeps the previous call's contents: the status word must start at zero (the
+    // dispatch counters are cleared by route_steps); every other region is fully written by this
+    // call before it is read.
     moe::DeviceStatus* st = at<moe::DeviceStatus>(scratch, 0);
     cudaMemsetAsync(st, 0, sizeof(moe::DeviceStatus), s);
     int launches = 0;
-    moe::launch_route_topk(logits, p->T, p->E, p->k, ids, w, s, p->flags);
-    launches += 1;
-    moe::launch_capacity_select(ids, w, p->T, p->E, p->k, capacity_of(p),
-                                at<int32_t>(scratch, o_cnt), at<int32_t>(scratch, o_base),
-                                at<int32_t>(scratch, o_nrecv), at<int32_t>(scratch, o_cand),
-                                slot, drop, counts, nullptr, nullptr, st, s, &launches, false,
-                                p->flags);
+    const RouteScratch rs{st, at<int32_t>(scratch, o_gcnt), at<int32_t>(scratch, o_cand),
+                          moe::select_bits_bytes(p->T, p->E) ? at<uint32_t>(scratch, o_bits)
+                                                             : nullptr};
+    route_steps(p, logits, ids, w, slot, drop, counts, nullptr, nullptr, rs, s, &launches);
     return finish(launches);
 }

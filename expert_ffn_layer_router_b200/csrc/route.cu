@@ -7,15 +7,18 @@
 // expert keeps at most K pairs, those with the highest router weight (ties: lower token), and
 // the slot of a kept pair is its rank among the expert's kept tokens in ascending token order.
 //
-// Dispatch pipeline, all deterministic (no result depends on the order of atomics):
-//   count  : one warp per chunk of 32 tokens counts its pairs per expert  -> cnt[E][nC]
-//   scan   : one block per expert, exclusive prefix over chunks           -> base[E][nC], n[E]
-//   scatter: one warp per chunk writes its pairs into the expert's candidate list at
-//            base + (rank among equal experts inside the chunk)             -> cand[E][T]
-//            (a stable counting sort: every list is in ascending token order)
+// Dispatch, two launches, deterministic (no result depends on the order of atomics):
+//   route + place: the router (one thread per token for E <= 64 and k <= 8, one warp per token
+//            otherwise) also appends every (token, expert) pair to its expert's candidate list
+//            cand[e][.]; positions come from per-block counters in shared memory plus one global
+//            atomic per (block, expert) on gcnt[e].  The order inside a list is arbitrary.
 //   select : one block per expert; if n_e > K a 4-pass radix select on the fp32 weight bits
-//            finds the K-th largest weight, then one ordered pass with block scans assigns
-//            slots, drop flags, rowtok and the counts.
+//            finds the K-th largest weight (ties at the boundary: lower token first, by a second
+//            radix select on the pair index); the kept tokens are marked in a bitmap over the
+//            batch, whose prefix popcounts give each kept pair its slot (its rank in token
+//            order), so the result does not depend on the list order.
+// gcnt must be zero when the route kernel starts; the kernel before it in the same call clears
+// it (the router GEMM, the fp32 logits kernel, or a memset in moe_route).
 #include <atomic>
 #include <cfloat>
 #include <cstdint>
@@ -30,76 +33,8 @@ namespace {
 constexpr unsigned kFull = 0xffffffffu;
 
 // ---------------------------------------------------------------------------------------------
-// Router: softmax over E + top-k, one warp per token.  Lane l holds experts l, l+32, ...
-// Softmax sum order: lane partials left to right, then xor-butterfly 16, 8, 4, 2, 1.
+// Router: softmax over E + top-k, one warp per token (route_token_warp, softmax.cuh).
 // ---------------------------------------------------------------------------------------------
-// One token's routing by one warp: L points at the token's E logits (global or shared).
-template <int EPL>
-__device__ __forceinline__ void route_token_warp(const float* L, int E, int k, size_t t,
-                                                 int32_t* __restrict__ ids,
-                                                 float* __restrict__ w, unsigned flags) {
-    const int lane = threadIdx.x & 31;
-    float v[EPL];
-    uint32_t key[EPL];
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        v[i] = e < E ? L[e] : 0.0f;
-        key[i] = e < E ? float_key(v[i]) : 0u;
-    }
-    uint32_t lmax = 0;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) lmax = max(lmax, key[i]);
-    const float m = key_float(__reduce_max_sync(kFull, lmax));
-    float u[EPL];
-    float part = 0.0f;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        u[i] = e < E ? exp_cody_waite(__fsub_rn(v[i], m)) : 0.0f;
-        if (e < E) part = __fadd_rn(part, u[i]);
-    }
-#pragma unroll
-    for (int h = 16; h >= 1; h >>= 1) part = __fadd_rn(part, __shfl_xor_sync(kFull, part, h));
-    const float S = part;
-
-    int my_id = 0;
-    float my_w = 0.0f;
-    uint32_t taken = 0;
-    for (int j = 0; j < k; ++j) {
-        uint32_t bk = 0;
-        int bi = 0;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            const bool ok = !((taken >> i) & 1u) && key[i] > bk;
-            bk = ok ? key[i] : bk;
-            bi = ok ? i : bi;
-        }
-        const uint32_t wk = __reduce_max_sync(kFull, bk);
-        const unsigned cand = (bk == wk && bk != 0u) ? (unsigned)(lane + 32 * bi) : 0x7fffffffu;
-        const int we = (int)__reduce_min_sync(kFull, cand);
-        float up = 0.0f;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) up = (i == bi) ? u[i] : up;
-        const float wu = __shfl_sync(kFull, up, we & 31);
-        if (lane == (we & 31)) taken |= 1u << (we >> 5);
-        if (lane == j) {
-            my_id = we;
-            my_w = __fdiv_rn(wu, S);
-        }
-    }
-    if (flags & MOE_FLAG_RENORMALIZE) {
-        // Sum of the k weights in j order, then one division each.
-        float sum = 0.0f;
-        for (int j = 0; j < k; ++j) sum = __fadd_rn(sum, __shfl_sync(kFull, my_w, j));
-        my_w = __fdiv_rn(my_w, sum);
-    }
-    if (lane < k) {
-        ids[t * k + lane] = my_id;
-        w[t * k + lane] = my_w;
-    }
-}
-
 template <int EPL>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T,
                                                          int E, int k, int32_t* __restrict__ ids,
@@ -174,34 +109,6 @@ __global__ void __launch_bounds__(1024) router_small_kernel(
     if (tid < 32) route_token_warp<EPL>(s_L, E, k, (size_t)t, ids, w, flags);
 }
 
-// ---------------------------------------------------------------------------------------------
-// Dispatch: count pairs per (expert, 32-token chunk).
-// ---------------------------------------------------------------------------------------------
-constexpr int kChunk = 32;   // tokens per chunk
-
-__global__ void __launch_bounds__(128) count_chunks_kernel(const int32_t* __restrict__ ids, int T,
-                                                           int E, int k, int nC,
-                                                           int32_t* __restrict__ cnt,
-                                                           DeviceStatus* st) {
-    pdl_begin();
-    extern __shared__ int32_t s_cnt[];                 // [4][E]
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int32_t* my = s_cnt + warp * E;
-    for (int e = lane; e < E; e += 32) my[e] = 0;
-    __syncwarp();
-    const int c = blockIdx.x * 4 + warp;
-    if (c >= nC) return;
-    const long long p0 = (long long)c * kChunk * k;
-    const long long p1 = (long long)min(T, (c + 1) * kChunk) * k;
-    for (long long p = p0 + lane; p < p1; p += 32) {
-        const int e = ids[p];
-        if ((unsigned)e >= (unsigned)E) { report(st, MOE_DEV_BAD_INDEX, 101); continue; }
-        atomicAdd(&my[e], 1);
-    }
-    __syncwarp();
-    for (int e = lane; e < E; e += 32) cnt[(size_t)e * nC + c] = my[e];
-}
-
 // Block-wide exclusive scan of one value per thread (blockDim.x a multiple of 32, <= 1024).
 // Returns the exclusive prefix; *total receives the block total.
 __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* total) {
@@ -230,152 +137,211 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
     return before + x - v;
 }
 
-// One block per expert: base[e][c] = sum of cnt[e][c' < c]; n[e] = total.
-__global__ void __launch_bounds__(256) scan_chunks_kernel(const int32_t* __restrict__ cnt, int nC,
-                                                          int32_t* __restrict__ base,
-                                                          int32_t* __restrict__ nrecv) {
+// ---------------------------------------------------------------------------------------------
+// Route + place.
+// ---------------------------------------------------------------------------------------------
+// A group of G lanes per token (G = 8, 16, 32 for E <= 64, 128, 256; k <= G).  Lane q of a group
+// owns the warp router's lanes l in [q*32/G, (q+1)*32/G) and, for each, experts l, l+32, ...; so
+// the fp32 arithmetic is exactly route_token_warp's: m = max; u_e = exp(L_e - m); lane partials
+// added left to right; then the pairwise tree p[l] += p[l + h], h = 16, 8, 4, 2, 1 (shuffles down
+// within the group where l + h belongs to another lane), which adds the same pairs as the warp's
+// xor butterfly; top-k by (logit desc, expert asc); w = u / S.  A block of 8 warps routes 64
+// consecutive tokens and places their pairs (block counters in shared memory, one global atomic
+// per (block, expert)).
+constexpr int kGroupBlockTokens = 64;
+
+template <int G>
+__global__ void __launch_bounds__(256) route_place_group_kernel(
+    const float* __restrict__ logits, int T, int E, int k, unsigned flags,
+    int32_t* __restrict__ ids, float* __restrict__ w, int32_t* __restrict__ gcnt,
+    int32_t* __restrict__ cand, DeviceStatus* st) {
     pdl_begin();
-    __shared__ int s_warp[32];
-    const int e = blockIdx.x;
-    const int32_t* in = cnt + (size_t)e * nC;
-    int32_t* out = base + (size_t)e * nC;
-    int carry = 0;
-    for (int c0 = 0; c0 < nC; c0 += blockDim.x) {
-        const int c = c0 + threadIdx.x;
-        const int v = c < nC ? in[c] : 0;
-        int tot;
-        const int ex = block_exclusive_scan(v, s_warp, &tot);
-        if (c < nC) out[c] = carry + ex;
-        carry += tot;
+    constexpr int LPL = 32 / G;                        // warp-router lanes per group lane
+    constexpr int NI = G / 4;                          // experts per warp-router lane: E <= 32 NI
+    constexpr int TPW = kGroupBlockTokens / 8;         // tokens per warp
+    constexpr int TPP = 32 / G;                        // tokens per warp per round
+    constexpr int R = TPW / TPP;                       // rounds
+    __shared__ int s_n[32 * NI], s_base[32 * NI];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane / G, q = lane % G;
+    for (int e = tid; e < 32 * NI; e += blockDim.x) s_n[e] = 0;
+    __syncthreads();
+    int my_e[R], my_pos[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        my_e[r] = -1;
+        my_pos[r] = 0;
+        const int t = blockIdx.x * kGroupBlockTokens + warp * TPW + r * TPP + g;
+        const bool active = t < T;                     // group-uniform
+        const float* Lr = logits + (size_t)(active ? t : 0) * E;
+        float v[LPL][NI];
+#pragma unroll
+        for (int li = 0; li < LPL; ++li)
+#pragma unroll
+            for (int i = 0; i < NI; ++i) {
+                const int e = q * LPL + li + 32 * i;
+                v[li][i] = (active && e < E) ? __ldg(Lr + e) : 0.0f;
+            }
+        float m = -INFINITY;
+#pragma unroll
+        for (int li = 0; li < LPL; ++li)
+#pragma unroll
+            for (int i = 0; i < NI; ++i)
+                if (q * LPL + li + 32 * i < E && v[li][i] > m) m = v[li][i];
+#pragma unroll
+        for (int o = G / 2; o >= 1; o >>= 1) {
+            const float y = __shfl_xor_sync(kFull, m, o, G);
+            m = y > m ? y : m;
+        }
+        float p[LPL];
+#pragma unroll
+        for (int li = 0; li < LPL; ++li) {
+            float acc = 0.0f;
+#pragma unroll
+            for (int i = 0; i < NI; ++i)
+                if (q * LPL + li + 32 * i < E)
+                    acc = __fadd_rn(acc, exp_cody_waite(__fsub_rn(v[li][i], m)));
+            p[li] = acc;
+        }
+#pragma unroll
+        for (int h = 16; h >= 1; h >>= 1) {
+            if (h >= LPL) {
+                const int dl = h / LPL;                // partner lane offset within the group
+#pragma unroll
+                for (int li = 0; li < LPL; ++li) {
+                    const float y = __shfl_down_sync(kFull, p[li], dl, G);
+                    if (q < dl) p[li] = __fadd_rn(p[li], y);
+                }
+            } else {
+#pragma unroll
+                for (int li = 0; li < LPL; ++li)
+                    if (li < h) p[li] = __fadd_rn(p[li], p[li + h]);
+            }
+        }
+        const float S = __shfl_sync(kFull, p[0], 0, G);
+        uint32_t taken = 0;                            // bit li * NI + i
+        int id_j = 0;
+        float w_j = 0.0f, wsum = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            float bl = 0.0f;
+            int be = 0x7fffffff, bb = -1;
+#pragma unroll
+            for (int li = 0; li < LPL; ++li)
+#pragma unroll
+                for (int i = 0; i < NI; ++i) {
+                    const int e = q * LPL + li + 32 * i;
+                    const bool ok = e < E && !((taken >> (li * NI + i)) & 1u) &&
+                                    (bb < 0 || v[li][i] > bl || (v[li][i] == bl && e < be));
+                    if (ok) { bl = v[li][i]; be = e; bb = li * NI + i; }
+                }
+#pragma unroll
+            for (int o = G / 2; o >= 1; o >>= 1) {
+                const float yl = __shfl_xor_sync(kFull, bl, o, G);
+                const int ye = __shfl_xor_sync(kFull, be, o, G);
+                if (ye != 0x7fffffff && (be == 0x7fffffff || yl > bl || (yl == bl && ye < be))) {
+                    bl = yl;
+                    be = ye;
+                }
+            }
+            if (bb >= 0 && q * LPL + bb / NI + 32 * (bb % NI) == be) taken |= 1u << bb;
+            const float wj = __fdiv_rn(exp_cody_waite(__fsub_rn(bl, m)), S);
+            wsum = __fadd_rn(wsum, wj);
+            if (q == j) { id_j = be; w_j = wj; }
+        }
+        if (active && q < k) {
+            const size_t pj = (size_t)t * k + q;
+            ids[pj] = id_j;
+            w[pj] = (flags & MOE_FLAG_RENORMALIZE) ? __fdiv_rn(w_j, wsum) : w_j;
+            my_e[r] = id_j;
+            my_pos[r] = atomicAdd(&s_n[id_j], 1);
+        }
     }
-    if (threadIdx.x == 0) nrecv[e] = carry;
+    __syncthreads();
+    for (int e = tid; e < E; e += blockDim.x) s_base[e] = s_n[e] ? atomicAdd(&gcnt[e], s_n[e]) : 0;
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        if (my_e[r] < 0) continue;
+        const int t = blockIdx.x * kGroupBlockTokens + warp * TPW + r * TPP + g;
+        const long long pos = (long long)s_base[my_e[r]] + my_pos[r];
+        if (pos < T) cand[(size_t)my_e[r] * T + pos] = t * k + q;
+        else report(st, MOE_DEV_BAD_INDEX, 131);        // counters were not zero at entry
+    }
 }
 
-// One warp per chunk: stable scatter of the chunk's pairs into cand[e][.] (ascending tokens).
-__global__ void __launch_bounds__(128) scatter_chunks_kernel(const int32_t* __restrict__ ids,
-                                                             int T, int E, int k, int nC,
-                                                             const int32_t* __restrict__ base,
-                                                             int32_t* __restrict__ cand) {
+// One warp per token (any E <= 1024, k <= 32): route_token_warp, then the same placement.  A
+// block of 8 warps takes 64 consecutive tokens, 8 per warp; lane j keeps pair j of each.
+constexpr int kWarpRouteTokens = 64;
+
+template <int EPL>
+__global__ void __launch_bounds__(256) route_place_warp_kernel(
+    const float* __restrict__ logits, int T, int E, int k, unsigned flags,
+    int32_t* __restrict__ ids, float* __restrict__ w, int32_t* __restrict__ gcnt,
+    int32_t* __restrict__ cand, DeviceStatus* st) {
     pdl_begin();
-    extern __shared__ int32_t s_run[];                 // [4][E]
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int c = blockIdx.x * 4 + warp;
-    if (c >= nC) return;
-    int32_t* run = s_run + warp * E;
-    for (int e = lane; e < E; e += 32) run[e] = base[(size_t)e * nC + c];
-    __syncwarp();
-    const long long p0 = (long long)c * kChunk * k;
-    const long long p1 = (long long)min(T, (c + 1) * kChunk) * k;
-    // The chunk's ids are loaded 8 rounds of 32 at a time (independent loads in flight), then
-    // placed round by round in pair order.
-    for (long long pg = p0; pg < p1; pg += 8 * 32) {
-        int ev[8];
+    extern __shared__ int s_nb[];                       // [E] counts, then [E] bases
+    int* s_n = s_nb;
+    int* s_base = s_nb + E;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int e = tid; e < E; e += blockDim.x) s_n[e] = 0;
+    __syncthreads();
+    constexpr int kPer = kWarpRouteTokens / 8;
+    int my_e[kPer], my_pos[kPer];
+    const int t0 = blockIdx.x * kWarpRouteTokens + warp * kPer;
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            const long long p = pg + 32 * r + lane;
-            ev[r] = p < p1 ? ids[p] : -1;
-        }
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            const long long p = pg + 32 * r + lane;
-            if (pg + 32 * r >= p1) break;               // warp-uniform
-            int e = ev[r];
-            if ((unsigned)e >= (unsigned)E) e = -1;    // bad ids were reported by the count pass
-            const unsigned peers = __match_any_sync(kFull, e);
-            const int rank = __popc(peers & ((1u << lane) - 1u));
-            const int pos = (e >= 0) ? run[e] + rank : 0;
-            __syncwarp();
-            if (p < p1 && e >= 0) {
-                cand[(size_t)e * T + pos] = (int32_t)p;
-                if (lane == __ffs(peers) - 1) run[e] = pos + __popc(peers);
-            }
-            __syncwarp();
+    for (int i = 0; i < kPer; ++i) {
+        my_e[i] = -1;
+        const int t = t0 + i;
+        if (t < T) {
+            my_e[i] = route_token_warp<EPL>(logits + (size_t)t * E, E, k, (size_t)t, ids, w, flags);
+            if (my_e[i] >= 0) my_pos[i] = atomicAdd(&s_n[my_e[i]], 1);
         }
     }
+    __syncthreads();
+    for (int e = tid; e < E; e += blockDim.x) s_base[e] = s_n[e] ? atomicAdd(&gcnt[e], s_n[e]) : 0;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+        if (my_e[i] >= 0) {
+            const long long pos = (long long)s_base[my_e[i]] + my_pos[i];
+            if (pos < T) cand[(size_t)my_e[i] * T + pos] = (t0 + i) * k + lane;
+            else report(st, MOE_DEV_BAD_INDEX, 132);    // counters were not zero at entry
+        }
 }
 
 // ---------------------------------------------------------------------------------------------
-// Capacity selection: one block per expert.
+// Capacity selection from unordered candidate lists: one block per expert.
 // ---------------------------------------------------------------------------------------------
 constexpr int kSelThreads = 1024;
-constexpr int kSelSmemKeys = 16384;   // candidates of one expert whose list and keys stay on chip
+constexpr int kSelSmem = 220 * 1024;  // dynamic shared memory of the selection kernel
+constexpr int kSelBitWords = 8192;    // token-bitmap words kept on chip (T <= 262144)
 
-__global__ void __launch_bounds__(kSelThreads) select_kernel(
-    const int32_t* __restrict__ cand, const int32_t* __restrict__ nrecv,
-    const float* __restrict__ w, int T, int E, int k, long long K, int32_t* __restrict__ slot,
-    uint8_t* __restrict__ drop, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-    int32_t* __restrict__ rowtok, unsigned flags) {
-    pdl_begin();
-    extern __shared__ uint32_t s_keys[];              // [kSelSmemKeys] keys, then the list
-    int32_t* s_list = reinterpret_cast<int32_t*>(s_keys + kSelSmemKeys);
-    __shared__ int s_warp[32];
-    __shared__ int s_hist[256];
-    __shared__ uint32_t s_prefix;
-    __shared__ int s_remaining;
-    const int e = blockIdx.x;
+// Radix select over the keys of candidates i < n (most significant byte first), restricted to
+// those with filter(i): finds the `want`-th largest key; returns it, and in *rem how many
+// candidates equal to it are among the `want` largest.
+template <class KeyFn, class FilterFn>
+__device__ __forceinline__ uint32_t radix_select(int n, int want, KeyFn key_of, FilterFn filter,
+                                                 int* s_hist, uint32_t* s_prefix, int* s_rem,
+                                                 int* rem) {
     const int tid = threadIdx.x;
-    const int n = nrecv[e];
-    const int kept = (int)min((long long)n, K);
-
-    // Row offset of this expert: sum of kept counts of the experts before it.
-    int part = 0;
-    for (int q = tid; q < e; q += blockDim.x) part += (int)min((long long)nrecv[q], K);
-    int off_tot;
-    (void)block_exclusive_scan(part, s_warp, &off_tot);
-    const int off = off_tot;
-    if (tid == 0) {
-        if (counts) { counts[e] = n; counts[E + e] = kept; }
-        if (offsets) {
-            offsets[e] = off;
-            if (e == E - 1) offsets[E] = off + kept;
-        }
-    }
-    const int32_t* list = cand + (size_t)e * T;
-
-    if (K == 0) {                       // no slots: every pair of this expert is dropped
-        for (int i = tid; i < n; i += blockDim.x) {
-            const int p = list[i];
-            slot[p] = -1;
-            drop[p] = 1;
-        }
-        return;
-    }
-    if (n <= K || (flags & MOE_FLAG_ARRIVAL_ORDER)) {
-        // Everything fits, or arrival order: the first K candidates (ascending token) get in.
-        for (int i = tid; i < n; i += blockDim.x) {
-            const int p = list[i];
-            const bool keep = i < K;
-            slot[p] = keep ? i : -1;
-            drop[p] = keep ? 0 : 1;
-            if (keep && rowtok) rowtok[off + i] = p / k;
-        }
-        return;
-    }
-
-    // Weight bit patterns of the candidates (weights are >= +0, so the bits order like the
-    // values), gathered once into shared memory when they fit.
-    const bool on_chip = n <= kSelSmemKeys;
-    if (on_chip)
-        for (int i = tid; i < n; i += blockDim.x) {
-            const int p = list[i];
-            s_list[i] = p;
-            s_keys[i] = __float_as_uint(w[p]);
-        }
-    __syncthreads();
-    auto key_of = [&](int i) -> uint32_t {
-        return on_chip ? s_keys[i] : __float_as_uint(w[list[i]]);
-    };
-
-    // Radix select (most significant byte first) of the K-th largest key.
     uint32_t prefix = 0, mask = 0;
-    int remaining = (int)K;
+    int remaining = want;
     for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
         for (int b = tid; b < 256; b += blockDim.x) s_hist[b] = 0;
         __syncthreads();
-        for (int i = tid; i < n; i += blockDim.x) {
-            const uint32_t key = key_of(i);
-            if ((key & mask) == prefix) atomicAdd(&s_hist[(key >> shift) & 255u], 1);
+        // Keys share few values in their high bytes (softmax weights differ mostly in the
+        // mantissa): one atomic per distinct bin per warp, not per key.
+        for (int i0 = 0; i0 < n; i0 += blockDim.x) {
+            const int i = i0 + tid;
+            int bin = -1;
+            if (i < n && filter(i)) {
+                const uint32_t key = key_of(i);
+                if ((key & mask) == prefix) bin = (int)((key >> shift) & 255u);
+            }
+            const unsigned peers = __match_any_sync(kFull, bin);
+            if (bin >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1)
+                atomicAdd(&s_hist[bin], __popc(peers));
         }
         __syncthreads();
         if (tid < 32) {
@@ -398,8 +364,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
                 for (int q = 0; q < 8; ++q) {
                     const int b = 255 - 8 * tid - q;
                     if (run + s_hist[b] >= remaining) {
-                        s_prefix = prefix | ((uint32_t)b << shift);
-                        s_remaining = remaining - run;
+                        *s_prefix = prefix | ((uint32_t)b << shift);
+                        *s_rem = remaining - run;
                         break;
                     }
                     run += s_hist[b];
@@ -407,38 +373,148 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
             }
         }
         __syncthreads();
-        prefix = s_prefix;
-        remaining = s_remaining;
+        prefix = *s_prefix;
+        remaining = *s_rem;
         mask |= 255u << shift;
         __syncthreads();
     }
-    const uint32_t tau = prefix;        // K-th largest weight bits
-    const int need_eq = remaining;      // how many weights equal to tau are kept (lowest t first)
-    // After the last pass s_hist[tau & 255] counts the keys equal to tau.  When all of them are
-    // kept (no tie straddles the capacity boundary, the usual case) keep = (key >= tau) and the
-    // tie ranks are not needed.
-    const bool all_eq_kept = s_hist[tau & 255u] == need_eq;
+    *rem = remaining;
+    return prefix;
+}
 
-    int eq_carry = 0, keep_carry = 0;
-    for (int i0 = 0; i0 < n; i0 += blockDim.x) {
-        const int i = i0 + tid;
-        int p = 0;
-        uint32_t key = 0;
-        if (i < n) { p = on_chip ? s_list[i] : list[i]; key = key_of(i); }
-        const int is_eq = (i < n && key == tau) ? 1 : 0;
-        int eq_tot = 0, eq_rank = 0;
-        if (!all_eq_kept) eq_rank = eq_carry + block_exclusive_scan(is_eq, s_warp, &eq_tot);
-        const int keep =
-            (i < n) && (key > tau || (is_eq && (all_eq_kept || eq_rank < need_eq))) ? 1 : 0;
-        int keep_tot;
-        const int s = keep_carry + block_exclusive_scan(keep, s_warp, &keep_tot);
-        if (i < n) {
-            slot[p] = keep ? s : -1;
-            drop[p] = keep ? 0 : 1;
-            if (keep && rowtok) rowtok[off + s] = p / k;
+// Keys order candidates by priority, larger first: the weight's bit pattern (weights are >= +0,
+// so their bits order like their values), or for MOE_FLAG_ARRIVAL_ORDER the complement of the
+// pair index (earlier tokens first).  Among equal weights the lower pair index (the lower
+// token) wins.  `gbits` (null when the bitmap fits on chip) is [E][2 * ceil(T/32)] words.
+__global__ void __launch_bounds__(kSelThreads) select_kernel(
+    const int32_t* __restrict__ cand, const int32_t* __restrict__ gcnt,
+    const float* __restrict__ w, int T, int E, int k, long long K, unsigned flags,
+    uint32_t* __restrict__ gbits, int keys_cap, int32_t* __restrict__ slot,
+    uint8_t* __restrict__ drop, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ rowtok, DeviceStatus* st) {
+    pdl_begin();
+    extern __shared__ uint32_t s_dyn[];
+    __shared__ int s_warp[32];
+    __shared__ int s_hist[256];
+    __shared__ uint32_t s_prefix;
+    __shared__ int s_rem;
+    const int e = blockIdx.x, tid = threadIdx.x;
+    const int nw = (T + 31) / 32;
+    uint32_t* bits = gbits ? gbits + (size_t)e * 2 * nw : s_dyn;       // [nw] kept tokens
+    uint32_t* pre = bits + nw;                                          // [nw] prefix popcounts
+    uint32_t* s_keys = s_dyn + (gbits ? 0 : 2 * nw);                   // [keys_cap]
+    int32_t* s_list = reinterpret_cast<int32_t*>(s_keys + keys_cap);   // [keys_cap]
+    const long long P = (long long)T * k;
+
+    int n = gcnt[e];
+    if (n < 0 || n > T) {
+        if (tid == 0) report(st, MOE_DEV_BAD_INDEX, 121);
+        n = n < 0 ? 0 : T;
+    }
+    const int kept = (int)min((long long)n, K);
+    // Row offset of this expert: kept counts of the experts before it.
+    int part = 0;
+    for (int q = tid; q < e; q += blockDim.x) part += (int)min((long long)min(max(gcnt[q], 0), T), K);
+    int off;
+    (void)block_exclusive_scan(part, s_warp, &off);
+    if (tid == 0) {
+        if (counts) { counts[e] = n; counts[E + e] = kept; }
+        if (offsets) {
+            offsets[e] = off;
+            if (e == E - 1) offsets[E] = off + kept;
         }
-        eq_carry += eq_tot;
-        keep_carry += keep_tot;
+    }
+    if (n == 0) return;
+    const int32_t* list = cand + (size_t)e * T;
+    const bool arrival = (flags & MOE_FLAG_ARRIVAL_ORDER) != 0;
+    const bool on_chip = n <= keys_cap;
+    auto pair_of = [&](int i) -> int32_t {
+        const int32_t p = on_chip ? s_list[i] : list[i];
+        return p;
+    };
+    auto key_from = [&](int32_t p) -> uint32_t {
+        return arrival ? ~(uint32_t)p : __float_as_uint(w[p]);
+    };
+    if (on_chip)
+        for (int i = tid; i < n; i += blockDim.x) {
+            int32_t p = list[i];
+            if (p < 0 || p >= P) { report(st, MOE_DEV_BAD_INDEX, 122); p = -1; }
+            s_list[i] = p;
+            s_keys[i] = p < 0 ? 0u : key_from(p);
+        }
+    for (int i = tid; i < nw; i += blockDim.x) bits[i] = 0;
+    __syncthreads();
+    auto key_of = [&](int i) -> uint32_t {
+        if (on_chip) return s_keys[i];
+        const int32_t p = list[i];
+        return (p < 0 || p >= P) ? 0u : key_from(p);
+    };
+    auto valid = [&](int i) -> bool {
+        const int32_t p = pair_of(i);
+        return p >= 0 && p < P;
+    };
+
+    uint32_t tau = 0;                 // keys > tau are kept; keys == tau when pair <= p_tau
+    int32_t p_tau = 0x7fffffff;
+    bool select_all = n <= K;
+    if (!select_all && K > 0) {
+        int need_eq;
+        tau = radix_select(n, (int)K, key_of, valid, s_hist, &s_prefix, &s_rem, &need_eq);
+        // Candidates equal to tau: are all of them among the K largest?  Count them.
+        int eqc = 0;
+        for (int i = tid; i < n; i += blockDim.x) eqc += (valid(i) && key_of(i) == tau) ? 1 : 0;
+        int eq_tot;
+        (void)block_exclusive_scan(eqc, s_warp, &eq_tot);
+        if (eq_tot > need_eq) {
+            // Ties straddle the boundary: keep the need_eq tied pairs with the lowest index.
+            int dummy;
+            p_tau = (int32_t)~radix_select(
+                n, need_eq, [&](int i) -> uint32_t { return ~(uint32_t)pair_of(i); },
+                [&](int i) -> bool { return valid(i) && key_of(i) == tau; }, s_hist, &s_prefix,
+                &s_rem, &dummy);
+        }
+    }
+    // Mark kept tokens.
+    for (int i = tid; i < n; i += blockDim.x) {
+        if (!valid(i)) continue;
+        const int32_t p = pair_of(i);
+        const uint32_t key = key_of(i);
+        const bool keep = K > 0 && (select_all || key > tau || (key == tau && p <= p_tau));
+        if (keep) {
+            const int t = p / k;
+            atomicOr(&bits[t >> 5], 1u << (t & 31));
+        }
+    }
+    __syncthreads();
+    // Exclusive prefix of popcounts over the bitmap words, 1024 words per round.
+    int carry = 0;
+    for (int w0 = 0; w0 < nw; w0 += blockDim.x) {
+        const int wi = w0 + tid;
+        const int c = wi < nw ? __popc(bits[wi]) : 0;
+        int tot;
+        const int ex = block_exclusive_scan(c, s_warp, &tot);
+        if (wi < nw) pre[wi] = carry + ex;
+        carry += tot;
+    }
+    __syncthreads();
+    for (int i = tid; i < n; i += blockDim.x) {
+        if (!valid(i)) continue;
+        const int32_t p = pair_of(i);
+        const int t = p / k;
+        const uint32_t word = bits[t >> 5], bit = 1u << (t & 31);
+        if (word & bit) {
+            const int sl = (int)pre[t >> 5] + __popc(word & (bit - 1u));
+            if (sl >= kept) {                   // only with duplicated pairs in the list
+                report(st, MOE_DEV_BAD_INDEX, 123);
+                continue;
+            }
+            slot[p] = sl;
+            drop[p] = 0;
+            if (rowtok) rowtok[off + sl] = t;
+        } else {
+            slot[p] = -1;
+            drop[p] = 1;
+        }
     }
 }
 
@@ -650,7 +726,6 @@ void launch_route_topk(const float* logits, int T, int E, int k, int32_t* ids, f
     else launch_route_t<32>(logits, T, E, k, ids, w, s, flags);
 }
 
-int chunk_count(int T) { return (T + kChunk - 1) / kChunk; }
 
 bool dispatch_small_fits(int T, int k) { return (long long)T * k <= kSmallPairs; }
 
@@ -707,34 +782,82 @@ void launch_dispatch_small(const int32_t* ids, const float* w, int T, int E, int
     *launches += 1;
 }
 
-void launch_capacity_select(const int32_t* ids, const float* w, int T, int E, int k, long long K,
-                            int32_t* cnt, int32_t* base, int32_t* nrecv, int32_t* cand,
-                            int32_t* slot, uint8_t* drop, int32_t* counts, int32_t* offsets,
-                            int32_t* rowtok, DeviceStatus* st, cudaStream_t s, int* launches,
-                            bool counts_ready, unsigned flags) {
-    const int nC = chunk_count(T);
-    const int blocks = (nC + 3) / 4;
-    const size_t smem = (size_t)4 * E * sizeof(int32_t);
-    if (!counts_ready) {
-        launch_pdl(count_chunks_kernel, dim3(blocks), dim3(128), smem, s, ids, T, E, k, nC, cnt,
-                   st);
-        *launches += 1;
+// Lanes per token of the group router (0: the warp router with more experts per lane).
+int route_group_lanes(int E, int k) {
+    const int G = E <= 64 ? 8 : (E <= 128 ? 16 : (E <= 256 ? 32 : 0));
+    return (G > 0 && k <= G) ? G : 0;
+}
+
+void launch_route_place(const float* logits, int T, int E, int k, unsigned flags, int32_t* ids,
+                        float* w, int32_t* gcnt, int32_t* cand, DeviceStatus* st, cudaStream_t s,
+                        int* launches) {
+    if (T == 0) return;
+    const int G = route_group_lanes(E, k);
+    if (G > 0) {
+        const dim3 g((T + kGroupBlockTokens - 1) / kGroupBlockTokens);
+        if (G == 8)
+            launch_pdl(route_place_group_kernel<8>, g, dim3(256), 0, s, logits, T, E, k, flags,
+                       ids, w, gcnt, cand, st);
+        else if (G == 16)
+            launch_pdl(route_place_group_kernel<16>, g, dim3(256), 0, s, logits, T, E, k, flags,
+                       ids, w, gcnt, cand, st);
+        else
+            launch_pdl(route_place_group_kernel<32>, g, dim3(256), 0, s, logits, T, E, k, flags,
+                       ids, w, gcnt, cand, st);
+    } else {
+        const dim3 g((T + kWarpRouteTokens - 1) / kWarpRouteTokens);
+        const size_t smem = 2 * sizeof(int) * (size_t)E;
+        const int epl = (E + 31) / 32;
+        if (epl <= 1)
+            launch_pdl(route_place_warp_kernel<1>, g, dim3(256), smem, s, logits, T, E, k, flags,
+                       ids, w, gcnt, cand, st);
+        else if (epl <= 2)
+            launch_pdl(route_place_warp_kernel<2>, g, dim3(256), smem, s, logits, T, E, k, flags,
+                       ids, w, gcnt, cand, st);
+        else if (epl <= 4)
+            launch_pdl(route_place_warp_kernel<4>, g, dim3(256), smem, s, logits, T, E, k, flags,
+                       ids, w, gcnt, cand, st);
+        else if (epl <= 8)
+            launch_pdl(route_place_warp_kernel<8>, g, dim3(256), smem, s, logits, T, E, k, flags,
+                       ids, w, gcnt, cand, st);
+        else if (epl <= 16)
+            launch_pdl(route_place_warp_kernel<16>, g, dim3(256), smem, s, logits, T, E, k, flags,
+                       ids, w, gcnt, cand, st);
+        else
+            launch_pdl(route_place_warp_kernel<32>, g, dim3(256), smem, s, logits, T, E, k, flags,
+                       ids, w, gcnt, cand, st);
     }
-    launch_pdl(scan_chunks_kernel, dim3(E), dim3(256), 0, s, cnt, nC, base, nrecv);
-    launch_pdl(scatter_chunks_kernel, dim3(blocks), dim3(128), smem, s, ids, T, E, k, nC, base,
-               cand);
+    *launches += 1;
+}
+
+size_t select_bits_bytes(int T, int E) {
+    const size_t nw = ((size_t)T + 31) / 32;
+    return nw <= (size_t)kSelBitWords ? 0 : (size_t)E * 2 * nw * sizeof(uint32_t);
+}
+
+void launch_select(const int32_t* cand, const int32_t* gcnt, const float* w, int T, int E, int k,
+                   long long K, unsigned flags, uint32_t* gbits, int32_t* slot, uint8_t* drop,
+                   int32_t* counts, int32_t* offsets, int32_t* rowtok, DeviceStatus* st,
+                   cudaStream_t s, int* launches) {
+    const size_t nw = ((size_t)T + 31) / 32;
+    const bool bits_on_chip = nw <= (size_t)kSelBitWords;
+    // Candidates whose keys and pair indices fit next to the bitmap stay on chip; an expert with
+    // more keeps reading them from global memory.
+    const size_t bits_smem = bits_on_chip ? 2 * nw * 4 : 0;
+    const int keys_cap = (int)((kSelSmem - bits_smem) / 8);
+    const size_t smem = kSelSmem;
     static std::atomic<uint64_t> attr_done{0};
     int dev = 0;
     cudaGetDevice(&dev);
     const uint64_t bit = 1ull << (dev & 63);
     if (!(attr_done.load() & bit)) {
-        cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSelSmemKeys * 8);
+        cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelSmem);
         attr_done.fetch_or(bit);
     }
-    launch_pdl(select_kernel, dim3(E), dim3(kSelThreads), kSelSmemKeys * 8, s, cand, nrecv, w, T, E,
-               k, K, slot, drop, counts, offsets, rowtok, flags);
-    *launches += 3;
+    launch_pdl(select_kernel, dim3(E), dim3(kSelThreads), smem, s, cand, gcnt, w, T, E, k, K,
+               flags, bits_on_chip ? nullptr : gbits, keys_cap, slot, drop, counts, offsets, rowtok,
+               st);
+    *launches += 1;
 }
 
 void launch_dispatch(const int32_t* ids, const int32_t* slot, int T, int E, int k,

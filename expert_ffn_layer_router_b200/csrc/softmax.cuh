@@ -1,9 +1,15 @@
 // softmax.cuh -- the router's fp32 arithmetic, shared by the warp-per-token router (route.cu)
 // and the fused router epilogue of the logits GEMM (gemm_tc.cu), so both form bit-identical
 // weights from the same logits.
+//
+// One token is routed by one warp: lane l holds experts l, l+32, ...; the softmax sum adds the
+// lane partials left to right, then an xor butterfly 16, 8, 4, 2, 1; the top-k picks experts by
+// (logit descending, expert ascending) and divides exp(L - m) by the sum once.
 #pragma once
 
 #include <cstdint>
+
+#include "common.cuh"
 
 namespace moe {
 
@@ -46,6 +52,76 @@ __device__ __forceinline__ uint32_t float_key(float v) {
 }
 __device__ __forceinline__ float key_float(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Lane j < k receives the j-th expert of token t (largest logit first) and its weight, writes
+// them to ids[t*k + j], w[t*k + j] and returns the expert id; other lanes return -1.
+template <int EPL>
+__device__ __forceinline__ int route_token_warp(const float* L, int E, int k, size_t t,
+                                                int32_t* __restrict__ ids, float* __restrict__ w,
+                                                unsigned flags) {
+    constexpr unsigned kFull = 0xffffffffu;
+    const int lane = threadIdx.x & 31;
+    float v[EPL];
+    uint32_t key[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = e < E ? L[e] : 0.0f;
+        key[i] = e < E ? float_key(v[i]) : 0u;
+    }
+    uint32_t lmax = 0;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) lmax = max(lmax, key[i]);
+    const float m = key_float(__reduce_max_sync(kFull, lmax));
+    float u[EPL];
+    float part = 0.0f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        u[i] = e < E ? exp_cody_waite(__fsub_rn(v[i], m)) : 0.0f;
+        if (e < E) part = __fadd_rn(part, u[i]);
+    }
+#pragma unroll
+    for (int h = 16; h >= 1; h >>= 1) part = __fadd_rn(part, __shfl_xor_sync(kFull, part, h));
+    const float S = part;
+
+    int my_id = 0;
+    float my_w = 0.0f;
+    uint32_t taken = 0;
+    for (int j = 0; j < k; ++j) {
+        uint32_t bk = 0;
+        int bi = 0;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const bool ok = !((taken >> i) & 1u) && key[i] > bk;
+            bk = ok ? key[i] : bk;
+            bi = ok ? i : bi;
+        }
+        const uint32_t wk = __reduce_max_sync(kFull, bk);
+        const unsigned cand = (bk == wk && bk != 0u) ? (unsigned)(lane + 32 * bi) : 0x7fffffffu;
+        const int we = (int)__reduce_min_sync(kFull, cand);
+        float up = 0.0f;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) up = (i == bi) ? u[i] : up;
+        const float wu = __shfl_sync(kFull, up, we & 31);
+        if (lane == (we & 31)) taken |= 1u << (we >> 5);
+        if (lane == j) {
+            my_id = we;
+            my_w = __fdiv_rn(wu, S);
+        }
+    }
+    if (flags & MOE_FLAG_RENORMALIZE) {
+        // Sum of the k weights in j order, then one division each.
+        float sum = 0.0f;
+        for (int j = 0; j < k; ++j) sum = __fadd_rn(sum, __shfl_sync(kFull, my_w, j));
+        my_w = __fdiv_rn(my_w, sum);
+    }
+    if (lane < k) {
+        ids[t * k + lane] = my_id;
+        w[t * k + lane] = my_w;
+    }
+    return lane < k ? my_id : -1;
 }
 
 }  // namespace moe

@@ -154,8 +154,10 @@ moe_status moe_combine(const moe_problem* p, const void* x, const void* Y, const
 /* The whole layer: logits = x Wr + br (Wr [d_model, E] float32, br [E] float32 or NULL), then
  * the four steps.  out [T, d_model] in x's dtype.  Optional outputs (NULL = keep in ws):
  * logits_out [T, E], ids_out, w_out, slot_out [T*k], drop_out [T*k], counts_out [2E].
- * With dtype MOE_BF16 the logits come from the tensor cores with Wr split exactly into three
- * bfloat16 terms and float32 accumulation. */
+ * With dtype MOE_BF16 the logits come from the tensor cores with Wr split into two bfloat16 terms
+ * (hi = bf16(Wr), mid = bf16(Wr - hi); the remainder is below 2^-18 |Wr|) and float32
+ * accumulation; the routing of those logits is bit for bit the routing moe_route gives for them
+ * (logits_out exports them). */
 moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, const float* br,
                        const void* W1, const float* b1, const void* W2, const float* b2,
                        void* out, float* logits_out, int32_t* ids_out, float* w_out,

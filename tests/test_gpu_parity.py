@@ -85,6 +85,15 @@ def test_route_weight_ties():
     _assert_route_equal(g, ro, 12)
 
 
+def test_route_large_batch_global_bitmap():
+    # More than 262144 tokens: the capacity selection keeps its token bitmap in the workspace.
+    T, E, k = 300000, 4, 2
+    L = inputs.random_logits(T, E, 12, 1.0)
+    _, g, ro = _route_both(L, T, E, k, 0.5)
+    _assert_route_equal(g, ro, E)
+    assert ro["drop"].sum() > 0
+
+
 def test_route_empty():
     moe = _moe()
     layer = moe.MoELayer(0, 64, 64, 8, 2, 1.0, "bf16")
@@ -128,6 +137,10 @@ def test_dispatch_bit_exact(T, E, k, C, dtype):
     (1000, 256, 1408, 4, 1, 1.25, "bf16", 0.02),   # d_ff = 1408: 256-wide tiles, the last half full
     (700, 512, 320, 3, 3, 0.9, "bf16", 0.0),       # several m-tiles per expert, a ragged column tile
     (129, 64, 64, 2, 1, math.inf, "bf16", 0.1),    # 129 rows: one full tile + one row
+    (2000, 256, 1408, 4, 2, 1.25, "bf16", 0.02),   # gathered rows, half-width last tile
+    (2000, 640, 256, 4, 2, 1.25, "bf16", 0.02),    # second GEMM on CTA pairs, half-width last tile
+    (1024, 128, 192, 4, 1, math.inf, "bf16", 0.05),  # exactly 256 rows per expert: pairs
+    (1023, 128, 192, 4, 1, math.inf, "bf16", 0.05),  # one row short of that: single-CTA tiles
     (40, 16, 24, 4, 2, 1.0, "f32", 0.1),
     (8, 4, 8, 4, 1, 1.25, "f32", 0.1)])
 def test_expert_ffn_parity(T, d, F, E, k, C, dtype, bias):
