@@ -353,8 +353,9 @@ __global__ void logits_f32_kernel(const float* __restrict__ x, const float* __re
                                   const float* __restrict__ br, int T, int d, int E,
                                   float* __restrict__ L, int32_t* __restrict__ zero, int zero_n) {
     pdl_begin();
-    if (zero && blockIdx.x == 0)
-        for (int i = threadIdx.x; i < zero_n; i += blockDim.x) zero[i] = 0;
+    if (zero)
+        for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < zero_n; i += gridDim.x * blockDim.x)
+            zero[i] = 0;
     const long long n = (long long)T * E;
     for (long long q = blockIdx.x * (long long)blockDim.x + threadIdx.x; q < n;
          q += (long long)gridDim.x * blockDim.x) {

@@ -197,6 +197,14 @@ __device__ __forceinline__ void pdl_begin() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// The first failed launch (or stream operation) of the current API call on this host thread; the
+// entry points clear it on entry and report it as MOE_ERR_CUDA.
+inline thread_local cudaError_t g_launch_error = cudaSuccess;
+inline cudaError_t note_launch(cudaError_t e) {
+    if (e != cudaSuccess && g_launch_error == cudaSuccess) g_launch_error = e;
+    return e;
+}
+
 // <<<grid, block, smem, s>>> with the programmatic-stream-serialization attribute.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
@@ -211,7 +219,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, args...);
+    return note_launch(cudaLaunchKernelEx(&cfg, kernel, args...));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -736,10 +736,12 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
                                                            int32_t* __restrict__ zero,
                                                            int zero_n) {
     pdl_begin();
-    // The dispatch counters of this call start at zero (the routing kernel after the logits GEMM
-    // adds to them).
-    if (zero && blockIdx.x == 0 && blockIdx.y == 0)
-        for (int i = threadIdx.x; i < zero_n; i += blockDim.x) zero[i] = 0;
+    // The dispatch counters and histograms of this call start at zero (the routing kernel after
+    // the logits GEMM adds to them); every block clears a slice.
+    if (zero) {
+        const int nb = gridDim.x * gridDim.y, bid = blockIdx.y * gridDim.x + blockIdx.x;
+        for (int i = bid * blockDim.x + threadIdx.x; i < zero_n; i += nb * blockDim.x) zero[i] = 0;
+    }
     constexpr int kPer = (kSplitK * Eg + 255) / 256;
     __shared__ float s_w[kSplitK][Eg + 1];
     const int k0 = blockIdx.x * kSplitK, nt = blockIdx.y;
@@ -884,7 +886,7 @@ cudaError_t launch_gemm_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const 
     at2[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at2;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmD, a);
+    return note_launch(cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmD, a));
 }
 
 template <int EPI, bool GATHER, bool PAIR>

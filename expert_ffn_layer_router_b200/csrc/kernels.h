@@ -15,8 +15,11 @@ struct DeviceStatus;
 void launch_route_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
                        cudaStream_t s, unsigned flags);
 // Routing of T tokens from their logits (ids, w) that also appends every pair p = t*k + j to its
-// expert's candidate list cand[e][.] ([E][T]) and counts it in gcnt[e]; gcnt must be zero at
-// entry.  A group of route_group_lanes(E, k) lanes per token when that is not 0, else a warp.
+// expert's candidate list cand[e][.] ([E][T]), counts it in gcnt[e] and in a per-expert histogram
+// of weight keys that follows gcnt; the dispatch_counter_ints(E) ints at gcnt must be zero at
+// entry.
+// A group of route_group_lanes(E, k) lanes routes each token when that is not 0, else a warp.
+size_t dispatch_counter_ints(int E);
 int route_group_lanes(int E, int k);
 void launch_route_place(const float* logits, int T, int E, int k, unsigned flags, int32_t* ids,
                         float* w, int32_t* gcnt, int32_t* cand, DeviceStatus* st, cudaStream_t s,

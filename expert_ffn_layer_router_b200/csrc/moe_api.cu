@@ -76,7 +76,7 @@ Plan make_plan(const moe_problem* p) {
         return at;
     };
     q.status = take(sizeof(moe::DeviceStatus));
-    q.gcnt = take((size_t)p->E * 4);
+    q.gcnt = take(moe::dispatch_counter_ints(p->E) * 4);
     q.logits = take((size_t)p->T * p->E * 4);
     q.ids = take(P * 4);
     q.w = take(P * 4);
@@ -110,7 +110,7 @@ moe_status check_ws(const moe_problem* p, const void* ws, size_t ws_bytes, Plan*
 
 moe_status finish(int launches) {
     const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (e != cudaSuccess || moe::g_launch_error != cudaSuccess) return MOE_ERR_CUDA;
     g_last_launches = launches;
     return MOE_OK;
 }
@@ -121,13 +121,15 @@ moe_status pre(const moe_problem* p, bool needs_ffn) {
     if (bad_problem(p)) return MOE_ERR_INVALID_ARG;
     if (needs_ffn && unsupported(p)) return MOE_ERR_UNSUPPORTED;
     cudaGetLastError();   // a stale error from unrelated work must not be blamed on this call
+    moe::g_launch_error = cudaSuccess;
     return MOE_OK;
 }
 
 // Scratch of the routing and capacity selection (the workspace's, or the static array's).
 struct RouteScratch {
     moe::DeviceStatus* st;
-    int32_t* gcnt;      // [E] pairs received per expert, zero at entry of the route kernel
+    int32_t* gcnt;      // [E] pairs received per expert, then [E][2048] weight-key histograms;
+                        // dispatch_counter_ints(E) ints, zero at entry of the route kernel
     int32_t* cand;      // [E][T] candidate lists
     uint32_t* bits;     // select_bits_bytes(T, E) bytes, or null when that is 0
 };
@@ -147,7 +149,7 @@ void route_steps(const moe_problem* p, const float* logits, int32_t* ids, float*
                                    offsets, rowtok, rs.st, s, launches);
         return;
     }
-    cudaMemsetAsync(rs.gcnt, 0, sizeof(int32_t) * p->E, s);
+    moe::note_launch(cudaMemsetAsync(rs.gcnt, 0, sizeof(int32_t) * moe::dispatch_counter_ints(p->E), s));
     moe::launch_route_place(logits, p->T, p->E, p->k, p->flags, ids, w, rs.gcnt, rs.cand, rs.st,
                             s, launches);
     moe::launch_select(rs.cand, rs.gcnt, w, p->T, p->E, p->k, K, p->flags, rs.bits, slot, drop,
@@ -236,7 +238,7 @@ void* current_context() {
 size_t route_static_layout(const moe_problem* p, size_t* gcnt, size_t* cand, size_t* bits) {
     size_t off = align_up(sizeof(moe::DeviceStatus));
     *gcnt = off;
-    off = align_up(off + (size_t)p->E * 4);
+    off = align_up(off + moe::dispatch_counter_ints(p->E) * 4);
     *cand = off;
     off = align_up(off + (size_t)p->E * p->T * 4);
     *bits = off;
@@ -300,7 +302,7 @@ moe_status moe_route(const moe_problem* p, const float* logits, int32_t* ids, fl
     cudaStream_t s = (cudaStream_t)stream;
     int launches = 0;
     if (p->T == 0) {
-        cudaMemsetAsync(counts, 0, sizeof(int32_t) * 2 * p->E, s);
+        moe::note_launch(cudaMemsetAsync(counts, 0, sizeof(int32_t) * 2 * p->E, s));
         return finish(0);
     }
     route_steps(p, logits, ids, w, slot, drop, counts, nullptr, nullptr, scratch_of(ws, q), s,
@@ -385,7 +387,7 @@ moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, con
     int launches = 0;
     int32_t* counts = counts_out ? counts_out : at<int32_t>(ws, q.counts);
     if (p->T == 0) {
-        cudaMemsetAsync(counts, 0, sizeof(int32_t) * 2 * p->E, s);
+        moe::note_launch(cudaMemsetAsync(counts, 0, sizeof(int32_t) * 2 * p->E, s));
         return finish(0);
     }
     moe::DeviceStatus* st = at<moe::DeviceStatus>(ws, q.status);
@@ -407,13 +409,13 @@ moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, con
     const bool small = p->dtype == MOE_BF16 && moe::router_small_fits(p->T, p->E, p->d_model);
     const bool small_dispatch = moe::dispatch_small_fits(p->T, p->k);
     int32_t* gcnt = small_dispatch ? nullptr : at<int32_t>(ws, q.gcnt);
-    const int zero_n = small_dispatch ? 0 : p->E;
+    const int zero_n = small_dispatch ? 0 : (int)moe::dispatch_counter_ints(p->E);
     if (small) {
         // The large dispatch re-reads the logits: keep them (in the workspace if not asked for).
         moe::launch_router_small(x, Wr, br, p->T, p->d_model, p->E, p->k,
                                  small_dispatch ? logits_out : logits, ids, w, p->flags, s,
                                  &launches);
-        if (!small_dispatch) cudaMemsetAsync(gcnt, 0, sizeof(int32_t) * p->E, s);
+        if (!small_dispatch) moe::note_launch(cudaMemsetAsync(gcnt, 0, sizeof(int32_t) * (size_t)zero_n, s));
     } else if (p->dtype == MOE_BF16) {
         if (moe::launch_router_gemm(x, p->T, p->d_model, Wr, br, p->E, at<void>(ws, q.split),
                                     logits, gcnt, zero_n, st, s, &launches) != cudaSuccess)
@@ -507,6 +509,7 @@ moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, int32_t limit_us
     if (!ws || ws_bytes < sizeof(moe::DeviceStatus) || limit_us < 1 || limit_us > 10000000)
         return MOE_ERR_INVALID_ARG;
     cudaGetLastError();
+    moe::g_launch_error = cudaSuccess;
     moe::launch_wait_timeout_selftest(reinterpret_cast<moe::DeviceStatus*>(ws),
                                       (long long)limit_us * 1000, (cudaStream_t)stream);
     return finish(1);
@@ -555,14 +558,14 @@ extern "C" moe_status moe_route_static(const moe_problem* p, const float* logits
     if (!scratch) return MOE_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
     if (p->T == 0) {
-        cudaMemsetAsync(counts, 0, sizeof(int32_t) * 2 * p->E, s);
+        moe::note_launch(cudaMemsetAsync(counts, 0, sizeof(int32_t) * 2 * p->E, s));
         return finish(0);
     }
     // The array keeps the previous call's contents: the status word must start at zero (the
     // dispatch counters are cleared by route_steps); every other region is fully written by this
     // call before it is read.
     moe::DeviceStatus* st = at<moe::DeviceStatus>(scratch, 0);
-    cudaMemsetAsync(st, 0, sizeof(moe::DeviceStatus), s);
+    moe::note_launch(cudaMemsetAsync(st, 0, sizeof(moe::DeviceStatus), s));
     int launches = 0;
     const RouteScratch rs{st, at<int32_t>(scratch, o_gcnt), at<int32_t>(scratch, o_cand),
                           moe::select_bits_bytes(p->T, p->E) ? at<uint32_t>(scratch, o_bits)

@@ -150,11 +150,19 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
 // per (block, expert)).
 constexpr int kGroupBlockTokens = 64;
 
+// Per-expert histogram of the weight keys, built while routing: bin = bits 29..19 of the fp32
+// weight (weights are in [0, 1], so bit 30 is 0 and the bin grows with the weight: 7 exponent
+// bits and the top 4 mantissa bits).
+constexpr int kHistBins = 2048;
+__device__ __forceinline__ int hist_bin(float wv) {
+    return (int)min(__float_as_uint(wv) >> 19, (uint32_t)(kHistBins - 1));
+}
+
 template <int G>
 __global__ void __launch_bounds__(256) route_place_group_kernel(
     const float* __restrict__ logits, int T, int E, int k, unsigned flags,
     int32_t* __restrict__ ids, float* __restrict__ w, int32_t* __restrict__ gcnt,
-    int32_t* __restrict__ cand, DeviceStatus* st) {
+    int32_t* __restrict__ cand, uint32_t* __restrict__ hist, DeviceStatus* st) {
     pdl_begin();
     constexpr int LPL = 32 / G;                        // warp-router lanes per group lane
     constexpr int NI = G / 4;                          // experts per warp-router lane: E <= 32 NI
@@ -219,21 +227,39 @@ __global__ void __launch_bounds__(256) route_place_group_kernel(
             }
         }
         const float S = __shfl_sync(kFull, p[0], 0, G);
-        uint32_t taken = 0;                            // bit li * NI + i
+        // Top-k: each lane sorts its candidates once by (logit desc, expert asc), invalid ones
+        // (e >= E) last; each round the group takes the best head and its owner pops it.
+        constexpr int NC = LPL * NI;
+        float cl[NC];
+        int ce[NC];
+#pragma unroll
+        for (int li = 0; li < LPL; ++li)
+#pragma unroll
+            for (int i = 0; i < NI; ++i) {
+                const int e = q * LPL + li + 32 * i;
+                cl[li * NI + i] = e < E ? v[li][i] : 0.0f;
+                ce[li * NI + i] = e < E ? e : 0x7fffffff;
+            }
+        // Odd-even transposition sort (NC rounds of neighbour compare-exchange).
+#pragma unroll
+        for (int rnd = 0; rnd < NC; ++rnd)
+#pragma unroll
+            for (int a = rnd & 1; a + 1 < NC; a += 2) {
+                const bool sw = ce[a + 1] != 0x7fffffff &&
+                                (ce[a] == 0x7fffffff || cl[a + 1] > cl[a] ||
+                                 (cl[a + 1] == cl[a] && ce[a + 1] < ce[a]));
+                const float tl = sw ? cl[a + 1] : cl[a];
+                const int te = sw ? ce[a + 1] : ce[a];
+                cl[a + 1] = sw ? cl[a] : cl[a + 1];
+                ce[a + 1] = sw ? ce[a] : ce[a + 1];
+                cl[a] = tl;
+                ce[a] = te;
+            }
+        float my_l = 0.0f;
         int id_j = 0;
-        float w_j = 0.0f, wsum = 0.0f;
         for (int j = 0; j < k; ++j) {
-            float bl = 0.0f;
-            int be = 0x7fffffff, bb = -1;
-#pragma unroll
-            for (int li = 0; li < LPL; ++li)
-#pragma unroll
-                for (int i = 0; i < NI; ++i) {
-                    const int e = q * LPL + li + 32 * i;
-                    const bool ok = e < E && !((taken >> (li * NI + i)) & 1u) &&
-                                    (bb < 0 || v[li][i] > bl || (v[li][i] == bl && e < be));
-                    if (ok) { bl = v[li][i]; be = e; bb = li * NI + i; }
-                }
+            float bl = cl[0];
+            int be = ce[0];
 #pragma unroll
             for (int o = G / 2; o >= 1; o >>= 1) {
                 const float yl = __shfl_xor_sync(kFull, bl, o, G);
@@ -243,17 +269,28 @@ __global__ void __launch_bounds__(256) route_place_group_kernel(
                     be = ye;
                 }
             }
-            if (bb >= 0 && q * LPL + bb / NI + 32 * (bb % NI) == be) taken |= 1u << bb;
-            const float wj = __fdiv_rn(exp_cody_waite(__fsub_rn(bl, m)), S);
-            wsum = __fadd_rn(wsum, wj);
-            if (q == j) { id_j = be; w_j = wj; }
+            if (ce[0] == be) {                         // the owner pops its head
+#pragma unroll
+                for (int a = 0; a + 1 < NC; ++a) { cl[a] = cl[a + 1]; ce[a] = ce[a + 1]; }
+                cl[NC - 1] = 0.0f;
+                ce[NC - 1] = 0x7fffffff;
+            }
+            if (q == j) { id_j = be; my_l = bl; }
         }
+        // Lane j < k forms weight j: w = exp(L - m) / S; the renormalised form divides by the sum
+        // of the k weights added in j order.
+        const float w_j = __fdiv_rn(exp_cody_waite(__fsub_rn(my_l, m)), S);
+        float wsum = 0.0f;
+        if (flags & MOE_FLAG_RENORMALIZE)
+            for (int j = 0; j < k; ++j) wsum = __fadd_rn(wsum, __shfl_sync(kFull, w_j, j, G));
         if (active && q < k) {
             const size_t pj = (size_t)t * k + q;
+            const float wf = (flags & MOE_FLAG_RENORMALIZE) ? __fdiv_rn(w_j, wsum) : w_j;
             ids[pj] = id_j;
-            w[pj] = (flags & MOE_FLAG_RENORMALIZE) ? __fdiv_rn(w_j, wsum) : w_j;
+            w[pj] = wf;
             my_e[r] = id_j;
             my_pos[r] = atomicAdd(&s_n[id_j], 1);
+            if (hist) atomicAdd(&hist[(size_t)id_j * kHistBins + hist_bin(wf)], 1u);
         }
     }
     __syncthreads();
@@ -277,7 +314,7 @@ template <int EPL>
 __global__ void __launch_bounds__(256) route_place_warp_kernel(
     const float* __restrict__ logits, int T, int E, int k, unsigned flags,
     int32_t* __restrict__ ids, float* __restrict__ w, int32_t* __restrict__ gcnt,
-    int32_t* __restrict__ cand, DeviceStatus* st) {
+    int32_t* __restrict__ cand, uint32_t* __restrict__ hist, DeviceStatus* st) {
     pdl_begin();
     extern __shared__ int s_nb[];                       // [E] counts, then [E] bases
     int* s_n = s_nb;
@@ -294,7 +331,12 @@ __global__ void __launch_bounds__(256) route_place_warp_kernel(
         const int t = t0 + i;
         if (t < T) {
             my_e[i] = route_token_warp<EPL>(logits + (size_t)t * E, E, k, (size_t)t, ids, w, flags);
-            if (my_e[i] >= 0) my_pos[i] = atomicAdd(&s_n[my_e[i]], 1);
+            if (my_e[i] >= 0) {
+                my_pos[i] = atomicAdd(&s_n[my_e[i]], 1);
+                if (hist)
+                    atomicAdd(&hist[(size_t)my_e[i] * kHistBins + hist_bin(w[(size_t)t * k + lane])],
+                              1u);
+            }
         }
     }
     __syncthreads();
@@ -313,7 +355,8 @@ __global__ void __launch_bounds__(256) route_place_warp_kernel(
 // Capacity selection from unordered candidate lists: one block per expert.
 // ---------------------------------------------------------------------------------------------
 constexpr int kSelThreads = 1024;
-constexpr int kSelSmem = 220 * 1024;  // dynamic shared memory of the selection kernel
+constexpr int kSelSmem = 200 * 1024;  // dynamic shared memory of the selection kernel (the
+                                      // static arrays take about 9 KB more)
 constexpr int kSelBitWords = 8192;    // token-bitmap words kept on chip (T <= 262144)
 
 // Radix select over the keys of candidates i < n (most significant byte first), restricted to
@@ -389,12 +432,15 @@ __device__ __forceinline__ uint32_t radix_select(int n, int want, KeyFn key_of, 
 __global__ void __launch_bounds__(kSelThreads) select_kernel(
     const int32_t* __restrict__ cand, const int32_t* __restrict__ gcnt,
     const float* __restrict__ w, int T, int E, int k, long long K, unsigned flags,
-    uint32_t* __restrict__ gbits, int keys_cap, int32_t* __restrict__ slot,
-    uint8_t* __restrict__ drop, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-    int32_t* __restrict__ rowtok, DeviceStatus* st) {
+    uint32_t* __restrict__ gbits, int keys_cap, const uint32_t* __restrict__ hist,
+    int32_t* __restrict__ slot, uint8_t* __restrict__ drop, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ rowtok, DeviceStatus* st) {
     pdl_begin();
     extern __shared__ uint32_t s_dyn[];
     __shared__ int s_warp[32];
+    __shared__ uint32_t s_tk[kSelThreads];    // tie bin: keys and pair indices
+    __shared__ int32_t s_tp[kSelThreads];
+    __shared__ int s_nt, s_bstar, s_need, s_found;
     __shared__ int s_hist[256];
     __shared__ uint32_t s_prefix;
     __shared__ int s_rem;
@@ -435,13 +481,26 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     auto key_from = [&](int32_t p) -> uint32_t {
         return arrival ? ~(uint32_t)p : __float_as_uint(w[p]);
     };
-    if (on_chip)
-        for (int i = tid; i < n; i += blockDim.x) {
-            int32_t p = list[i];
-            if (p < 0 || p >= P) { report(st, MOE_DEV_BAD_INDEX, 122); p = -1; }
-            s_list[i] = p;
-            s_keys[i] = p < 0 ? 0u : key_from(p);
+    if (on_chip) {
+        // Four candidates per thread in flight: their list entries, then their weights.
+        for (int i0 = 0; i0 < n; i0 += 4 * kSelThreads) {
+            int32_t pv[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int i = i0 + b * kSelThreads + tid;
+                pv[b] = i < n ? list[i] : -1;
+            }
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int i = i0 + b * kSelThreads + tid;
+                if (i >= n) continue;
+                int32_t p = pv[b];
+                if (p < 0 || p >= P) { report(st, MOE_DEV_BAD_INDEX, 122); p = -1; }
+                s_list[i] = p;
+                s_keys[i] = p < 0 ? 0u : key_from(p);
+            }
         }
+    }
     for (int i = tid; i < nw; i += blockDim.x) bits[i] = 0;
     __syncthreads();
     auto key_of = [&](int i) -> uint32_t {
@@ -457,7 +516,63 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     uint32_t tau = 0;                 // keys > tau are kept; keys == tau when pair <= p_tau
     int32_t p_tau = 0x7fffffff;
     bool select_all = n <= K;
-    if (!select_all && K > 0) {
+    bool by_hist = false;
+    int bstar = 0;
+    if (!select_all && K > 0 && hist && !arrival) {
+        // Threshold bin from the histogram: thread t holds bins 2047 - 2t and 2046 - 2t (top
+        // down); b* is the bin where the count from the top reaches K.  Keys above b* are kept,
+        // below dropped; the `need` largest (ties: lower pair) of bin b* are kept.  Any
+        // inconsistency (histogram total != n, a tie bin larger than one key per thread) falls
+        // back to the radix selection below.
+        const uint32_t* h = hist + (size_t)e * kHistBins;
+        const int b_hi = kHistBins - 1 - 2 * tid, b_lo = b_hi - 1;
+        const int c_hi = (int)h[b_hi], c_lo = (int)h[b_lo];
+        if (tid == 0) { s_nt = 0; s_bstar = -1; s_found = 0; }
+        int tot;
+        const int above = block_exclusive_scan(c_hi + c_lo, s_warp, &tot);
+        if (above < K && above + c_hi >= K) {
+            s_bstar = b_hi;
+            s_need = (int)(K - above);
+        } else if (above + c_hi < K && above + c_hi + c_lo >= K) {
+            s_bstar = b_lo;
+            s_need = (int)(K - above - c_hi);
+        }
+        __syncthreads();
+        bstar = s_bstar;
+        const int need = s_need;
+        const int mt = bstar >= 0 ? (int)h[bstar] : kSelThreads + 1;
+        if (tot == n && mt <= kSelThreads) {
+            for (int i = tid; i < n; i += blockDim.x) {
+                if (!valid(i)) continue;
+                const uint32_t key = key_of(i);
+                if ((int)min(key >> 19, (uint32_t)(kHistBins - 1)) == bstar) {
+                    const int at = atomicAdd(&s_nt, 1);
+                    if (at < kSelThreads) { s_tk[at] = key; s_tp[at] = pair_of(i); }
+                }
+            }
+            __syncthreads();
+            const int m = s_nt;
+            // Rank of each tied candidate by (key desc, pair asc); the need-th one bounds the
+            // kept set: key > tau, or key == tau and pair <= p_tau.
+            if (m == mt && tid < m) {
+                const uint32_t kt = s_tk[tid];
+                const int32_t pt = s_tp[tid];
+                int rank = 0;
+                for (int j = 0; j < m; ++j) {
+                    const uint32_t kj = s_tk[j];
+                    rank += (kj > kt || (kj == kt && s_tp[j] < pt)) ? 1 : 0;
+                }
+                if (rank == need - 1) { s_prefix = kt; s_rem = pt; s_found = 1; }
+            }
+            __syncthreads();
+            if (s_found) {
+                by_hist = true;
+                tau = s_prefix;
+                p_tau = s_rem;
+            }
+        }
+    }
+    if (!select_all && K > 0 && !by_hist) {
         int need_eq;
         tau = radix_select(n, (int)K, key_of, valid, s_hist, &s_prefix, &s_rem, &need_eq);
         // Candidates equal to tau: are all of them among the K largest?  Count them.
@@ -474,7 +589,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
                 &s_rem, &dummy);
         }
     }
-    // Mark kept tokens.
+    // Mark kept tokens.  (With the histogram, tau lies in bin b*: keys in higher bins are above
+    // tau and keys in lower bins below it, so the same rule holds.)
     for (int i = tid; i < n; i += blockDim.x) {
         if (!valid(i)) continue;
         const int32_t p = pair_of(i);
@@ -788,44 +904,49 @@ int route_group_lanes(int E, int k) {
     return (G > 0 && k <= G) ? G : 0;
 }
 
+size_t dispatch_counter_ints(int E) { return (size_t)E * (1 + kHistBins); }
+
 void launch_route_place(const float* logits, int T, int E, int k, unsigned flags, int32_t* ids,
                         float* w, int32_t* gcnt, int32_t* cand, DeviceStatus* st, cudaStream_t s,
                         int* launches) {
+    // The histogram follows the counters; arrival-order selection does not use it.
+    uint32_t* hist = (flags & MOE_FLAG_ARRIVAL_ORDER) ? nullptr
+                                                      : reinterpret_cast<uint32_t*>(gcnt + E);
     if (T == 0) return;
     const int G = route_group_lanes(E, k);
     if (G > 0) {
         const dim3 g((T + kGroupBlockTokens - 1) / kGroupBlockTokens);
         if (G == 8)
             launch_pdl(route_place_group_kernel<8>, g, dim3(256), 0, s, logits, T, E, k, flags,
-                       ids, w, gcnt, cand, st);
+                       ids, w, gcnt, cand, hist, st);
         else if (G == 16)
             launch_pdl(route_place_group_kernel<16>, g, dim3(256), 0, s, logits, T, E, k, flags,
-                       ids, w, gcnt, cand, st);
+                       ids, w, gcnt, cand, hist, st);
         else
             launch_pdl(route_place_group_kernel<32>, g, dim3(256), 0, s, logits, T, E, k, flags,
-                       ids, w, gcnt, cand, st);
+                       ids, w, gcnt, cand, hist, st);
     } else {
         const dim3 g((T + kWarpRouteTokens - 1) / kWarpRouteTokens);
         const size_t smem = 2 * sizeof(int) * (size_t)E;
         const int epl = (E + 31) / 32;
         if (epl <= 1)
             launch_pdl(route_place_warp_kernel<1>, g, dim3(256), smem, s, logits, T, E, k, flags,
-                       ids, w, gcnt, cand, st);
+                       ids, w, gcnt, cand, hist, st);
         else if (epl <= 2)
             launch_pdl(route_place_warp_kernel<2>, g, dim3(256), smem, s, logits, T, E, k, flags,
-                       ids, w, gcnt, cand, st);
+                       ids, w, gcnt, cand, hist, st);
         else if (epl <= 4)
             launch_pdl(route_place_warp_kernel<4>, g, dim3(256), smem, s, logits, T, E, k, flags,
-                       ids, w, gcnt, cand, st);
+                       ids, w, gcnt, cand, hist, st);
         else if (epl <= 8)
             launch_pdl(route_place_warp_kernel<8>, g, dim3(256), smem, s, logits, T, E, k, flags,
-                       ids, w, gcnt, cand, st);
+                       ids, w, gcnt, cand, hist, st);
         else if (epl <= 16)
             launch_pdl(route_place_warp_kernel<16>, g, dim3(256), smem, s, logits, T, E, k, flags,
-                       ids, w, gcnt, cand, st);
+                       ids, w, gcnt, cand, hist, st);
         else
             launch_pdl(route_place_warp_kernel<32>, g, dim3(256), smem, s, logits, T, E, k, flags,
-                       ids, w, gcnt, cand, st);
+                       ids, w, gcnt, cand, hist, st);
     }
     *launches += 1;
 }
@@ -854,9 +975,12 @@ void launch_select(const int32_t* cand, const int32_t* gcnt, const float* w, int
         cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelSmem);
         attr_done.fetch_or(bit);
     }
+    const uint32_t* hist = (flags & MOE_FLAG_ARRIVAL_ORDER)
+                               ? nullptr
+                               : reinterpret_cast<const uint32_t*>(gcnt + E);
     launch_pdl(select_kernel, dim3(E), dim3(kSelThreads), smem, s, cand, gcnt, w, T, E, k, K,
-               flags, bits_on_chip ? nullptr : gbits, keys_cap, slot, drop, counts, offsets, rowtok,
-               st);
+               flags, bits_on_chip ? nullptr : gbits, keys_cap, hist, slot, drop, counts, offsets,
+               rowtok, st);
     *launches += 1;
 }
 
@@ -865,7 +989,7 @@ void launch_dispatch(const int32_t* ids, const int32_t* slot, int T, int E, int 
                      cudaStream_t s, int* launches) {
     const long long P = (long long)T * k;
     const int blocks = (int)std::min<long long>((P + 255) / 256, 148 * 8);
-    cudaMemsetAsync(kept_tmp, 0, sizeof(int32_t) * E, s);
+    note_launch(cudaMemsetAsync(kept_tmp, 0, sizeof(int32_t) * E, s));
     if (P > 0) launch_pdl(kept_count_kernel, dim3(blocks), dim3(256), 0, s, ids, slot, P, E, T,
                           kept_tmp, st);
     launch_pdl(offsets_kernel, dim3(1), dim3(1024), 0, s, kept_tmp, E, offsets);

@@ -85,6 +85,16 @@ def test_route_weight_ties():
     _assert_route_equal(g, ro, 12)
 
 
+def test_route_tie_bin_larger_than_a_block():
+    # Every token has the same logits: one expert receives all 3000 pairs with the same weight,
+    # more than one block of equal keys at the capacity boundary; the lower tokens are kept.
+    T, E, k = 3000, 2, 1
+    L = np.zeros((T, E), np.float32)
+    _, g, ro = _route_both(L, T, E, k, 0.5)
+    _assert_route_equal(g, ro, E)
+    assert ro["kept"][0] == 750 and (ro["slot"][:750, 0] == np.arange(750)).all()
+
+
 def test_route_large_batch_global_bitmap():
     # More than 262144 tokens: the capacity selection keeps its token bitmap in the workspace.
     T, E, k = 300000, 4, 2
