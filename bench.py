@@ -415,13 +415,13 @@ def run_cuda(args):
     gemm_flop_each = 2.0 * kept * dm * F
     g1_flop = gemm_flop_each * (2 if spec.gated else 1)
     # Algorithmic work per stage (the method's, not the implementation's): the router's flops
-    # are 2 T d E; bytes count every input read once and every output written once.  With the
-    # routing fused into the logits GEMM (bf16, E <= 64, T > 1024) the router stage reads x and
-    # Wr and writes ids, weights and per-chunk counts, and the separate top-k stage is empty;
-    # otherwise the logits round-trip through HBM between the two stages.
-    n_chunks = (T + 31) // 32
-    fused = spec.dtype == "bf16" and E <= 64 and T > 1024
-    router_out = T * k * 8 + E * n_chunks * 4 if fused else T * E * 4
+    # are 2 T d E; bytes count every input read once and every output written once.  Small bf16
+    # batches with the single-block dispatch (T <= 1024, T k <= 1024) compute logits and routing
+    # in one launch: the router stage reads x and Wr and writes ids and weights, and the top-k
+    # stage is empty.  Otherwise the logits round-trip through HBM between the two stages.
+    fused = (spec.dtype == "bf16" and T <= 1024 and E <= 256 and dm <= 12288
+             and T * k <= 1024)
+    router_out = T * k * 8 if fused else T * E * 4
     by = {
         "router_logits": dict(flop=2.0 * T * dm * E, bytes=T * dm * esz + dm * E * 4 + router_out),
         "route_topk": dict(bytes=0 if fused else T * E * 4 + T * k * 8),

@@ -1,24 +1,28 @@
 // route.cu -- router softmax/top-k and capacity-limited dispatch (sm_100a).
 //
-// Step 1, router ("Dynamic Token Routing AI", How it works): one warp per token computes the
-// softmax of its E logits in fp32 and keeps the k largest in registers.
+// Step 1, router ("Dynamic Token Routing AI", How it works): a warp, or a group of lanes, per
+// token computes the softmax of its E logits in fp32 and keeps the k largest in registers.
 // Step 2, capacity ("Expert Networks > Worked Example: Expert Specialization", capacity
 // paragraph; "Some Tokens Do Not Get In", "Why there is a buffer" / "Past the edge"): each
 // expert keeps at most K pairs, those with the highest router weight (ties: lower token), and
 // the slot of a kept pair is its rank among the expert's kept tokens in ascending token order.
 //
 // Dispatch, two launches, deterministic (no result depends on the order of atomics):
-//   route + place: the router (one thread per token for E <= 64 and k <= 8, one warp per token
-//            otherwise) also appends every (token, expert) pair to its expert's candidate list
-//            cand[e][.]; positions come from per-block counters in shared memory plus one global
-//            atomic per (block, expert) on gcnt[e].  The order inside a list is arbitrary.
-//   select : one block per expert; if n_e > K a 4-pass radix select on the fp32 weight bits
-//            finds the K-th largest weight (ties at the boundary: lower token first, by a second
-//            radix select on the pair index); the kept tokens are marked in a bitmap over the
-//            batch, whose prefix popcounts give each kept pair its slot (its rank in token
-//            order), so the result does not depend on the list order.
-// gcnt must be zero when the route kernel starts; the kernel before it in the same call clears
-// it (the router GEMM, the fp32 logits kernel, or a memset in moe_route).
+//   route + place: the router (a group of 8, 16 or 32 lanes per token for E <= 64, 128, 256 and
+//            k <= the group, one warp per token otherwise) also appends every (token, expert)
+//            pair to its expert's candidate list cand[e][.] and counts its weight in a
+//            2048-bin histogram of the expert's weights; list positions come from per-block
+//            counters in shared memory plus one global atomic per (block, expert) on gcnt[e].
+//            The order inside a list is arbitrary.
+//   select : one block per expert; if n_e > K the histogram gives the bin that holds the K-th
+//            largest weight, and ranking that bin's candidates (ties: lower token first) gives
+//            the exact boundary; a radix select on the weight bits covers the cases the
+//            histogram cannot (arrival order, a bin of more than 1024 candidates).  The kept
+//            tokens are marked in a bitmap over the batch, whose prefix popcounts give each kept
+//            pair its slot (its rank in token order), so the result does not depend on the list
+//            order.
+// The counters and histograms must be zero when the route kernel starts; the kernel before it
+// in the same call clears them (the router's weight split, the fp32 logits kernel, or a memset).
 #include <atomic>
 #include <cfloat>
 #include <cstdint>

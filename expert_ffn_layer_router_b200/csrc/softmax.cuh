@@ -1,5 +1,5 @@
-// softmax.cuh -- the router's fp32 arithmetic, shared by the warp-per-token router (route.cu)
-// and the fused router epilogue of the logits GEMM (gemm_tc.cu), so both form bit-identical
+// softmax.cuh -- the router's fp32 arithmetic, shared by the routers of route.cu (warp per
+// token, group of lanes per token, the small-batch router), so all of them form bit-identical
 // weights from the same logits.
 //
 // One token is routed by one warp: lane l holds experts l, l+32, ...; the softmax sum adds the

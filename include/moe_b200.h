@@ -179,9 +179,9 @@ moe_status moe_set_stage_events(void* const* events, int32_t n);
  *   Same arguments, outputs and results as moe_route (bit for bit), minus ws/ws_bytes.  The
  *   router/capacity scratch lives in one fixed 8 MiB array of device memory per GPU, part of the
  *   library image and held by every GPU that loads the library until the process exits.  Needs
- *   16 + 8*E*ceil(T/32) + 4*E + 4*E*T bytes (each part rounded up to 256); larger problems get
- *   MOE_ERR_WORKSPACE before anything is launched (T=16384 with E=64 fits; T=65536 with E=128
- *   does not).
+ *   256 + 4*E*2049 + 4*E*T bytes (each part rounded up to 256; above T = 262144 tokens also
+ *   8*E*ceil(T/32) for the selection's token bitmaps); larger problems get MOE_ERR_WORKSPACE
+ *   before anything is launched (T=16384 with E=64 fits; T=65536 with E=128 does not).
  *   The first call in a CUDA context (for runtime-API callers: the first call on a device) looks
  *   up the array's device address in that context and caches it; make that first call before
  *   any stream capture.  The cached address dies with its context: do not call it across a

@@ -1,10 +1,13 @@
-"""The fused forward at the workloads' full sizes, in the configuration the bench times.
+"""The whole forward (moe_forward) at the workloads' full sizes, in the configuration the bench
+times.
 
-Routing is compared in full (expert ids exactly; capacity decisions exactly except where the
-oracle's own weights tie within the logit error at an expert's capacity boundary); outputs on a
-seeded sample of tokens (random tokens plus partially and fully dropped ones), since each
-token's output depends only on its own row given the routing.  Fully dropped tokens must come
-out bit for bit equal to their input.
+Routing is compared in full and bit for bit with the oracle's routing of the fp32 logits the
+forward exported (ids, weight bits, slots, drops, counts); outputs on a seeded sample of tokens
+(random tokens plus partially and fully dropped ones), since each token's output depends only
+on its own row given the routing.  Fully dropped tokens must come out bit for bit equal to their
+input.  A second, looser comparison routes the oracle's own float64 logits: expert sets exactly,
+capacity decisions exactly except where the oracle's weights tie within the logit error at a
+capacity boundary.
 """
 import numpy as np
 import pytest

@@ -205,7 +205,7 @@ def test_combine_parity(T, d, E, k, C, dtype):
 
 
 # ------------------------------------------------------------------------------------------
-# The fused forward against the oracle's whole layer.
+# The whole forward against the oracle's whole layer.
 # ------------------------------------------------------------------------------------------
 def _assert_forward_route_equal(g, ro, E):
     """The forward's exported routing against the oracle's routing of the same fp32 logits."""
@@ -317,17 +317,17 @@ def test_unsupported_and_invalid():
 
 
 # ------------------------------------------------------------------------------------------
-# Fused router: with bf16 and E <= 64 the logits GEMM's epilogue also forms the softmax, the
-# top-k and the per-chunk counts.  Its routing must equal, bit for bit, both moe_route's and the
-# oracle's routing of the logits the forward exported.
+# The forward's routing (the router that also places the pairs in candidate lists, then the
+# histogram-based capacity selection; or the small-batch router and dispatch) must equal, bit
+# for bit, both moe_route's and the oracle's routing of the logits the forward exported.
 # ------------------------------------------------------------------------------------------
 @pytest.mark.parametrize("T,d,E,k,C", [(3000, 128, 64, 6, 1.0), (1000, 256, 8, 2, 1.25),
                                        (777, 64, 33, 4, 0.75), (200, 64, 16, 8, math.inf),
                                        (5000, 64, 64, 6, 0.5), (129, 64, 1, 1, 1.0)])
 @pytest.mark.parametrize("flags", [0, 1, 3])
-def test_fused_router_matches_route(T, d, E, k, C, flags):
+def test_forward_routing_matches_route(T, d, E, k, C, flags):
     moe = _moe()
-    spec = inputs.LayerSpec("fused", T, d, 64, E, k, C, "bf16", router="normal",
+    spec = inputs.LayerSpec("fwd_route", T, d, 64, E, k, C, "bf16", router="normal",
                             router_bias=0.5)
     L = inputs.make_layer(spec, seed=E + T)
     layer = moe.MoELayer(T, d, 64, E, k, C, "bf16", flags=flags)

@@ -438,7 +438,7 @@ def test_combine_given_y_detects_float_accumulation():
 
 def test_combine_given_y_agrees_with_combine_tokens():
     # Expert outputs from the oracle's own FFN rows (pinned against torch float64 above), then
-    # the standalone combine: the same layer output as the fused oracle path.
+    # the standalone combine: the same layer output as the oracle's whole-layer path.
     spec = inputs.LayerSpec("cg", 48, 16, 24, 6, 2, 0.6, "f32", router="normal",
                             router_bias=0.3, bias_std=0.1)
     layer = inputs.make_layer(spec, seed=3)
