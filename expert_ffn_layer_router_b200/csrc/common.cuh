@@ -186,15 +186,24 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
 }
 
 // ---------------------------------------------------------------------------------------------
-// Programmatic dependent launch.  Every kernel starts with pdl_begin(): it waits until the
+// Programmatic dependent launch.  Most kernels start with pdl_begin(): it waits until the
 // preceding grid in the stream has completed and its memory is visible (a no-op without a
 // programmatic dependency), then lets the next grid be scheduled, whose blocks in turn park in
-// their own wait.  So no kernel touches global memory before its predecessor is done, and a
-// dependent launch overlaps only its scheduling and set-up with the tail of the previous grid.
+// their own wait.  A dependent grid is scheduled only once every block of this grid has
+// triggered, so all of them are resident by then and a waiting dependent cannot starve them.
+// No kernel reads memory that a predecessor writes, or writes any memory, before its wait.
+// Kernels whose set-up needs nothing from their predecessors split the two steps: the
+// small-batch router and dispatch trigger first, so the expert GEMM can be scheduled early; a
+// weight-streaming GEMM does its set-up (barriers, tensor memory, an L2 prefetch of its weights,
+// which are read but never written by the call) before it waits.
 // ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ void pdl_begin() {
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_begin() {
+    pdl_wait();
+    pdl_trigger();
 }
 
 // The first failed launch (or stream operation) of the current API call on this host thread; the

@@ -70,20 +70,30 @@ struct GemmArgs {
     long long ldd;            // elements
     int router_E;             // router epilogue: number of experts (columns of D)
     DeviceStatus* st;
+    const void* W;            // B's base address (the L2 prefetch below)
+    long long pf_bytes;       // > 0: before waiting for its predecessor, each CTA prefetches up
+                              // to this many bytes of its first tile's weight rows into L2
 };
 
 // PAIR: two CTAs of a cluster share one 256-row tile; each holds its 128 A rows and half of the
 // BN B rows in shared memory, the pair's tensor cores compute the 256 x BN product together.
 // The router epilogue (BN = 2 Eg: hi and mid columns of Eg experts) stages the tile's logits in a
 // padded [128][Eg + 1] fp32 array instead of the bf16 staging buffers.
-template <int BN, bool PAIR, int EPI>
+//
+// HALFM (weight streaming, single CTAs): m-tiles of 64 rows.  The MMAs stay M = 128; A stages are
+// 8 KB apart and each MMA reads 16 KB from its stage, so rows 64-127 of the product come from the
+// next stage (or, for the last A stage, from the first B stage) and are never stored.  Halving
+// the A stages leaves room for more weight stages in flight.
+template <int BN, bool PAIR, int EPI, bool HALFM = false>
 struct Cfg {
     static constexpr bool kRouter = EPI == kEpiRouter;
     static constexpr int kEg = BN / 2;
     static constexpr int kLStride = kEg + 1;                      // floats per staged logits row
-    static constexpr int kTileM = PAIR ? 256 : 128;
+    static constexpr int kTileM = PAIR ? 256 : (HALFM ? 64 : 128);
+    static constexpr int kCtaRows = HALFM ? 64 : 128;             // A rows of one CTA's tile
+    static constexpr int kMmaM = PAIR ? 256 : 128;
     static constexpr int kBRows = PAIR ? BN / 2 : BN;          // B rows held by this CTA
-    static constexpr int kABytes = kBM * kBK * 2;                // 16 KB
+    static constexpr int kABytes = kCtaRows * kBK * 2;           // 16 KB (8 KB with HALFM)
     static constexpr int kBBytes = kBRows * kBK * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStageBudget = (kRouter ? 168 : 200) * 1024;
@@ -100,6 +110,9 @@ struct Cfg {
     static_assert(8 * (3 * kStages + 4) + 4 <= 512, "barrier area");
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
     static_assert(kStgBytes % 8 == 0, "barriers stay 8-byte aligned");
+    static_assert(!HALFM || (!PAIR && !kRouter), "64-row tiles: single-CTA FFN GEMMs only");
+    // With HALFM the MMA of the last A stage reads 8 KB past the A stages: inside B stage 0.
+    static_assert(!HALFM || kBBytes >= 8192, "the last A stage's read stays in shared memory");
 };
 
 __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c,
@@ -249,7 +262,7 @@ struct TileCoord {
     int e, row0, rows, nt;
 };
 
-template <int kTileM>
+template <int kTileM, int kCtaRows>
 __device__ __forceinline__ TileCoord tile_coord(int tile, const int* s_mt, int E, int n_tiles,
                                                 const GemmArgs& a, int half) {
     TileCoord c;
@@ -263,8 +276,8 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, const int* s_mt, int E
     c.e = lo;
     const int g0 = a.offsets ? __ldg(a.offsets + lo) : 0;
     const int g1 = a.offsets ? __ldg(a.offsets + lo + 1) : a.rows0;
-    c.row0 = g0 + (mt - s_mt[lo]) * kTileM + half * kBM;
-    c.rows = min(kBM, g1 - c.row0);         // <= 0: this CTA's half of the tile is empty
+    c.row0 = g0 + (mt - s_mt[lo]) * kTileM + half * kCtaRows;
+    c.rows = min(kCtaRows, g1 - c.row0);    // <= 0: this CTA's half of the tile is empty
     return c;
 }
 
@@ -294,13 +307,16 @@ __device__ __forceinline__ void router_tile(const float* sL, int LS, int Eg, con
     named_bar(2, kRouteWarps * 32);
 }
 
-template <int BN, int EPI, bool GATHER, bool PAIR>
+template <int BN, int EPI, bool GATHER, bool PAIR, bool HALFM>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmD, const GemmArgs args) {
-    pdl_begin();
-    using C = Cfg<BN, PAIR, EPI>;
+    // Weight-streaming kernels do their set-up (and an L2 prefetch of their weights) before
+    // waiting for the previous kernel; the others wait first.  (Measured on B200: moving the wait,
+    // or adding the prefetch branch, in the compute-bound kernels slowed them by 2%.)
+    if constexpr (!HALFM) pdl_begin();
+    using C = Cfg<BN, PAIR, EPI, HALFM>;
     constexpr int S = C::kStages;
     constexpr int TM = C::kTileM;
     extern __shared__ uint8_t smem_raw[];
@@ -355,6 +371,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_relinquish();
         }
     }
+    if constexpr (HALFM) {
+        if (args.pf_bytes > 0 && warp == 3) {
+            // Weight streaming (few rows per group): start reading this CTA's first weight tile
+            // into L2 while the kernels before it still run, its first k-blocks for all of the
+            // tile's rows (the boxes the producer loads first).  The tile is the one a schedule
+            // of one m-tile per group gives (tile = group * n_tiles + column tile), which is exact
+            // when every group has 1 to TM rows; otherwise some prefetched bytes go unused.
+            const int e = cid / args.n_tiles, nt = cid % args.n_tiles;
+            if (e < E) {
+                const int brow = e * args.b_rows_per_group + nt * BN;
+                const int nkb_pf =
+                    (int)min((long long)(args.K / kBK), args.pf_bytes / C::kBBytes);
+                for (int kb = lane; kb < nkb_pf; kb += 32)
+                    asm volatile(
+                        "cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+                        ::"l"(&tmB), "r"(kb * kBK), "r"(brow) : "memory");
+            }
+        }
+        // Nothing above reads memory that a predecessor writes.
+        pdl_wait();
+        pdl_trigger();
+    }
     if (warp == 2) {
         // Tile prefix over groups: lane l sums groups [l*per, (l+1)*per).  Row ranges given by
         // the caller are checked first: offsets[0] = 0, non-decreasing, offsets[E] <= max_rows,
@@ -402,12 +440,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_tiles = args.n_tiles;
     const int total = s_mt[E] * n_tiles;
     const int nkb = args.K / kBK;
-    constexpr uint32_t kIdesc = idesc_bf16(TM, BN);
+    constexpr uint32_t kIdesc = idesc_bf16(C::kMmaM, BN);
     // A last column tile with at most BN/2 valid columns (d_ff = 1408 on 256-wide tiles) runs
     // N = BN/2 MMAs: the padded half is neither multiplied nor read back.  On pairs each CTA then
     // supplies BN/4 of the tile's weight rows (the first BN/4 rows of its B stage).
     constexpr bool kHalfOk = (EPI == kEpiSiLU || EPI == kEpiBias) && (BN / 2) % 16 == 0;
-    constexpr uint32_t kIdescHalf = idesc_bf16(TM, kHalfOk ? BN / 2 : BN);
+    constexpr uint32_t kIdescHalf = idesc_bf16(C::kMmaM, kHalfOk ? BN / 2 : BN);
     const bool last_half = kHalfOk && (n_tiles * BN - args.Nout) >= BN / 2;
     // Barriers of the pair's leader that both CTAs signal.
     auto lead = [&](uint32_t addr) { return PAIR ? map_to_cta(addr, 0) : addr; };
@@ -420,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int tile = cid; ok && tile < total; tile += ncl) {
-                const TileCoord tc = tile_coord<TM>(tile, s_mt, E, n_tiles, args, (int)crank);
+                const TileCoord tc = tile_coord<TM, C::kCtaRows>(tile, s_mt, E, n_tiles, args, (int)crank);
                 const bool half = last_half && tc.nt == n_tiles - 1;
                 const int brow = tc.e * args.b_rows_per_group + tc.nt * BN +
                                  (int)crank * (half ? BN / 4 : C::kBRows);
@@ -503,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t stg = base + C::kStgOff + (uint32_t)(warp - 2) * 2048u;
         uint32_t lt = 0;
         for (int tile = cid; tile < total; tile += ncl, ++lt) {
-            const TileCoord tc = tile_coord<TM>(tile, s_mt, E, n_tiles, args, (int)crank);
+            const TileCoord tc = tile_coord<TM, C::kCtaRows>(tile, s_mt, E, n_tiles, args, (int)crank);
             const uint32_t b = lt & 1u, use = lt >> 1;
             if (!mbar_wait<PAIR>(tfull_bar(b), use & 1u, st, 4)) {
                 // The router's routing warps meet two barriers per tile: keep meeting them.
@@ -655,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool have_next = false;
         int nidx[8];
         for (int tile = cid; ok && tile < total; tile += ncl) {
-            const TileCoord tc = tile_coord<TM>(tile, s_mt, E, n_tiles, args, (int)crank);
+            const TileCoord tc = tile_coord<TM, C::kCtaRows>(tile, s_mt, E, n_tiles, args, (int)crank);
             const __nv_bfloat16* src[8];
             uint32_t dst_off[8];
             bool valid[8];
@@ -678,7 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const int next = tile + ncl;
             TileCoord nc{0, 0, 0, 0};
-            if (next < total) nc = tile_coord<TM>(next, s_mt, E, n_tiles, args, (int)crank);
+            if (next < total) nc = tile_coord<TM, C::kCtaRows>(next, s_mt, E, n_tiles, args, (int)crank);
             have_next = false;
             for (int kb = 0; kb < nkb; ++kb, ++it) {
                 const int s = it % S;
@@ -705,7 +743,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------- router: warps 10-13 help write each tile's logits ----------------
         float* sL = reinterpret_cast<float*>(base_ptr + C::kStgOff);
         for (int tile = cid; tile < total; tile += ncl) {
-            const TileCoord tc = tile_coord<TM>(tile, s_mt, E, n_tiles, args, 0);
+            const TileCoord tc = tile_coord<TM, C::kCtaRows>(tile, s_mt, E, n_tiles, args, 0);
             router_tile(sL, C::kLStride, C::kEg, tc, args, warp - 2);
         }
     }
@@ -831,11 +869,11 @@ int num_sms() {
 }
 
 // The dynamic shared-memory attribute is per device; remember which devices have it.
-template <int BN, int EPI, bool GATHER, bool PAIR>
+template <int BN, int EPI, bool GATHER, bool PAIR, bool HALFM = false>
 cudaError_t launch_gemm_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,
                           const GemmArgs& a, long long tiles, cudaStream_t s) {
-    using C = Cfg<BN, PAIR, EPI>;
-    auto kern = grouped_gemm_kernel<BN, EPI, GATHER, PAIR>;
+    using C = Cfg<BN, PAIR, EPI, HALFM>;
+    auto kern = grouped_gemm_kernel<BN, EPI, GATHER, PAIR, HALFM>;
     static std::atomic<uint64_t> attr_done{0};
     static std::atomic<int> pair_slots[64];
     int dev = 0;
@@ -889,15 +927,15 @@ cudaError_t launch_gemm_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const 
     return note_launch(cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmD, a));
 }
 
-template <int EPI, bool GATHER, bool PAIR>
+template <int EPI, bool GATHER, bool PAIR, bool HALFM = false>
 cudaError_t launch_gemm_bn(int BN, const CUtensorMap& tmA, const CUtensorMap& tmB,
                            const CUtensorMap& tmD, const GemmArgs& a, long long tiles,
                            cudaStream_t s) {
     switch (BN) {
-        case 256: return launch_gemm_t<256, EPI, GATHER, PAIR>(tmA, tmB, tmD, a, tiles, s);
-        case 192: return launch_gemm_t<192, EPI, GATHER, PAIR>(tmA, tmB, tmD, a, tiles, s);
-        case 176: return launch_gemm_t<176, EPI, GATHER, PAIR>(tmA, tmB, tmD, a, tiles, s);
-        case 128: return launch_gemm_t<128, EPI, GATHER, PAIR>(tmA, tmB, tmD, a, tiles, s);
+        case 256: return launch_gemm_t<256, EPI, GATHER, PAIR, HALFM>(tmA, tmB, tmD, a, tiles, s);
+        case 192: return launch_gemm_t<192, EPI, GATHER, PAIR, HALFM>(tmA, tmB, tmD, a, tiles, s);
+        case 176: return launch_gemm_t<176, EPI, GATHER, PAIR, HALFM>(tmA, tmB, tmD, a, tiles, s);
+        case 128: return launch_gemm_t<128, EPI, GATHER, PAIR, HALFM>(tmA, tmB, tmD, a, tiles, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -924,8 +962,10 @@ cudaError_t launch_router_bn(int BN, const CUtensorMap& tmA, const CUtensorMap& 
 //    weight bytes, BN + 32, and the persistent grid finishes with its last partial wave, so
 //    the cost is ceil(tiles / SMs) x (BN + 32).  Measured on B200 at T = 64, E = 64, k = 8:
 //    d_model = 2048 outputs on 128-wide tiles (6.9 waves) beat 256-wide ones (3.5) by 13%.
+bool weight_streaming(long long max_rows, int E) { return max_rows <= 64LL * E; }
+
 int pick_bn(int nout, long long max_rows, int E, int num_sm) {
-    const bool streaming = max_rows <= 64LL * E;
+    const bool streaming = weight_streaming(max_rows, E);
     const long long m_tiles = streaming ? E : (max_rows + 127) / 128 + E;
     // Ties go to the wider tile when compute-bound, to the narrower one (finer waves) when
     // streaming.
@@ -992,17 +1032,33 @@ cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const in
     a.ldd = ldd;
     a.router_E = 0;
     a.st = st;
-    const int tm_rows = pair ? 256 : kBM;
+    // Weight streaming: 64-row m-tiles (more weight stages in flight), and each CTA reads up to
+    // 512 KB of its first weight tile into L2 before it waits for the dispatch (at most 76 MB on
+    // 148 SMs, well inside the 126 MB L2).
+    const bool halfm = weight_streaming(max_rows, E) && !pair;
+    a.W = W;
+    a.pf_bytes = halfm ? 512 * 1024 : 0;
+    const int tm_rows = pair ? 256 : (halfm ? 64 : kBM);
     const long long max_tiles = ((max_rows + tm_rows - 1) / tm_rows + E) * a.n_tiles;
-    // Contiguous A rows: a TMA tile map over the A buffer, 128-row boxes (unused when gathering).
+    // Contiguous A rows: a TMA tile map over the A buffer, 128-row boxes (64 with 64-row tiles;
+    // unused when gathering).
     CUtensorMap tmA = tm;
     const bool gather = a_rows != nullptr;
-    if (!gather && !make_tmap(&tmA, A, (long long)a_row_limit, K, kBM))
+    if (!gather && !make_tmap(&tmA, A, (long long)a_row_limit, K, halfm ? 64 : kBM))
         return cudaErrorInvalidValue;
     CUtensorMap tmD;
     if (!make_tmap_out(&tmD, D, max_rows, Nout, ldd)) return cudaErrorInvalidValue;
     cudaError_t e;
-    if (gather) {
+    if (halfm) {
+        if (gather)
+            e = which == 0
+                    ? launch_gemm_bn<kEpiSiLU, true, false, true>(BN, tmA, tm, tmD, a, max_tiles, s)
+                    : launch_gemm_bn<kEpiBias, true, false, true>(BN, tmA, tm, tmD, a, max_tiles, s);
+        else
+            e = which == 0
+                    ? launch_gemm_bn<kEpiSiLU, false, false, true>(BN, tmA, tm, tmD, a, max_tiles, s)
+                    : launch_gemm_bn<kEpiBias, false, false, true>(BN, tmA, tm, tmD, a, max_tiles, s);
+    } else if (gather) {
         e = which == 0 ? launch_gemm_bn<kEpiSiLU, true, false>(BN, tmA, tm, tmD, a, max_tiles, s)
                        : launch_gemm_bn<kEpiBias, true, false>(BN, tmA, tm, tmD, a, max_tiles, s);
     } else if (pair) {

@@ -59,7 +59,8 @@ __global__ void __launch_bounds__(1024) router_small_kernel(
     const __nv_bfloat16* __restrict__ x, const float* __restrict__ Wr,
     const float* __restrict__ br, int T, int d, int E, int k, float* __restrict__ logits_out,
     int32_t* __restrict__ ids, float* __restrict__ w, unsigned flags) {
-    pdl_begin();
+    pdl_trigger();                                    // the dispatch after it may be scheduled
+    pdl_wait();
     extern __shared__ float s_x[];                    // [d]
     __shared__ float s_part[1024];
     __shared__ float s_L[256];
@@ -754,7 +755,8 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(
     long long K, unsigned flags, int32_t* __restrict__ slot, uint8_t* __restrict__ drop,
     int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ rowtok,
     DeviceStatus* st) {
-    pdl_begin();
+    pdl_trigger();                                    // the expert GEMM may be scheduled (it
+    pdl_wait();                                       // prefetches its weights, then waits)
     extern __shared__ int32_t sm[];
     dispatch_small_block(ids, w, T, E, k, K, flags, slot, drop, counts, offsets, rowtok, st, sm);
 }

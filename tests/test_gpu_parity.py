@@ -151,6 +151,11 @@ def test_dispatch_bit_exact(T, E, k, C, dtype):
     (2000, 640, 256, 4, 2, 1.25, "bf16", 0.02),    # second GEMM on CTA pairs, half-width last tile
     (1024, 128, 192, 4, 1, math.inf, "bf16", 0.05),  # exactly 256 rows per expert: pairs
     (1023, 128, 192, 4, 1, math.inf, "bf16", 0.05),  # one row short of that: single-CTA tiles
+    # Weight streaming (at most 64 rows per expert on average): 64-row m-tiles.
+    (700, 256, 320, 16, 1, math.inf, "bf16", 0.05),  # experts above 64 rows: two m-tiles
+    (200, 128, 192, 8, 2, math.inf, "bf16", 0.05),   # ragged 64-row tiles, half-width last tile
+    (128, 64, 64, 2, 1, math.inf, "bf16", 0.1),      # 128 rows over two experts
+    (64, 2048, 1024, 64, 8, math.inf, "bf16", 0.0),  # the decode shape
     (40, 16, 24, 4, 2, 1.0, "f32", 0.1),
     (8, 4, 8, 4, 1, 1.25, "f32", 0.1)])
 def test_expert_ffn_parity(T, d, F, E, k, C, dtype, bias):
