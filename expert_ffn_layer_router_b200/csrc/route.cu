@@ -445,8 +445,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     __shared__ int s_warp[32];
     __shared__ uint32_t s_tk[kSelThreads];    // tie bin: keys and pair indices
     __shared__ int32_t s_tp[kSelThreads];
-    __shared__ int s_nt, s_bstar, s_need, s_found;
+    __shared__ int s_nt, s_bstar, s_need, s_found, s_b2, s_need2;
     __shared__ int s_hist[256];
+    __shared__ int s_h2[kHistBins];           // second-level histogram of the threshold bin
     __shared__ uint32_t s_prefix;
     __shared__ int s_rem;
     const int e = blockIdx.x, tid = threadIdx.x;
@@ -486,23 +487,24 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     auto key_from = [&](int32_t p) -> uint32_t {
         return arrival ? ~(uint32_t)p : __float_as_uint(w[p]);
     };
+    const bool need_keys = n > K && K > 0;      // otherwise every candidate is kept
     if (on_chip) {
-        // Four candidates per thread in flight: their list entries, then their weights.
-        for (int i0 = 0; i0 < n; i0 += 4 * kSelThreads) {
-            int32_t pv[4];
+        // Eight candidates per thread in flight: their list entries, then their weights.
+        for (int i0 = 0; i0 < n; i0 += 8 * kSelThreads) {
+            int32_t pv[8];
 #pragma unroll
-            for (int b = 0; b < 4; ++b) {
+            for (int b = 0; b < 8; ++b) {
                 const int i = i0 + b * kSelThreads + tid;
                 pv[b] = i < n ? list[i] : -1;
             }
 #pragma unroll
-            for (int b = 0; b < 4; ++b) {
+            for (int b = 0; b < 8; ++b) {
                 const int i = i0 + b * kSelThreads + tid;
                 if (i >= n) continue;
                 int32_t p = pv[b];
                 if (p < 0 || p >= P) { report(st, MOE_DEV_BAD_INDEX, 122); p = -1; }
                 s_list[i] = p;
-                s_keys[i] = p < 0 ? 0u : key_from(p);
+                s_keys[i] = (p < 0 || !need_keys) ? 0u : key_from(p);
             }
         }
     }
@@ -526,13 +528,17 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     if (!select_all && K > 0 && hist && !arrival) {
         // Threshold bin from the histogram: thread t holds bins 2047 - 2t and 2046 - 2t (top
         // down); b* is the bin where the count from the top reaches K.  Keys above b* are kept,
-        // below dropped; the `need` largest (ties: lower pair) of bin b* are kept.  Any
-        // inconsistency (histogram total != n, a tie bin larger than one key per thread) falls
-        // back to the radix selection below.
+        // below dropped; the `need` largest (ties: lower pair) of bin b* are kept.  A second
+        // histogram of bin b*'s keys over their next 11 bits (18..8) narrows the boundary to one
+        // sub-bin b2, whose few candidates are ranked exactly by (key desc, pair asc).  Any
+        // inconsistency (histogram total != n, the top bin, more than one candidate per thread
+        // in b2) falls back to the radix selection below.
         const uint32_t* h = hist + (size_t)e * kHistBins;
         const int b_hi = kHistBins - 1 - 2 * tid, b_lo = b_hi - 1;
         const int c_hi = (int)h[b_hi], c_lo = (int)h[b_lo];
-        if (tid == 0) { s_nt = 0; s_bstar = -1; s_found = 0; }
+        if (tid == 0) { s_nt = 0; s_bstar = -1; s_found = 0; s_b2 = -1; }
+        s_h2[b_hi] = 0;
+        s_h2[b_lo] = 0;
         int tot;
         const int above = block_exclusive_scan(c_hi + c_lo, s_warp, &tot);
         if (above < K && above + c_hi >= K) {
@@ -545,35 +551,56 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
         __syncthreads();
         bstar = s_bstar;
         const int need = s_need;
-        const int mt = bstar >= 0 ? (int)h[bstar] : kSelThreads + 1;
-        if (tot == n && mt <= kSelThreads) {
+        if (tot == n && bstar >= 0 && bstar < kHistBins - 1) {
             for (int i = tid; i < n; i += blockDim.x) {
                 if (!valid(i)) continue;
                 const uint32_t key = key_of(i);
-                if ((int)min(key >> 19, (uint32_t)(kHistBins - 1)) == bstar) {
-                    const int at = atomicAdd(&s_nt, 1);
-                    if (at < kSelThreads) { s_tk[at] = key; s_tp[at] = pair_of(i); }
-                }
+                if ((int)(key >> 19) == bstar) atomicAdd(&s_h2[(key >> 8) & (kHistBins - 1)], 1);
             }
             __syncthreads();
-            const int m = s_nt;
-            // Rank of each tied candidate by (key desc, pair asc); the need-th one bounds the
-            // kept set: key > tau, or key == tau and pair <= p_tau.
-            if (m == mt && tid < m) {
-                const uint32_t kt = s_tk[tid];
-                const int32_t pt = s_tp[tid];
-                int rank = 0;
-                for (int j = 0; j < m; ++j) {
-                    const uint32_t kj = s_tk[j];
-                    rank += (kj > kt || (kj == kt && s_tp[j] < pt)) ? 1 : 0;
-                }
-                if (rank == need - 1) { s_prefix = kt; s_rem = pt; s_found = 1; }
+            const int d_hi = s_h2[b_hi], d_lo = s_h2[b_lo];
+            int tot2;
+            const int above2 = block_exclusive_scan(d_hi + d_lo, s_warp, &tot2);
+            if (above2 < need && above2 + d_hi >= need) {
+                s_b2 = b_hi;
+                s_need2 = need - above2;
+            } else if (above2 + d_hi < need && above2 + d_hi + d_lo >= need) {
+                s_b2 = b_lo;
+                s_need2 = need - above2 - d_hi;
             }
             __syncthreads();
-            if (s_found) {
-                by_hist = true;
-                tau = s_prefix;
-                p_tau = s_rem;
+            const int b2 = s_b2, need2 = s_need2;
+            const int mt = b2 >= 0 ? s_h2[b2] : kSelThreads + 1;
+            if (mt <= kSelThreads) {
+                const uint32_t pre24 = ((uint32_t)bstar << 11) | (uint32_t)b2;   // key bits 29..8
+                for (int i = tid; i < n; i += blockDim.x) {
+                    if (!valid(i)) continue;
+                    const uint32_t key = key_of(i);
+                    if ((key >> 8) == pre24) {
+                        const int at = atomicAdd(&s_nt, 1);
+                        if (at < kSelThreads) { s_tk[at] = key; s_tp[at] = pair_of(i); }
+                    }
+                }
+                __syncthreads();
+                const int m = s_nt;
+                // Rank of each candidate of b2 by (key desc, pair asc); the need2-th one bounds
+                // the kept set: key > tau, or key == tau and pair <= p_tau.
+                if (m == mt && tid < m) {
+                    const uint32_t kt = s_tk[tid];
+                    const int32_t pt = s_tp[tid];
+                    int rank = 0;
+                    for (int j = 0; j < m; ++j) {
+                        const uint32_t kj = s_tk[j];
+                        rank += (kj > kt || (kj == kt && s_tp[j] < pt)) ? 1 : 0;
+                    }
+                    if (rank == need2 - 1) { s_prefix = kt; s_rem = pt; s_found = 1; }
+                }
+                __syncthreads();
+                if (s_found) {
+                    by_hist = true;
+                    tau = s_prefix;
+                    p_tau = s_rem;
+                }
             }
         }
     }
@@ -631,10 +658,23 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
             }
             slot[p] = sl;
             drop[p] = 0;
-            if (rowtok) rowtok[off + sl] = t;
         } else {
             slot[p] = -1;
             drop[p] = 1;
+        }
+    }
+    // Row map in token order, one bitmap word per thread: each thread writes the rows of its
+    // word's kept tokens, and neighbouring threads write neighbouring rows.
+    if (rowtok) {
+        for (int wi = tid; wi < nw; wi += blockDim.x) {
+            uint32_t word = bits[wi];
+            int sl = (int)pre[wi];
+            while (word) {
+                const int j = __ffs(word) - 1;
+                word &= word - 1u;
+                if (sl < kept) rowtok[off + sl] = wi * 32 + j;
+                ++sl;
+            }
         }
     }
 }
