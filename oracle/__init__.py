@@ -39,6 +39,9 @@ def lib():
         L.oracle_route.restype = ctypes.c_int
         L.oracle_route.argtypes = [ctypes.c_int] * 3 + [ctypes.c_longlong, _f32p, _i32p, _f32p,
                                                         _i32p, _u8p, _i32p, ctypes.c_int]
+        L.oracle_select.restype = ctypes.c_int
+        L.oracle_select.argtypes = [ctypes.c_int] * 3 + [ctypes.c_longlong, _i32p, _f32p,
+                                                         _i32p, _u8p, _i32p, ctypes.c_int]
         L.oracle_dispatch.restype = ctypes.c_int
         L.oracle_dispatch.argtypes = [ctypes.c_int] * 3 + [_i32p, _i32p, _i32p, _i32p]
         L.oracle_expert_rows.restype = ctypes.c_int
@@ -124,6 +127,22 @@ def route(logits_, k, K, flags=0):
         raise ValueError("oracle_route rejected its arguments")
     return dict(ids=ids, w=w, slot=slot, drop=drop, received=counts[:E].copy(),
                 kept=counts[E:].copy())
+
+
+def select(ids, w, E, K, flags=0):
+    """Capacity selection of a given routing: ids/w [T, k] (pair p = t*k + j); each expert keeps
+    at most K pairs by (weight descending, token ascending), or its first K in token order with
+    ARRIVAL_ORDER; slots rank the kept tokens in token order."""
+    ids = _c(ids, np.int32)
+    w = _c(w, np.float32)
+    T, k = ids.shape
+    slot = np.empty((T, k), np.int32)
+    drop = np.empty((T, k), np.uint8)
+    counts = np.empty(2 * E, np.int32)
+    rc = lib().oracle_select(T, E, k, int(K), ids, w, slot, drop, counts, int(flags))
+    if rc != 0:
+        raise ValueError("oracle_select rejected its arguments")
+    return dict(slot=slot, drop=drop, received=counts[:E].copy(), kept=counts[E:].copy())
 
 
 def dispatch(ids, slot, E):

@@ -218,38 +218,19 @@ void oracle_logits(int T, int d, int E, int dtype, const void* x, const float* W
     });
 }
 
-// Routing: softmax, top-k, capacity selection and slot map.
-//   ids[T*k], w[T*k]: pair p = t*k + j, j = 0 is the largest logit;
+// Capacity selection of a given routing ("Expert Networks > Worked Example: Expert
+// Specialization", capacity paragraph; "Some Tokens Do Not Get In", "Past the edge"):
+//   ids[T*k], w[T*k]: pair p = t*k + j routed to expert ids[p] with router weight w[p];
+//   each expert keeps at most K of its pairs, by (weight descending, token ascending) -- or, with
+//   flags & 2, its first K pairs in token order;
 //   slot[T*k]: rank among the expert's kept tokens (ascending t), -1 if dropped;
 //   drop[T*k]: 1 if dropped;  counts[2E]: received per expert, then kept per expert.
-// Returns 0, or -1 on bad arguments.
-// flags: 1 = renormalise each token's k weights by their sum (fp32, j ascending, one division
-// each); 2 = capacity by arrival (token) order instead of by weight ("Some Tokens Do Not Get
-// In", "Past the edge").
-int oracle_route(int T, int E, int k, long long K, const float* logits, int32_t* ids, float* w,
-                 int32_t* slot, uint8_t* drop, int32_t* counts, int flags) {
-    if (T < 0 || E <= 0 || k <= 0 || k > E || K < 0) return -1;
-    std::vector<float> p(E);
-    for (int t = 0; t < T; ++t) {
-        const float* L = logits + (size_t)t * E;
-        softmax_row(L, E, p.data());
-        std::vector<char> taken(E, 0);
-        for (int j = 0; j < k; ++j) {
-            int best = -1;
-            for (int e = 0; e < E; ++e) {
-                if (taken[e]) continue;
-                if (best < 0 || topk_before(L[e], e, L[best], best)) best = e;
-            }
-            taken[best] = 1;
-            ids[(size_t)t * k + j] = best;
-            w[(size_t)t * k + j] = p[best];
-        }
-        if (flags & 1) {
-            float sum = 0.0f;
-            for (int j = 0; j < k; ++j) sum = sum + w[(size_t)t * k + j];
-            for (int j = 0; j < k; ++j) w[(size_t)t * k + j] = w[(size_t)t * k + j] / sum;
-        }
-    }
+// Returns 0, or -1 on bad arguments (an id outside [0, E)).
+int oracle_select(int T, int E, int k, long long K, const int32_t* ids, const float* w,
+                  int32_t* slot, uint8_t* drop, int32_t* counts, int flags) {
+    if (T < 0 || E <= 0 || k <= 0 || K < 0) return -1;
+    for (long long p = 0; p < (long long)T * k; ++p)
+        if (ids[p] < 0 || ids[p] >= E) return -1;
     // Candidate pairs of each expert, ascending token index.
     std::vector<std::vector<int>> cand(E);
     for (int t = 0; t < T; ++t)
@@ -278,6 +259,37 @@ int oracle_route(int T, int E, int k, long long K, const float* logits, int32_t*
         counts[E + e] = s;
     }
     return 0;
+}
+
+// Routing: softmax, top-k, then the capacity selection above.
+//   ids[T*k], w[T*k]: pair p = t*k + j, j = 0 is the largest logit.
+// flags: 1 = renormalise each token's k weights by their sum (fp32, j ascending, one division
+// each); 2 = capacity by arrival (token) order instead of by weight.
+int oracle_route(int T, int E, int k, long long K, const float* logits, int32_t* ids, float* w,
+                 int32_t* slot, uint8_t* drop, int32_t* counts, int flags) {
+    if (T < 0 || E <= 0 || k <= 0 || k > E || K < 0) return -1;
+    std::vector<float> p(E);
+    for (int t = 0; t < T; ++t) {
+        const float* L = logits + (size_t)t * E;
+        softmax_row(L, E, p.data());
+        std::vector<char> taken(E, 0);
+        for (int j = 0; j < k; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if (taken[e]) continue;
+                if (best < 0 || topk_before(L[e], e, L[best], best)) best = e;
+            }
+            taken[best] = 1;
+            ids[(size_t)t * k + j] = best;
+            w[(size_t)t * k + j] = p[best];
+        }
+        if (flags & 1) {
+            float sum = 0.0f;
+            for (int j = 0; j < k; ++j) sum = sum + w[(size_t)t * k + j];
+            for (int j = 0; j < k; ++j) w[(size_t)t * k + j] = w[(size_t)t * k + j] / sum;
+        }
+    }
+    return oracle_select(T, E, k, K, ids, w, slot, drop, counts, flags);
 }
 
 // Expert-sorted row layout: offsets[E+1] (exclusive prefix of kept counts) and

@@ -215,6 +215,53 @@ def test_route_matches_brute_force(seed, T, E, k, C):
                 assert r["drop"][t, j] == 1 and r["slot"][t, j] == -1
 
 
+def _given_routing(T, E, k, seed, ties):
+    """A routing that no router produced: each token's k distinct experts drawn at random, weights
+    from a few values (ties across tokens) or continuous."""
+    rng = np.random.default_rng(seed)
+    ids = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    if ties:
+        w = (rng.integers(1, 5, size=(T, k)) * 0.125).astype(np.float32)
+    else:
+        w = rng.random((T, k)).astype(np.float32)
+    return ids, w
+
+
+@pytest.mark.parametrize("seed", range(4))
+@pytest.mark.parametrize("T,E,k,K", [(30, 4, 1, 5), (40, 6, 2, 9), (25, 5, 3, 0), (50, 8, 4, 100),
+                                     (64, 3, 2, 17)])
+@pytest.mark.parametrize("flags", [0, 2])
+def test_select_matches_brute_force(seed, T, E, k, K, flags):
+    # Capacity selection of a given routing ("Expert Networks > Worked Example", capacity
+    # paragraph: the lowest-confidence tokens drop; "Some Tokens Do Not Get In", "Past the edge":
+    # in arrival order) against an exhaustive sort of each expert's candidates.
+    ids, w = _given_routing(T, E, k, seed, ties=seed % 2 == 0)
+    r = oracle.select(ids, w, E, K, flags)
+    for e in range(E):
+        cand = [(t, j) for t in range(T) for j in range(k) if ids[t, j] == e]
+        if flags & oracle.ARRIVAL_ORDER:
+            ranked = sorted(cand)
+        else:
+            ranked = sorted(cand, key=lambda tj: (-float(w[tj]), tj[0]))
+        keep = set(ranked[:K])
+        kept_sorted = sorted(keep)
+        assert r["received"][e] == len(cand)
+        assert r["kept"][e] == min(len(cand), K)
+        for tj in cand:
+            if tj in keep:
+                assert r["drop"][tj] == 0 and r["slot"][tj] == kept_sorted.index(tj)
+            else:
+                assert r["drop"][tj] == 1 and r["slot"][tj] == -1
+
+
+def test_select_rejects_ids_outside_the_experts():
+    ids = np.array([[0], [4]], np.int32)
+    with pytest.raises(ValueError):
+        oracle.select(ids, np.ones((2, 1), np.float32), 4, 1)
+    with pytest.raises(ValueError):
+        oracle.select(-ids, np.ones((2, 1), np.float32), 4, 1)
+
+
 def test_drop_is_by_confidence_not_arrival():
     # Expert 0 receives tokens 0, 1, 2; token 0 (first to arrive) has the lowest confidence and
     # must be the one dropped; an arrival-order buffer would drop token 2 instead.
