@@ -24,6 +24,11 @@ int route_group_lanes(int E, int k);
 void launch_route_place(const float* logits, int T, int E, int k, unsigned flags, int32_t* ids,
                         float* w, int32_t* gcnt, int32_t* cand, DeviceStatus* st, cudaStream_t s,
                         int* launches);
+// Candidate lists and weight histograms of a given routing (ids, w [T*k]), as launch_route_place
+// builds them; the same counters must be zero at entry.
+void launch_place_given(const int32_t* ids, const float* w, int T, int E, int k, unsigned flags,
+                        int32_t* gcnt, int32_t* cand, DeviceStatus* st, cudaStream_t s,
+                        int* launches);
 // Capacity selection from the candidate lists: slot, drop, counts (nullable), offsets and rowtok
 // (nullable).  flags: MOE_FLAG_ARRIVAL_ORDER keeps an overflowing expert's first K pairs in token
 // order.  gbits: select_bits_bytes(T, E) bytes of scratch (unused and nullable when that is 0).

@@ -310,6 +310,69 @@ moe_status moe_route(const moe_problem* p, const float* logits, int32_t* ids, fl
     return finish(launches);
 }
 
+moe_status moe_capacity_dispatch(const moe_problem* p, long long K, const int32_t* ids,
+                                 const float* w, int32_t* slot, uint8_t* drop, int32_t* counts,
+                                 int32_t* offsets, int32_t* rowtok, void* ws, size_t ws_bytes,
+                                 void* stream) {
+    moe_status r = pre(p, false);
+    if (r != MOE_OK) return r;
+    if (K < 0 || !counts || (p->T > 0 && (!ids || !w || !slot || !drop)) ||
+        (rowtok && !offsets))
+        return MOE_ERR_INVALID_ARG;
+    Plan q;
+    if ((r = check_ws(p, ws, ws_bytes, &q)) != MOE_OK) return r;
+    cudaStream_t s = (cudaStream_t)stream;
+    int launches = 0;
+    if (p->T == 0) {
+        moe::note_launch(cudaMemsetAsync(counts, 0, sizeof(int32_t) * 2 * p->E, s));
+        if (offsets)
+            moe::note_launch(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (p->E + 1), s));
+        return finish(0);
+    }
+    const RouteScratch rs = scratch_of(ws, q);
+    if (moe::dispatch_small_fits(p->T, p->k)) {
+        moe::launch_dispatch_small(ids, w, p->T, p->E, p->k, K, p->flags, slot, drop, counts,
+                                   offsets, rowtok, rs.st, s, &launches);
+        return finish(launches);
+    }
+    moe::note_launch(cudaMemsetAsync(rs.gcnt, 0, sizeof(int32_t) * moe::dispatch_counter_ints(p->E), s));
+    moe::launch_place_given(ids, w, p->T, p->E, p->k, p->flags, rs.gcnt, rs.cand, rs.st, s,
+                            &launches);
+    moe::launch_select(rs.cand, rs.gcnt, w, p->T, p->E, p->k, K, p->flags, rs.bits, slot, drop,
+                       counts, offsets, rowtok, rs.st, s, &launches);
+    return finish(launches);
+}
+
+moe_status moe_router_logits(const moe_problem* p, const void* x, const float* Wr,
+                             const float* br, float* logits, void* ws, size_t ws_bytes,
+                             void* stream) {
+    moe_status r = pre(p, false);
+    if (r != MOE_OK) return r;
+    if (!Wr || (p->T > 0 && (!x || !logits))) return MOE_ERR_INVALID_ARG;
+    if (p->dtype == MOE_BF16 && misaligned(x, 16)) return MOE_ERR_INVALID_ARG;
+    Plan q;
+    if ((r = check_ws(p, ws, ws_bytes, &q)) != MOE_OK) return r;
+    if (p->T == 0) return finish(0);
+    cudaStream_t s = (cudaStream_t)stream;
+    int launches = 0;
+    // The kernels of moe_forward's first stage, so the logits are the forward's bit for bit.
+    if (p->dtype == MOE_BF16 && moe::router_small_fits(p->T, p->E, p->d_model)) {
+        moe::launch_router_small(x, Wr, br, p->T, p->d_model, p->E, p->k, logits,
+                                 at<int32_t>(ws, q.ids), at<float>(ws, q.w), p->flags, s,
+                                 &launches);
+    } else if (p->dtype == MOE_BF16) {
+        if (p->d_model % 64 != 0) return MOE_ERR_UNSUPPORTED;
+        if (moe::launch_router_gemm(x, p->T, p->d_model, Wr, br, p->E, at<void>(ws, q.split),
+                                    logits, nullptr, 0, at<moe::DeviceStatus>(ws, q.status), s,
+                                    &launches) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    } else {
+        moe::launch_logits_f32((const float*)x, Wr, br, p->T, p->d_model, p->E, logits, nullptr,
+                               0, s, &launches);
+    }
+    return finish(launches);
+}
+
 moe_status moe_dispatch(const moe_problem* p, const int32_t* ids, const int32_t* slot,
                         int32_t* offsets, int32_t* rowtok, const void* x, void* x_perm,
                         void* ws, size_t ws_bytes, void* stream) {

@@ -357,6 +357,56 @@ __global__ void __launch_bounds__(256) route_place_warp_kernel(
 }
 
 // ---------------------------------------------------------------------------------------------
+// Placement of a given routing (no router): pairs p in [0, T*k) with expert ids[p] and weight
+// w[p] go to their experts' candidate lists and weight histograms, as the routers above place
+// theirs.  Each thread takes kGivenPairs pairs; per-block counters in shared memory ([E] ints,
+// dynamic), one global atomic per (block, expert).  An id outside [0, E) is recorded as
+// MOE_DEV_BAD_INDEX (site 135) and its pair left out; a weight that is not >= +0 (negative, -0,
+// NaN) is recorded (site 134): the selection orders weights by their bit patterns.
+// ---------------------------------------------------------------------------------------------
+constexpr int kGivenPairs = 4;
+
+__global__ void __launch_bounds__(256) place_given_kernel(
+    const int32_t* __restrict__ ids, const float* __restrict__ w, long long P, int T, int E,
+    int32_t* __restrict__ gcnt, int32_t* __restrict__ cand, uint32_t* __restrict__ hist,
+    DeviceStatus* st) {
+    pdl_begin();
+    extern __shared__ int s_given[];                   // [E] block counts, then [E] bases
+    int* s_n = s_given;
+    int* s_base = s_given + E;
+    const int tid = threadIdx.x;
+    for (int e = tid; e < E; e += blockDim.x) s_n[e] = 0;
+    __syncthreads();
+    const long long p0 = (long long)blockIdx.x * blockDim.x * kGivenPairs;
+    int my_e[kGivenPairs], my_pos[kGivenPairs];
+#pragma unroll
+    for (int i = 0; i < kGivenPairs; ++i) {
+        const long long p = p0 + (long long)i * blockDim.x + tid;
+        my_e[i] = -1;
+        my_pos[i] = 0;
+        if (p >= P) continue;
+        const int e = ids[p];
+        const float wv = w[p];
+        if ((unsigned)e >= (unsigned)E) { report(st, MOE_DEV_BAD_INDEX, 135); continue; }
+        if (!(wv >= 0.0f) || (__float_as_uint(wv) >> 31)) report(st, MOE_DEV_BAD_INDEX, 134);
+        my_e[i] = e;
+        my_pos[i] = atomicAdd(&s_n[e], 1);
+        if (hist) atomicAdd(&hist[(size_t)e * kHistBins + hist_bin(wv)], 1u);
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += blockDim.x) s_base[e] = s_n[e] ? atomicAdd(&gcnt[e], s_n[e]) : 0;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kGivenPairs; ++i) {
+        if (my_e[i] < 0) continue;
+        const long long p = p0 + (long long)i * blockDim.x + tid;
+        const long long pos = (long long)s_base[my_e[i]] + my_pos[i];
+        if (pos < T) cand[(size_t)my_e[i] * T + pos] = (int32_t)p;
+        else report(st, MOE_DEV_BAD_INDEX, 133);       // a token listed one expert twice, or
+    }                                                  // the counters were not zero at entry
+}
+
+// ---------------------------------------------------------------------------------------------
 // Capacity selection from unordered candidate lists: one block per expert.
 // ---------------------------------------------------------------------------------------------
 constexpr int kSelThreads = 1024;
@@ -994,6 +1044,20 @@ void launch_route_place(const float* logits, int T, int E, int k, unsigned flags
             launch_pdl(route_place_warp_kernel<32>, g, dim3(256), smem, s, logits, T, E, k, flags,
                        ids, w, gcnt, cand, hist, st);
     }
+    *launches += 1;
+}
+
+void launch_place_given(const int32_t* ids, const float* w, int T, int E, int k, unsigned flags,
+                        int32_t* gcnt, int32_t* cand, DeviceStatus* st, cudaStream_t s,
+                        int* launches) {
+    uint32_t* hist = (flags & MOE_FLAG_ARRIVAL_ORDER) ? nullptr
+                                                      : reinterpret_cast<uint32_t*>(gcnt + E);
+    const long long P = (long long)T * k;
+    if (P == 0) return;
+    const long long per_block = 256LL * kGivenPairs;
+    const dim3 g((unsigned)((P + per_block - 1) / per_block));
+    launch_pdl(place_given_kernel, g, dim3(256), 2 * sizeof(int) * (size_t)E, s, ids, w, P, T, E,
+               gcnt, cand, hist, st);
     *launches += 1;
 }
 

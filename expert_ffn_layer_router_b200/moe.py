@@ -47,6 +47,8 @@ def _load():
         "moe_capacity": [P, ctypes.POINTER(ctypes.c_int64)],
         "moe_workspace_size": [P, ctypes.POINTER(ctypes.c_size_t)],
         "moe_route": [P, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+        "moe_capacity_dispatch": [P, ctypes.c_int64] + [vp] * 8 + [sz, vp],
+        "moe_router_logits": [P, vp, vp, vp, vp, vp, sz, vp],
         "moe_dispatch": [P, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "moe_expert_ffn": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "moe_combine": [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
@@ -73,7 +75,8 @@ _lib = _load()
 EXPORTS = ("moe_capacity", "moe_workspace_size", "moe_route", "moe_dispatch", "moe_expert_ffn",
            "moe_combine", "moe_forward", "moe_get_device_status", "moe_reset_device_status",
            "moe_last_launch_count", "moe_status_string", "moe_set_stage_events",
-           "moe_route_static", "moe_selftest_wait_timeout")
+           "moe_route_static", "moe_selftest_wait_timeout", "moe_capacity_dispatch",
+           "moe_router_logits")
 
 STAGE_EVENTS = 7
 STAGE_NAMES = ("router_logits", "route_topk", "capacity_dispatch", "expert_gemm1",
@@ -132,6 +135,20 @@ def moe_route(p, logits, ids, w, slot, drop, counts, ws, stream=None):
     _check(_lib.moe_route(ctypes.byref(p), _ptr(logits), _ptr(ids), _ptr(w), _ptr(slot),
                           _ptr(drop), _ptr(counts), _ptr(ws), ws.numel() * ws.element_size(),
                           _stream(stream)), "moe_route")
+
+
+def moe_capacity_dispatch(p, K, ids, w, slot, drop, counts, ws, offsets=None, rowtok=None,
+                          stream=None):
+    _check(_lib.moe_capacity_dispatch(ctypes.byref(p), int(K), _ptr(ids), _ptr(w), _ptr(slot),
+                                      _ptr(drop), _ptr(counts), _ptr(offsets), _ptr(rowtok),
+                                      _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_capacity_dispatch")
+
+
+def moe_router_logits(p, x, Wr, br, logits, ws, stream=None):
+    _check(_lib.moe_router_logits(ctypes.byref(p), _ptr(x), _ptr(Wr), _ptr(br), _ptr(logits),
+                                  _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_router_logits")
 
 
 def moe_dispatch(p, ids, slot, offsets, rowtok, ws, x=None, x_perm=None, stream=None):
@@ -242,6 +259,25 @@ class MoELayer:
                  counts=torch.empty(2 * p.E, dtype=torch.int32, device=dev))
         moe_route(p, logits, r["ids"], r["w"], r["slot"], r["drop"], r["counts"], self.ws,
                   stream)
+        return r
+
+    def router_logits(self, x, Wr, br, stream=None):
+        logits = torch.empty((self.p.T, self.p.E), dtype=torch.float32, device=x.device)
+        moe_router_logits(self.p, x, Wr, br, logits, self.ws, stream)
+        return logits
+
+    def capacity_dispatch(self, ids, w, K, stream=None):
+        """Capacity selection of a given routing (ids, w [T, k]) with capacity K; returns slot,
+        drop, counts and the expert-sorted layout (offsets, rowtok)."""
+        p, dev = self.p, ids.device
+        rows = max(min(p.T * p.k, p.E * int(K)), 1)
+        r = dict(slot=torch.empty((p.T, p.k), dtype=torch.int32, device=dev),
+                 drop=torch.empty((p.T, p.k), dtype=torch.uint8, device=dev),
+                 counts=torch.empty(2 * p.E, dtype=torch.int32, device=dev),
+                 offsets=torch.empty(p.E + 1, dtype=torch.int32, device=dev),
+                 rowtok=torch.empty(rows, dtype=torch.int32, device=dev))
+        moe_capacity_dispatch(p, K, ids, w, r["slot"], r["drop"], r["counts"], self.ws,
+                              r["offsets"], r["rowtok"], stream)
         return r
 
     def dispatch(self, ids, slot, x=None, permute=False, stream=None):

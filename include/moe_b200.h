@@ -118,6 +118,36 @@ moe_status moe_route(const moe_problem* p, const float* logits, int32_t* ids, fl
                      int32_t* slot, uint8_t* drop, int32_t* counts, void* ws, size_t ws_bytes,
                      void* stream);
 
+/* Capacity-limited dispatch of a given routing, steps 2-3 without the router ("Expert Networks >
+ * Worked Example: Expert Specialization", capacity paragraph; "Some Tokens Do Not Get In",
+ * "Past the edge"): for routings formed elsewhere, and for the owner of a set of experts under
+ * expert parallelism, which selects among candidates gathered from every rank.
+ *   p: T, E, k and flags (MOE_FLAG_ARRIVAL_ORDER keeps an overflowing expert's first K pairs in
+ *   token order; MOE_FLAG_RENORMALIZE is ignored: the weights are given); capacity_factor,
+ *   d_model and d_ff size the workspace only (moe_workspace_size with the same p).
+ *   K >= 0: the capacity of every expert, given explicitly (it need not be C*T*k/E of p).
+ *   ids [T*k] int32 in: pair p = t*k + j goes to expert ids[p]; a token's k ids must be
+ *   distinct (as a top-k gives them).  w [T*k] float32 in: its weight, >= +0 and finite.
+ *   slot, drop [T*k] and counts [2E] out, as moe_route gives them for the same ids and w.
+ *   offsets [E+1] int32 out (nullable): exclusive prefix of the kept counts.
+ *   rowtok (nullable; needs offsets) int32 out, min(T*k, E*K) entries: rowtok[offsets[e] +
+ *   slot] = token t of that kept pair.
+ * Errors: MOE_ERR_INVALID_ARG for K < 0 or missing buffers; device-detected bad ids (outside
+ * [0, E)) or weights (negative, -0, NaN) go to the status word as MOE_DEV_BAD_INDEX. */
+moe_status moe_capacity_dispatch(const moe_problem* p, long long K, const int32_t* ids,
+                                 const float* w, int32_t* slot, uint8_t* drop, int32_t* counts,
+                                 int32_t* offsets, int32_t* rowtok, void* ws, size_t ws_bytes,
+                                 void* stream);
+
+/* Router logits alone, step 1's first half ("Dynamic Token Routing AI", How it works: the gating
+ * network scores every token): logits [T, E] float32 = x Wr + br, with moe_forward's kernels, so
+ * the values equal its logits_out bit for bit.  x [T, d_model] in p's dtype (16-byte aligned for
+ * bf16), Wr [d_model, E] float32, br [E] float32 or NULL.  bf16 batches above 1024 tokens need
+ * d_model a multiple of 64 (else MOE_ERR_UNSUPPORTED). */
+moe_status moe_router_logits(const moe_problem* p, const void* x, const float* Wr,
+                             const float* br, float* logits, void* ws, size_t ws_bytes,
+                             void* stream);
+
 /* Dispatch layout from a routing.
  *   ids, slot [T*k] in;  offsets [E+1] int32 out (exclusive prefix of kept counts);
  *   rowtok [min(T*k, E*K)] int32 out: rowtok[offsets[e] + slot] = token of that kept pair.

@@ -106,3 +106,27 @@ def test_status_strings(moe):
     for s in range(6):
         assert moe.lib().moe_status_string(s)
     assert moe.lib().moe_status_string(99) == b"unknown status"
+
+
+def test_given_routing_and_logits_calls_reject_bad_arguments(moe):
+    """moe_capacity_dispatch and moe_router_logits check their arguments before any launch."""
+    lib = moe.lib()
+    fake = ctypes.c_void_p(4096)                     # never dereferenced: rejected first
+    p = moe.Problem(16, 64, 64, 4, 2, 1.0, 1, 0)
+    bad = moe.Problem(16, 64, 64, 0, 2, 1.0, 1, 0)
+    cd = lib.moe_capacity_dispatch
+    # K < 0, a missing input, a malformed problem, rowtok without offsets: invalid argument.
+    assert cd(ctypes.byref(p), -1, fake, fake, fake, fake, fake, None, None, fake, 1 << 20,
+              None) == 1
+    assert cd(ctypes.byref(p), 3, None, fake, fake, fake, fake, None, None, fake, 1 << 20,
+              None) == 1
+    assert cd(ctypes.byref(bad), 3, fake, fake, fake, fake, fake, None, None, fake, 1 << 20,
+              None) == 1
+    assert cd(ctypes.byref(p), 3, fake, fake, fake, fake, fake, None, fake, fake, 1 << 20,
+              None) == 1
+    # No workspace: MOE_ERR_WORKSPACE (3).
+    assert cd(ctypes.byref(p), 3, fake, fake, fake, fake, fake, None, None, None, 0, None) == 3
+    rl = lib.moe_router_logits
+    assert rl(ctypes.byref(bad), fake, fake, None, fake, fake, 1 << 20, None) == 1
+    assert rl(ctypes.byref(p), fake, None, None, fake, fake, 1 << 20, None) == 1
+    assert rl(ctypes.byref(p), fake, fake, None, fake, None, 0, None) == 3

@@ -1,0 +1,28 @@
+"""Expert parallelism on two gloo ranks (CPU): the exchange of candidates, slots, rows and
+expert outputs around the owner's capacity selection and FFN, with every compute step done by
+the oracle.  Each rank's outputs and routing must equal the single-batch oracle layer's on the
+union of both ranks' tokens, bit for bit ("Expert Networks > Worked Example: Expert
+Specialization": the experts run on different hardware units; the capacity, drop priority and
+slots are those of the whole batch)."""
+import math
+
+import pytest
+import torch.multiprocessing as mp
+
+from tests import ep_worker
+
+
+@pytest.mark.parametrize("cfg", [
+    (48, 16, 24, 8, 2, 1.0, "f32", 0, 1),        # drops at the experts' owners
+    (40, 16, 24, 4, 1, 0.5, "f32", 0, 2),        # top-1, half the pairs dropped
+    (32, 8, 12, 6, 3, 0.75, "f32", 2, 3),        # arrival order
+    (32, 8, 12, 6, 3, 1.0, "f32", 1, 4),         # renormalised weights
+    (24, 16, 32, 4, 2, math.inf, "bf16", 0, 5),  # dropless, bf16 values
+    (16, 8, 8, 2, 2, 0.5, "f32", 0, 6)])         # one expert per rank, k = E
+def test_expert_parallel_matches_single_batch(cfg):
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    port = 29600 + cfg[-1]
+    mp.start_processes(ep_worker.cpu_rank, args=(2, port, cfg, out), nprocs=2,
+                       start_method="spawn")
+    assert out[0] == [] and out[1] == [], (out[0], out[1])

@@ -352,6 +352,76 @@ def test_forward_routing_matches_route(T, d, E, k, C, flags):
 
 
 # ------------------------------------------------------------------------------------------
+# Capacity dispatch of a given routing (moe_capacity_dispatch) against the oracle's selection,
+# and the router logits alone (moe_router_logits) against the forward's own logits.
+# ------------------------------------------------------------------------------------------
+def _given_routing(T, E, k, seed, ties):
+    rng = np.random.default_rng(seed)
+    ids = np.argsort(rng.random((T, E)), axis=1)[:, :k].astype(np.int32)
+    if ties:
+        w = (rng.integers(1, 5, size=(T, k)) * 0.125).astype(np.float32)
+    else:
+        w = rng.random((T, k)).astype(np.float32)
+    return ids, w
+
+
+@pytest.mark.parametrize("T,E,k,K,flags,ties", [
+    (300, 8, 2, 50, 0, True),           # single-block path (T k <= 1024)
+    (512, 64, 2, 9, 2, False),          # single-block path, arrival order
+    (3000, 64, 6, 200, 0, False),       # candidate lists + histogram selection
+    (3000, 64, 6, 200, 0, True),        # weight ties: the threshold bin is one value
+    (3000, 64, 6, 200, 2, False),       # arrival order (radix path)
+    (5000, 16, 1, 400, 0, False),
+    (2000, 128, 8, 10000, 0, False),    # nothing dropped
+    (1100, 5, 3, 0, 0, False),          # K = 0: everything dropped
+    (20000, 32, 1, 700, 0, True)])
+def test_capacity_dispatch_matches_oracle(T, E, k, K, flags, ties):
+    moe = _moe()
+    ids, w = _given_routing(T, E, k, T + E, ties)
+    layer = moe.MoELayer(T, 64, 64, E, k, 1.0, "bf16", flags=flags)
+    r = layer.capacity_dispatch(to_dev(ids), to_dev(w), K)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(layer.ws) == 0
+    ro = oracle.select(ids, w, E, K, flags)
+    assert np.array_equal(to_host(r["slot"]), ro["slot"])
+    assert np.array_equal(to_host(r["drop"]), ro["drop"])
+    counts = to_host(r["counts"])
+    assert np.array_equal(counts[:E], ro["received"]) and np.array_equal(counts[E:], ro["kept"])
+    off_ref, rowtok_ref = oracle.dispatch(ids, ro["slot"], E)
+    assert np.array_equal(to_host(r["offsets"]), off_ref)
+    n = int(off_ref[-1])
+    assert np.array_equal(to_host(r["rowtok"])[:n], rowtok_ref)
+
+
+def test_capacity_dispatch_reports_bad_ids():
+    moe = _moe()
+    T, E, k = 2000, 8, 2
+    ids, w = _given_routing(T, E, k, 5, False)
+    ids[17, 1] = E                      # outside [0, E): left out and reported
+    layer = moe.MoELayer(T, 64, 64, E, k, 1.0, "bf16")
+    layer.capacity_dispatch(to_dev(ids), to_dev(w), 300)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(layer.ws) == moe.DEV_BAD_INDEX
+
+
+@pytest.mark.parametrize("T,d,E,dtype", [(64, 2048, 64, "bf16"), (3000, 256, 64, "bf16"),
+                                         (2000, 512, 128, "bf16"), (500, 48, 7, "f32")])
+def test_router_logits_equal_the_forward_logits(T, d, E, dtype):
+    moe = _moe()
+    k = min(4, E)
+    spec = inputs.LayerSpec("rl", T, d, 64, E, k, 1.0, dtype, router="normal", router_bias=0.5)
+    L = inputs.make_layer(spec, seed=T + d)
+    layer = moe.MoELayer(T, d, 64, E, k, 1.0, dtype)
+    args = [to_dev(L[n]) for n in ("x", "Wr", "br", "W1", "b1", "W2", "b2")]
+    _, rt = layer.forward(*args, want_routing=True)
+    lg = layer.router_logits(args[0], args[1], args[2])
+    torch.cuda.synchronize()
+    assert torch.equal(lg, rt["logits_out"])
+    ref = oracle.logits(L["x"], L["Wr"], L["br"])
+    assert np.abs(to_host(lg) - ref).max() <= 1e-4 * max(1.0, np.abs(ref).max())
+
+
+# ------------------------------------------------------------------------------------------
 # Routing-policy flags (renormalised weights, arrival-order capacity), bit for bit.
 # ------------------------------------------------------------------------------------------
 @pytest.mark.parametrize("flags", [1, 2, 3])
