@@ -70,6 +70,8 @@ struct GemmArgs {
     long long ldd;            // elements
     int router_E;             // router epilogue: number of experts (columns of D)
     DeviceStatus* st;
+    int32_t* zero;            // router: ints to clear (the dispatch counters), when its weight
+    int zero_n;               // split did not run in the same call (else null / 0)
     const void* W;            // B's base address (the L2 prefetch below)
     long long pf_bytes;       // > 0: before waiting for its predecessor, each CTA prefetches up
                               // to this many bytes of its first tile's weight rows into L2
@@ -438,6 +440,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
     const int n_tiles = args.n_tiles;
+    if constexpr (EPI == kEpiRouter) {
+        // The routing kernel after this one counts into these (the weight split clears them when
+        // it runs in the same call).
+        const int nthr = (int)(gridDim.x * blockDim.x);
+        for (int i = (int)(blockIdx.x * blockDim.x + threadIdx.x); i < args.zero_n; i += nthr)
+            args.zero[i] = 0;
+    }
     const int total = s_mt[E] * n_tiles;
     const int nkb = args.K / kBK;
     constexpr uint32_t kIdesc = idesc_bf16(C::kMmaM, BN);
@@ -1122,12 +1131,10 @@ size_t router_split_bytes(int d, int E) {
     return (size_t)ntl * 2 * Eg * d * 2;
 }
 
-cudaError_t launch_router_gemm(const void* x, int T, int d, const float* Wr, const float* br,
-                               int E, void* split_buf, float* logits, int32_t* zero, int zero_n,
-                               DeviceStatus* st, cudaStream_t s, int* launches) {
+void launch_router_split(const float* Wr, int d, int E, void* split_buf, int32_t* zero,
+                         int zero_n, cudaStream_t s, int* launches) {
     const int Eg = router_group(E);
     const int ntl = (E + Eg - 1) / Eg;
-    const int BN = 2 * Eg;
     const dim3 sg(d / kSplitK, ntl);
     __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(split_buf);
     if (Eg == 16)
@@ -1137,6 +1144,16 @@ cudaError_t launch_router_gemm(const void* x, int T, int d, const float* Wr, con
     else
         launch_pdl(router_split_kernel<64>, sg, dim3(256), 0, s, Wr, d, E, sb, zero, zero_n);
     *launches += 1;
+}
+
+cudaError_t launch_router_gemm(const void* x, int T, int d, const float* Wr, const float* br,
+                               int E, void* split_buf, bool prepared, float* logits,
+                               int32_t* zero, int zero_n, DeviceStatus* st, cudaStream_t s,
+                               int* launches) {
+    const int Eg = router_group(E);
+    const int ntl = (E + Eg - 1) / Eg;
+    const int BN = 2 * Eg;
+    if (!prepared) launch_router_split(Wr, d, E, split_buf, zero, zero_n, s, launches);
     CUtensorMap tm;
     if (!make_tmap(&tm, split_buf, (long long)ntl * BN, d, BN)) return cudaErrorInvalidValue;
     GemmArgs a{};
@@ -1157,6 +1174,8 @@ cudaError_t launch_router_gemm(const void* x, int T, int d, const float* Wr, con
     a.ldd = E;
     a.router_E = E;
     a.st = st;
+    a.zero = prepared ? zero : nullptr;
+    a.zero_n = prepared ? zero_n : 0;
     const long long tiles = (long long)((T + kBM - 1) / kBM) * ntl;
     CUtensorMap tmA;
     if (!make_tmap(&tmA, x, (long long)T, d, kBM)) return cudaErrorInvalidValue;

@@ -84,10 +84,15 @@ cudaError_t launch_expert_gemm(int which, const void* A, long long lda, const in
                                const void* W, const float* bias, void* D, long long ldd,
                                long long max_rows, DeviceStatus* st, cudaStream_t s,
                                int* launches);
-// Router logits L = x Wr + br [T, E] on the tensor cores (Wr split into two bf16 terms in
-// split_buf, router_split_bytes); also clears zero[0, zero_n) (the dispatch counters).
+// Router logits L = x Wr + br [T, E] on the tensor cores, from Wr split into two bf16 terms in
+// split_buf (router_split_bytes): split here, or already (prepared); either way zero[0, zero_n)
+// (the dispatch counters) is cleared.
 cudaError_t launch_router_gemm(const void* x, int T, int d, const float* Wr, const float* br,
-                               int E, void* split_buf, float* logits, int32_t* zero, int zero_n,
-                               DeviceStatus* st, cudaStream_t s, int* launches);
+                               int E, void* split_buf, bool prepared, float* logits,
+                               int32_t* zero, int zero_n, DeviceStatus* st, cudaStream_t s,
+                               int* launches);
+// The split alone (also clears zero[0, zero_n)).
+void launch_router_split(const float* Wr, int d, int E, void* split_buf, int32_t* zero,
+                         int zero_n, cudaStream_t s, int* launches);
 
 }  // namespace moe

@@ -31,7 +31,9 @@ bool bad_problem(const moe_problem* p) {
     if (p->k < 1 || p->k > p->E || p->k > 32) return true;
     if (std::isnan(p->capacity_factor) || p->capacity_factor < 0.0f) return true;
     if (p->dtype != MOE_F32 && p->dtype != MOE_BF16) return true;
-    if (p->flags & ~(MOE_FLAG_RENORMALIZE | MOE_FLAG_ARRIVAL_ORDER | MOE_FLAG_GATED)) return true;
+    if (p->flags & ~(MOE_FLAG_RENORMALIZE | MOE_FLAG_ARRIVAL_ORDER | MOE_FLAG_GATED |
+                     MOE_FLAG_ROUTER_PREPARED))
+        return true;
     if ((long long)p->T * p->k > 0x7fffffffLL) return true;
     if ((long long)p->T * p->E > 0x7fffffffLL) return true;
     return false;
@@ -343,6 +345,23 @@ moe_status moe_capacity_dispatch(const moe_problem* p, long long K, const int32_
     return finish(launches);
 }
 
+moe_status moe_prepare_router(const moe_problem* p, const float* Wr, void* ws, size_t ws_bytes,
+                              void* stream) {
+    moe_status r = pre(p, false);
+    if (r != MOE_OK) return r;
+    if (!Wr) return MOE_ERR_INVALID_ARG;
+    Plan q;
+    if ((r = check_ws(p, ws, ws_bytes, &q)) != MOE_OK) return r;
+    int launches = 0;
+    // Only the tensor-core router (bf16, more than 1024 tokens) reads the split.
+    if (p->dtype == MOE_BF16 && p->T > 0 && !moe::router_small_fits(p->T, p->E, p->d_model)) {
+        if (p->d_model % 64 != 0) return MOE_ERR_UNSUPPORTED;
+        moe::launch_router_split(Wr, p->d_model, p->E, at<void>(ws, q.split), nullptr, 0,
+                                 (cudaStream_t)stream, &launches);
+    }
+    return finish(launches);
+}
+
 moe_status moe_router_logits(const moe_problem* p, const void* x, const float* Wr,
                              const float* br, float* logits, void* ws, size_t ws_bytes,
                              void* stream) {
@@ -363,7 +382,8 @@ moe_status moe_router_logits(const moe_problem* p, const void* x, const float* W
     } else if (p->dtype == MOE_BF16) {
         if (p->d_model % 64 != 0) return MOE_ERR_UNSUPPORTED;
         if (moe::launch_router_gemm(x, p->T, p->d_model, Wr, br, p->E, at<void>(ws, q.split),
-                                    logits, nullptr, 0, at<moe::DeviceStatus>(ws, q.status), s,
+                                    (p->flags & MOE_FLAG_ROUTER_PREPARED) != 0, logits, nullptr,
+                                    0, at<moe::DeviceStatus>(ws, q.status), s,
                                     &launches) != cudaSuccess)
             return MOE_ERR_CUDA;
     } else {
@@ -481,7 +501,8 @@ moe_status moe_forward(const moe_problem* p, const void* x, const float* Wr, con
         if (!small_dispatch) moe::note_launch(cudaMemsetAsync(gcnt, 0, sizeof(int32_t) * (size_t)zero_n, s));
     } else if (p->dtype == MOE_BF16) {
         if (moe::launch_router_gemm(x, p->T, p->d_model, Wr, br, p->E, at<void>(ws, q.split),
-                                    logits, gcnt, zero_n, st, s, &launches) != cudaSuccess)
+                                    (p->flags & MOE_FLAG_ROUTER_PREPARED) != 0, logits, gcnt,
+                                    zero_n, st, s, &launches) != cudaSuccess)
             return MOE_ERR_CUDA;
     } else {
         moe::launch_logits_f32((const float*)x, Wr, br, p->T, p->d_model, p->E, logits, gcnt,

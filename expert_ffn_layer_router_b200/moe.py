@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 MOE_F32, MOE_BF16 = 0, 1
-FLAG_RENORMALIZE, FLAG_ARRIVAL_ORDER, FLAG_GATED = 1, 2, 4
+FLAG_RENORMALIZE, FLAG_ARRIVAL_ORDER, FLAG_GATED, FLAG_ROUTER_PREPARED = 1, 2, 4, 8
 MOE_OK = 0
 MOE_ERR_DEVICE = 5       # the status word holds an error (moe_get_device_status)
 DEV_OK, DEV_TIMEOUT, DEV_BAD_INDEX = 0, 1, 2
@@ -49,6 +49,7 @@ def _load():
         "moe_route": [P, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "moe_capacity_dispatch": [P, ctypes.c_int64] + [vp] * 8 + [sz, vp],
         "moe_router_logits": [P, vp, vp, vp, vp, vp, sz, vp],
+        "moe_prepare_router": [P, vp, vp, sz, vp],
         "moe_dispatch": [P, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "moe_expert_ffn": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "moe_combine": [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
@@ -76,7 +77,7 @@ EXPORTS = ("moe_capacity", "moe_workspace_size", "moe_route", "moe_dispatch", "m
            "moe_combine", "moe_forward", "moe_get_device_status", "moe_reset_device_status",
            "moe_last_launch_count", "moe_status_string", "moe_set_stage_events",
            "moe_route_static", "moe_selftest_wait_timeout", "moe_capacity_dispatch",
-           "moe_router_logits")
+           "moe_router_logits", "moe_prepare_router")
 
 STAGE_EVENTS = 7
 STAGE_NAMES = ("router_logits", "route_topk", "capacity_dispatch", "expert_gemm1",
@@ -143,6 +144,12 @@ def moe_capacity_dispatch(p, K, ids, w, slot, drop, counts, ws, offsets=None, ro
                                       _ptr(drop), _ptr(counts), _ptr(offsets), _ptr(rowtok),
                                       _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "moe_capacity_dispatch")
+
+
+def moe_prepare_router(p, Wr, ws, stream=None):
+    _check(_lib.moe_prepare_router(ctypes.byref(p), _ptr(Wr), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_prepare_router")
 
 
 def moe_router_logits(p, x, Wr, br, logits, ws, stream=None):
@@ -260,6 +267,12 @@ class MoELayer:
         moe_route(p, logits, r["ids"], r["w"], r["slot"], r["drop"], r["counts"], self.ws,
                   stream)
         return r
+
+    def prepare_router(self, Wr, stream=None):
+        """Splits Wr once into the workspace; later forwards skip the split (the problem's
+        MOE_FLAG_ROUTER_PREPARED is set).  Call again after Wr changes."""
+        self.p.flags |= FLAG_ROUTER_PREPARED
+        moe_prepare_router(self.p, Wr, self.ws, stream)
 
     def router_logits(self, x, Wr, br, stream=None):
         logits = torch.empty((self.p.T, self.p.E), dtype=torch.float32, device=x.device)

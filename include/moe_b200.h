@@ -95,6 +95,11 @@ typedef struct {
  * [0, d_ff) the gate, [d_ff, 2*d_ff) the up projection) and b1 [E, 2*d_ff]; the expert computes
  * a = SiLU(W1_gate x + b1_gate) * (W1_up x + b1_up), y = W2 a + b2.  bf16 needs d_ff % 128 == 0. */
 #define MOE_FLAG_GATED 4u
+/* Router weights prepared once: moe_forward skips splitting Wr into its two bfloat16 terms and
+ * reads the terms moe_prepare_router left in the workspace (bf16 batches above 1024 tokens; the
+ * other paths use Wr directly and ignore the flag).  The caller prepares again after Wr changes
+ * or after the workspace was used for another problem; with stale terms the logits are wrong. */
+#define MOE_FLAG_ROUTER_PREPARED 8u
 
 /* Host only.  Per-expert capacity K = min(T, floor(C * T * k / E)) evaluated in double
  * (worked example, capacity paragraph; generalised to k slots per token as in "Some Tokens Do
@@ -138,6 +143,14 @@ moe_status moe_capacity_dispatch(const moe_problem* p, long long K, const int32_
                                  const float* w, int32_t* slot, uint8_t* drop, int32_t* counts,
                                  int32_t* offsets, int32_t* rowtok, void* ws, size_t ws_bytes,
                                  void* stream);
+
+/* Splits Wr [d_model, E] float32 into the two bfloat16 terms the tensor-core router reads (hi =
+ * bf16(w), mid = bf16(w - hi)) and keeps them in ws, for moe_forward calls with
+ * MOE_FLAG_ROUTER_PREPARED on the same p and ws.  Weights are constant during inference, so the
+ * split need not be repeated per call.  A no-op for problems that do not use the tensor-core
+ * router (fp32, or at most 1024 tokens). */
+moe_status moe_prepare_router(const moe_problem* p, const float* Wr, void* ws, size_t ws_bytes,
+                              void* stream);
 
 /* Router logits alone, step 1's first half ("Dynamic Token Routing AI", How it works: the gating
  * network scores every token): logits [T, E] float32 = x Wr + br, with moe_forward's kernels, so

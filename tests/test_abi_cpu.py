@@ -94,10 +94,11 @@ def test_malformed_problems_rejected(moe, bad):
 
 def test_unknown_flags_rejected(moe):
     n = ctypes.c_size_t()
-    for bad in (8, 16, 0x80000000):
+    for bad in (16, 32, 0x80000000):
         p = moe.Problem(16, 64, 64, 4, 2, 1.0, 1, bad)
         assert moe.lib().moe_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 1
-    for good in (0, moe.FLAG_RENORMALIZE, moe.FLAG_ARRIVAL_ORDER, moe.FLAG_GATED, 7):
+    for good in (0, moe.FLAG_RENORMALIZE, moe.FLAG_ARRIVAL_ORDER, moe.FLAG_GATED,
+                 moe.FLAG_ROUTER_PREPARED, 15):
         p = moe.Problem(16, 64, 64, 4, 2, 1.0, 1, good)
         assert moe.lib().moe_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
 
@@ -130,3 +131,13 @@ def test_given_routing_and_logits_calls_reject_bad_arguments(moe):
     assert rl(ctypes.byref(bad), fake, fake, None, fake, fake, 1 << 20, None) == 1
     assert rl(ctypes.byref(p), fake, None, None, fake, fake, 1 << 20, None) == 1
     assert rl(ctypes.byref(p), fake, fake, None, fake, None, 0, None) == 3
+
+
+def test_prepare_router_rejects_bad_arguments(moe):
+    lib = moe.lib()
+    fake = ctypes.c_void_p(4096)
+    p = moe.Problem(2048, 64, 64, 8, 2, 1.0, 1, 0)
+    bad = moe.Problem(2048, 64, 64, 0, 2, 1.0, 1, 0)
+    assert lib.moe_prepare_router(ctypes.byref(bad), fake, fake, 1 << 30, None) == 1
+    assert lib.moe_prepare_router(ctypes.byref(p), None, fake, 1 << 30, None) == 1
+    assert lib.moe_prepare_router(ctypes.byref(p), fake, None, 0, None) == 3

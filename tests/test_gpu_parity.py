@@ -421,6 +421,37 @@ def test_router_logits_equal_the_forward_logits(T, d, E, dtype):
     assert np.abs(to_host(lg) - ref).max() <= 1e-4 * max(1.0, np.abs(ref).max())
 
 
+@pytest.mark.parametrize("T,d,E,k,C", [(3000, 256, 64, 6, 1.0), (2048, 512, 128, 8, 1.5),
+                                       (1500, 128, 16, 2, 1.25), (500, 128, 16, 2, 1.25)])
+def test_prepared_router_forward_equals_unprepared(T, d, E, k, C):
+    """moe_prepare_router once, then forwards with MOE_FLAG_ROUTER_PREPARED: the same logits,
+    routing and outputs, call after call, and again after the router weights change."""
+    moe = _moe()
+    spec = inputs.LayerSpec("prep", T, d, 128, E, k, C, "bf16", router="normal",
+                            router_bias=0.5, bias_std=0.05)
+    L = inputs.make_layer(spec, seed=T + E)
+    args = [to_dev(L[n]) for n in ("x", "Wr", "br", "W1", "b1", "W2", "b2")]
+
+    def same(a, b):
+        (oa, ra), (ob, rb) = a, b
+        assert torch.equal(oa.view(torch.int16), ob.view(torch.int16))
+        for key in ra:
+            assert torch.equal(ra[key], rb[key]), key
+
+    ref = moe.MoELayer(T, d, 128, E, k, C, "bf16")
+    layer = moe.MoELayer(T, d, 128, E, k, C, "bf16")
+    layer.prepare_router(args[1])
+    want = ref.forward(*args, want_routing=True)
+    same(layer.forward(*args, want_routing=True), want)
+    same(layer.forward(*args, want_routing=True), want)      # counters cleared every call
+    args2 = list(args)
+    args2[1] = args[1] * 1.5
+    layer.prepare_router(args2[1])
+    same(layer.forward(*args2, want_routing=True), ref.forward(*args2, want_routing=True))
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(layer.ws) == 0
+
+
 # ------------------------------------------------------------------------------------------
 # Routing-policy flags (renormalised weights, arrival-order capacity), bit for bit.
 # ------------------------------------------------------------------------------------------
