@@ -150,10 +150,11 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
 // the fp32 arithmetic is exactly route_token_warp's: m = max; u_e = exp(L_e - m); lane partials
 // added left to right; then the pairwise tree p[l] += p[l + h], h = 16, 8, 4, 2, 1 (shuffles down
 // within the group where l + h belongs to another lane), which adds the same pairs as the warp's
-// xor butterfly; top-k by (logit desc, expert asc); w = u / S.  A block of 8 warps routes 64
+// xor butterfly; top-k by (logit desc, expert asc); w = u / S.  A block of 16 warps routes 64
 // consecutive tokens and places their pairs (block counters in shared memory, one global atomic
 // per (block, expert)).
 constexpr int kGroupBlockTokens = 64;
+constexpr int kGroupWarps = 16;                        // one round of 4 tokens per warp (G = 8)
 
 // Per-expert histogram of the weight keys, built while routing: bin = bits 29..19 of the fp32
 // weight (weights are in [0, 1], so bit 30 is 0 and the bin grows with the weight: 7 exponent
@@ -164,14 +165,14 @@ __device__ __forceinline__ int hist_bin(float wv) {
 }
 
 template <int G>
-__global__ void __launch_bounds__(256) route_place_group_kernel(
+__global__ void __launch_bounds__(kGroupWarps * 32) route_place_group_kernel(
     const float* __restrict__ logits, int T, int E, int k, unsigned flags,
     int32_t* __restrict__ ids, float* __restrict__ w, int32_t* __restrict__ gcnt,
     int32_t* __restrict__ cand, uint32_t* __restrict__ hist, DeviceStatus* st) {
     pdl_begin();
     constexpr int LPL = 32 / G;                        // warp-router lanes per group lane
     constexpr int NI = G / 4;                          // experts per warp-router lane: E <= 32 NI
-    constexpr int TPW = kGroupBlockTokens / 8;         // tokens per warp
+    constexpr int TPW = kGroupBlockTokens / kGroupWarps;   // tokens per warp
     constexpr int TPP = 32 / G;                        // tokens per warp per round
     constexpr int R = TPW / TPP;                       // rounds
     __shared__ int s_n[32 * NI], s_base[32 * NI];
@@ -1013,14 +1014,14 @@ void launch_route_place(const float* logits, int T, int E, int k, unsigned flags
     if (G > 0) {
         const dim3 g((T + kGroupBlockTokens - 1) / kGroupBlockTokens);
         if (G == 8)
-            launch_pdl(route_place_group_kernel<8>, g, dim3(256), 0, s, logits, T, E, k, flags,
-                       ids, w, gcnt, cand, hist, st);
+            launch_pdl(route_place_group_kernel<8>, g, dim3(kGroupWarps * 32), 0, s, logits, T, E,
+                       k, flags, ids, w, gcnt, cand, hist, st);
         else if (G == 16)
-            launch_pdl(route_place_group_kernel<16>, g, dim3(256), 0, s, logits, T, E, k, flags,
-                       ids, w, gcnt, cand, hist, st);
+            launch_pdl(route_place_group_kernel<16>, g, dim3(kGroupWarps * 32), 0, s, logits, T, E,
+                       k, flags, ids, w, gcnt, cand, hist, st);
         else
-            launch_pdl(route_place_group_kernel<32>, g, dim3(256), 0, s, logits, T, E, k, flags,
-                       ids, w, gcnt, cand, hist, st);
+            launch_pdl(route_place_group_kernel<32>, g, dim3(kGroupWarps * 32), 0, s, logits, T, E,
+                       k, flags, ids, w, gcnt, cand, hist, st);
     } else {
         const dim3 g((T + kWarpRouteTokens - 1) / kWarpRouteTokens);
         const size_t smem = 2 * sizeof(int) * (size_t)E;
