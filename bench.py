@@ -497,6 +497,7 @@ def run_cuda(args):
                                    "router_fused": fused},
         "kernels": kernels,
         "step_ms_min": float(step_ms.min()), "step_ms_median": float(np.median(step_ms)),
+        "step_ms_each": [round(float(v), 4) for v in step_ms],
         "instrumented_ms_per_step": float(instr_ms.mean()),
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
