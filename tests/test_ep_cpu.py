@@ -26,3 +26,15 @@ def test_expert_parallel_matches_single_batch(cfg):
     mp.start_processes(ep_worker.cpu_rank, args=(2, port, cfg, out), nprocs=2,
                        start_method="spawn")
     assert out[0] == [] and out[1] == [], (out[0], out[1])
+
+
+@pytest.mark.parametrize("cfg", [
+    (16, 16, 24, 8, 2, 0.75, "f32", 0, 11),      # two experts per rank, drops
+    (12, 8, 16, 4, 2, 1.0, "bf16", 2, 12)])      # one expert per rank, arrival order
+def test_expert_parallel_four_ranks(cfg):
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    port = 29640 + cfg[-1]
+    mp.start_processes(ep_worker.cpu_rank, args=(4, port, cfg, out), nprocs=4,
+                       start_method="spawn")
+    assert all(out[r] == [] for r in range(4)), dict(out)
