@@ -422,12 +422,12 @@ def run_cuda(args):
     # batches with the single-block dispatch (T <= 1024, T k <= 1024) compute logits and routing
     # in one launch: the router stage reads x and Wr and writes ids and weights, and the top-k
     # stage is empty.  Otherwise the logits round-trip through HBM between the two stages.
-    fused = (spec.dtype == "bf16" and T <= 1024 and E <= 256 and dm <= 12288
+    router_routes = (spec.dtype == "bf16" and T <= 1024 and E <= 256 and dm <= 12288
              and T * k <= 1024)
-    router_out = T * k * 8 if fused else T * E * 4
+    router_out = T * k * 8 if router_routes else T * E * 4
     by = {
         "router_logits": dict(flop=2.0 * T * dm * E, bytes=T * dm * esz + dm * E * 4 + router_out),
-        "route_topk": dict(bytes=0 if fused else T * E * 4 + T * k * 8),
+        "route_topk": dict(bytes=0 if router_routes else T * E * 4 + T * k * 8),
         "capacity_dispatch": dict(bytes=T * k * 8 + T * k * 5 + kept * 4 + E * 16),
         "expert_gemm1": dict(flop=g1_flop,
                              bytes=T * dm * esz + E * F * dm * esz * (2 if spec.gated else 1)
@@ -494,7 +494,7 @@ def run_cuda(args):
         "route_dispatch_combine": {"gbs": rdc_gbs, "frac_of_hbm": rdc_gbs / pk["hbm_gbs"],
                                    "bytes_per_step": rdc_bytes, "hbm_peak_gbs": pk["hbm_gbs"],
                                    "stages": list(rdc_stages),
-                                   "router_fused": fused},
+                                   "router_stage_routes": router_routes},
         "kernels": kernels,
         "step_ms_min": float(step_ms.min()), "step_ms_median": float(np.median(step_ms)),
         "step_ms_each": [round(float(v), 4) for v in step_ms],

@@ -195,7 +195,7 @@ moe_status ffn_steps(const moe_problem* p, const void* x, const int32_t* offsets
 // that owns all device memory and gives its plug-ins no allocator, and latency-bound serving
 // loops whose policy forbids cudaMalloc/cudaFree on the request path (an allocation can
 // synchronise the device and stall every stream).  This entry point runs the same router and
-// capacity kernels as moe_route, with their scratch (per-chunk counts and prefixes, per-expert
+// capacity kernels as moe_route, with their scratch (per-expert counters and weight histograms,
 // candidate lists, the status word) placed in one file-scope __device__ array below.
 //
 // The array is a fixed kRouteStaticBytes per GPU, held by every GPU that loads the library until

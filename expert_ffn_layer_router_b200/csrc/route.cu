@@ -732,7 +732,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
 
 // ---------------------------------------------------------------------------------------------
 // Small batches (T*k <= kSmallPairs): counting, capacity selection, slots, offsets and the row
-// map in one block, one launch.  Same results as the chunked pipeline above: candidates of an
+// map in one block, one launch.  Same results as the two-launch dispatch above: candidates of an
 // expert are kept in ascending token order (warp-serial stable placement), an overflowing
 // expert keeps its K pairs of largest (weight, then lower token) -- or its first K with
 // MOE_FLAG_ARRIVAL_ORDER -- and slots rank the kept tokens in ascending token order.
