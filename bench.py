@@ -450,7 +450,26 @@ def run_cuda(args):
     tensor_peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
     g1, g2 = kernels["expert_gemm1"], kernels["expert_gemm2"]
     dom = "expert_gemm1" if g1["ms"] >= g2["ms"] else "expert_gemm2"
-    achieved = kernels[dom]["tflops"]
+    # The dominant kernel's bound: tensor cores when its flops per algorithmic byte exceed the
+    # ridge point of the two peaks (cfg3: ~780 flop/B against a ridge of ~210), HBM otherwise
+    # (decode: each expert's weights serve ~8 rows, ~8 flop/B).
+    ridge = tensor_peak * 1e12 / (pk["hbm_gbs"] * 1e9)
+    hbm_bound = by[dom]["flop"] / by[dom]["bytes"] < ridge
+    if hbm_bound:
+        roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gbs"],
+                    "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": kernels[dom]["gbs"] / pk["hbm_gbs"] if kernels[dom]["gbs"] else None,
+                    "peak_source": "%s hbm_gbs (copy bandwidth)" % pk_kind,
+                    "algorithmic_bytes_per_launch": by[dom]["bytes"]}
+    else:
+        achieved = kernels[dom]["tflops"]
+        roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved,
+                    "peak": tensor_peak, "unit": "TFLOP/s",
+                    "frac": achieved / tensor_peak if achieved else None,
+                    "peak_source": "%s bf16_tflops_sustained (kernel timed inside a long"
+                                   " loop of steps)" % pk_kind,
+                    "algorithmic_flop_per_launch": by[dom]["flop"]}
+    roofline["traffic"] = traffic_record(dom, traffic_key)
     gemm_ms = g1["ms"] + g2["ms"]
     gemm_tflops = (g1_flop + gemm_flop_each) / (gemm_ms * 1e-3) / 1e12
     rdc_stages = ("router_logits", "route_topk", "capacity_dispatch", "combine")
@@ -482,12 +501,7 @@ def run_cuda(args):
                 "ms_per_step": e2e_ms / K,
                 "pipeline": "copy-in / compute / copy-out streams, double-buffered device x and"
                             " out; pinned host buffers"},
-        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved,
-                     "peak": tensor_peak, "unit": "TFLOP/s",
-                     "frac": achieved / tensor_peak if achieved else None,
-                     "peak_source": "%s bf16_tflops_sustained (kernel timed inside a long"
-                                    " loop of steps)" % pk_kind,
-                     "traffic": traffic_record(dom, traffic_key)},
+        "roofline": roofline,
         "expert_gemm": {"tflops": gemm_tflops, "frac_of_peak": gemm_tflops / tensor_peak,
                         "frac_of_burst_peak": gemm_tflops / pk.get("bf16_tflops", tensor_peak),
                         "flop_per_step": g1_flop + gemm_flop_each},
