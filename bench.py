@@ -53,6 +53,13 @@ def parse():
                     help="override the workload's token count (profiling of smaller cases)")
     ap.add_argument("--gated", action="store_true",
                     help="gated experts (SiLU(gate) * up, W1 twice as tall) on the same shapes")
+    ap.add_argument("--drop-policy", default="weight", choices=["weight", "arrival"],
+                    help="capacity selection: lowest router weight dropped first (default) or"
+                         " the first K pairs of each expert in token order kept")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert-parallel layer: experts split over the ranks, NCCL all-to-all")
+    ap.add_argument("--renormalize", action="store_true",
+                    help="top-k weights renormalised to sum to 1 before the capacity selection")
     return ap.parse_args()
 
 
@@ -76,17 +83,27 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def workload_desc(spec):
+def layer_flags(spec, args):
+    """The layer's flag word (same bit values in the library and the oracle): 1 renormalised
+    top-k weights, 2 arrival-order capacity, 4 gated experts."""
+    return ((1 if getattr(args, "renormalize", False) else 0)
+            | (2 if getattr(args, "drop_policy", "weight") == "arrival" else 0)
+            | (4 if spec.gated else 0))
+
+
+def workload_desc(spec, flags=0):
     C = "dropless" if math.isinf(spec.C) else "C=%g" % spec.C
-    return "%s: T=%d, d_model=%d, d_ff=%d, E=%d, top-%d, %s, %s%s" % (
+    return "%s: T=%d, d_model=%d, d_ff=%d, E=%d, top-%d, %s, %s%s%s%s" % (
         spec.name, spec.T, spec.d_model, spec.d_ff, spec.E, spec.k, C, spec.dtype,
-        ", gated experts" if spec.gated else "")
+        ", gated experts" if spec.gated else "",
+        ", arrival-order capacity" if flags & 2 else "",
+        ", renormalised top-k weights" if flags & 1 else "")
 
 
 # ------------------------------------------------------------------------------------------------
 # CPU oracle timing (the reference arm and the cpu_baseline object)
 # ------------------------------------------------------------------------------------------------
-def oracle_step(L, spec, sample, nthreads):
+def oracle_step(L, spec, sample, nthreads, flags=0):
     """Time the oracle on one bounded sample; returns (seconds extrapolated to T tokens, info)."""
     import oracle
     T = spec.T
@@ -101,10 +118,11 @@ def oracle_step(L, spec, sample, nthreads):
     full = L["_full_logits"]
     t0 = time.perf_counter()
     K = oracle.capacity(T, spec.E, spec.k, spec.C)
-    r = oracle.route(full, spec.k, K)
+    r = oracle.route(full, spec.k, K, flags & (oracle.RENORMALIZE | oracle.ARRIVAL_ORDER))
     t_route = time.perf_counter() - t0
     t0 = time.perf_counter()
-    oracle.combine_tokens(L["x"], L["W1"], L["b1"], L["W2"], L["b2"], r, toks, nthreads)
+    oracle.combine_tokens(L["x"], L["W1"], L["b1"], L["W2"], L["b2"], r, toks, nthreads,
+                          flags=flags & oracle.GATED)
     t_ffn = time.perf_counter() - t0
     del Ls
     est = (t_logits + t_ffn) * T / sample + t_route
@@ -120,10 +138,10 @@ def prepare_oracle_inputs(L, spec, nthreads):
         L["_full_logits"] = oracle.logits(L["x"], L["Wr"], L["br"], nthreads)
 
 
-def calibrate_sample(L, spec, target_s, nthreads):
+def calibrate_sample(L, spec, target_s, nthreads, flags=0):
     """Tokens per sample so that one oracle step takes about target_s seconds."""
     s = max(1, min(spec.T, 8))
-    est, info = oracle_step(L, spec, s, nthreads)
+    est, info = oracle_step(L, spec, s, nthreads, flags)
     per_tok = max((info["t_logits"] + info["t_ffn"]) / s, 1e-6)
     budget = max(target_s - info["t_route"], 0.05)
     return int(max(1, min(spec.T, budget / per_tok)))
@@ -136,21 +154,32 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
+def bench_spec(args):
+    """The workload of this run: the named configuration with --tokens and --gated applied."""
+    spec = inputs.CONFIGS[args.config]
+    if args.tokens:
+        spec = dataclasses.replace(spec, T=args.tokens)
+    if args.gated:
+        spec = dataclasses.replace(spec, gated=True)
+    return spec
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    spec = inputs.CONFIGS[args.config]
+    spec = bench_spec(args)
+    flags = layer_flags(spec, args)
     L = inputs.make_layer(spec, seed=args.seed)
     cores = cpu_cores()
     prepare_oracle_inputs(L, spec, cores)
     step_budget = max(0.2, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
-    sample = calibrate_sample(L, spec, step_budget, cores)
+    sample = calibrate_sample(L, spec, step_budget, cores, flags)
     for _ in range(args.warmup):
-        oracle_step(L, spec, sample, cores)
+        oracle_step(L, spec, sample, cores, flags)
     ests, meas = [], []
     for _ in range(args.steps):
-        est, info = oracle_step(L, spec, sample, cores)
+        est, info = oracle_step(L, spec, sample, cores, flags)
         ests.append(est)
         meas.append(info["measured"])
     t = statistics.mean(ests)
@@ -161,7 +190,7 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": workload_desc(spec), "seed": args.seed},
+            "config": {"workload": workload_desc(spec, flags), "seed": args.seed},
             "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": desc, "value": value,
                              "unit": "tokens/s"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -280,14 +309,11 @@ def run_cuda(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
 
-    spec = inputs.CONFIGS[args.config]
-    if args.tokens:
-        spec = dataclasses.replace(spec, T=args.tokens)
-    if args.gated:
-        spec = dataclasses.replace(spec, gated=True)
+    spec = bench_spec(args)
+    flags = layer_flags(spec, args)
     L = inputs.make_layer(spec, seed=args.seed + rank)
     layer = moe.MoELayer(spec.T, spec.d_model, spec.d_ff, spec.E, spec.k, spec.C, spec.dtype,
-                         device=dev, flags=moe.FLAG_GATED if spec.gated else 0)
+                         device=dev, flags=flags)
     names = ("x", "Wr", "br", "W1", "b1", "W2", "b2")
     d = {n: to_dev(L[n], torch, dev) for n in names}
     # The router weights are constant: their two bf16 terms are formed once, as a serving
@@ -438,7 +464,7 @@ def run_cuda(args):
     }
     input_bytes = sum(int(t.numel() * t.element_size()) for t in d.values() if t is not None)
     traffic_key = spec.name + (" gated" if spec.gated else "") + \
-        (" T=%d" % spec.T if args.tokens else "")
+        (" T=%d" % spec.T if args.tokens else "") + (" flags=%d" % (flags & 3) if flags & 3 else "")
     kernels = {}
     for i, n in enumerate(names6):
         ms = float(st_avg[i])
@@ -481,7 +507,7 @@ def run_cuda(args):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if spec.dtype == "bf16" else "f32",
         "data": "synthetic (seeded numpy draws; random-init weights of the stated shape)",
-        "config": {"workload": workload_desc(spec), "seed": args.seed + rank,
+        "config": {"workload": workload_desc(spec, flags), "seed": args.seed + rank,
                    "per_rank_tokens": T, "parallelism": "dp%d (independent batches)" % world,
                    "l2": "flushed before every timed step (256 MiB write, outside the step's"
                          " events); per-step inputs %.0f MB" % (input_bytes / 1e6),
@@ -517,8 +543,8 @@ def run_cuda(args):
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         cores = cpu_cores()
         prepare_oracle_inputs(L, spec, cores)
-        sample = calibrate_sample(L, spec, max(1.0, args.cpu_seconds / 3), cores)
-        ests = [oracle_step(L, spec, sample, cores)[0] for _ in range(3)]
+        sample = calibrate_sample(L, spec, max(1.0, args.cpu_seconds / 3), cores, flags)
+        ests = [oracle_step(L, spec, sample, cores, flags)[0] for _ in range(3)]
         cv = spec.T / statistics.mean(ests)
         line["cpu_baseline"] = {
             "value": cv, "unit": "tokens/s", "cores": cores, "kind": "oracle",
@@ -532,10 +558,113 @@ def run_cuda(args):
     return 0
 
 
+def run_ep(args):
+    """--ep: the expert-parallel layer (expert_ffn_layer_router_b200/ep.py).  Every rank routes its
+    own T tokens and owns E/N experts; candidates, x rows and expert outputs cross ranks by NCCL
+    all-to-all.  The capacity is that of the whole N*T-token batch, so the result equals one
+    device running the union of the batches.  Timed like the default mode (flush, events, max
+    over ranks); value = N*T / step time."""
+    import torch
+    import torch.distributed as dist
+
+    from expert_ffn_layer_router_b200 import moe
+    from expert_ffn_layer_router_b200.ep import ExpertParallelLayer
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d" % (args.gpus, world))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29533")
+    dist.init_process_group("nccl", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=300), device_id=dev)
+    spec = bench_spec(args)
+    flags = layer_flags(spec, args)
+    if spec.E % world:
+        raise SystemExit("--ep needs E (%d) to be a multiple of the number of GPUs" % spec.E)
+    T = spec.T
+    # One global layer of world*T tokens: rank r holds tokens [rT, (r+1)T) and experts
+    # [r E/N, (r+1) E/N).
+    L = inputs.make_layer(dataclasses.replace(spec, T=world * T), seed=args.seed)
+    El = spec.E // world
+    ts, es = slice(rank * T, (rank + 1) * T), slice(rank * El, (rank + 1) * El)
+    d = {"x": to_dev(L["x"][ts], torch, dev), "Wr": to_dev(L["Wr"], torch, dev),
+         "br": to_dev(L["br"], torch, dev)}
+    for n in ("W1", "b1", "W2", "b2"):
+        d[n] = to_dev(L[n][es], torch, dev)
+    del L
+    ep = ExpertParallelLayer(dist.group.WORLD, T, spec.d_model, spec.d_ff, spec.E, spec.k, spec.C,
+                             spec.dtype, dev, flags)
+    ep.steps.router.prepare_router(d["Wr"])
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        return ep.forward(d["x"], d["Wr"], d["br"], d["W1"], d["b1"], d["W2"], d["b2"])
+
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    sampler.start()
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    for row in evs:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    l0 = ep.steps.launches
+    for i in range(K):
+        flush.zero_()
+        evs[i][0].record(stream)
+        out, r = step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks = sampler.stop()
+    launches = ep.steps.launches - l0
+    step_ms = np.array([evs[i][0].elapsed_time(evs[i][1]) for i in range(K)])
+    total_ms = max_over_ranks(float(step_ms.sum()), dist if world > 1 else None, dev)
+    ms_per_step = total_ms / K
+    kept = int((r["slot"] >= 0).sum().item())
+    line = {
+        "metric": METRIC, "value": world * T / (ms_per_step / 1e3), "unit": "tokens/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if spec.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded numpy draws; random-init weights of the stated shape)",
+        "mode": "expert-parallel",
+        "config": {"workload": workload_desc(spec, flags), "seed": args.seed,
+                   "per_rank_tokens": T, "experts_per_rank": El,
+                   "parallelism": "ep%d (experts split over ranks; candidates, x rows and expert"
+                                  " outputs by NCCL all-to-all; the whole batch's capacity)" % world,
+                   "l2": "flushed before every timed step (256 MiB write, outside the step's"
+                         " events)",
+                   "kept_pairs_of_rank0_tokens": kept},
+        "gpu_launches": launches,
+        "gpu_launches_per_step": launches / K,
+        "clocks": clocks,
+        "step_ms_min": float(step_ms.min()), "step_ms_median": float(np.median(step_ms)),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.ep:
+        return run_ep(args)
     return run_cuda(args)
 
 

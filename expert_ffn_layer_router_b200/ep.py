@@ -18,8 +18,10 @@ batch:
 5. the owner runs the expert FFN on the rows it received (moe_expert_ffn);
 6. the expert rows go back and each source combines its tokens (moe_combine).
 
-Transfers are torch.distributed all-to-alls (NCCL over NVLink on GPUs, gloo on CPU); their split
-sizes are exchanged first, so the forward synchronises the host once per exchange.  Every compute
+Transfers are torch.distributed all-to-alls (NCCL over NVLink on GPUs, gloo on CPU).  Their
+split sizes must be known on the host, so the forward synchronises the host twice: once for the
+candidate counts per owner and once for the kept-row counts; all later sizes follow from those.
+With one rank every exchange is the identity and copies nothing.  Every compute
 step runs in the library's kernels; the plumbing between them (grouping pairs by destination,
 index bookkeeping) uses torch tensor operations.  The compute steps are methods of one object
 (`CudaSteps` here), so the exchange logic can be checked on CPU ranks against the oracle with the
@@ -34,16 +36,36 @@ from . import moe
 
 
 def _a2a(send, send_counts, recv_counts, group):
-    """all_to_all_single along dim 0 with the given per-rank row counts (python lists)."""
+    """all_to_all_single along dim 0 with the given per-rank row counts (python lists).  With one
+    rank the exchange is the identity and nothing is copied."""
+    if dist.get_world_size(group) == 1:
+        return send
     out = send.new_empty((sum(recv_counts),) + tuple(send.shape[1:]))
     dist.all_to_all_single(out, send.contiguous(), recv_counts, send_counts, group=group)
     return out
 
 
 def _a2a_counts(send_counts, group):
+    if dist.get_world_size(group) == 1:
+        return send_counts
     recv = torch.empty_like(send_counts)
     dist.all_to_all_single(recv, send_counts.contiguous(), group=group)
     return recv
+
+
+def _group_order(dest, world):
+    """Positions 0..P-1 grouped by destination rank, ascending within each group (a stable
+    counting sort), and the group sizes."""
+    P = dest.numel()
+    if P == 0:
+        return dest.clone(), torch.zeros(world, dtype=torch.int64, device=dest.device)
+    csum = torch.cumsum(torch.nn.functional.one_hot(dest, world), dim=0)   # [P, world]
+    counts = csum[-1]
+    rank_in = csum.gather(1, dest.view(-1, 1)).view(-1) - 1
+    pos = (torch.cumsum(counts, 0) - counts)[dest] + rank_in
+    order = torch.empty_like(dest)
+    order[pos] = torch.arange(P, dtype=dest.dtype, device=dest.device)
+    return order, counts
 
 
 class CudaSteps:
@@ -65,6 +87,10 @@ class CudaSteps:
         self.sel_ws = self._ws(self._sel_problem(self.cand_max))
         self.ffn_ws = self._ws(self._ffn_problem(self.rows_max))
         self.comb_ws = torch.zeros(32, dtype=torch.int64, device=self.device)
+        self.launches = 0           # kernels this object's calls launched (moe_last_launch_count)
+
+    def _count(self):
+        self.launches += moe.moe_last_launch_count()
 
     def _ws(self, p):
         n = moe.moe_workspace_size(p)
@@ -80,7 +106,9 @@ class CudaSteps:
 
     def route(self, x, Wr, br):
         logits = self.router.router_logits(x, Wr, br)
+        self._count()
         r = self.router.route(logits)
+        self._count()
         return r["ids"], r["w"]
 
     def select(self, e_v, w_v, K):
@@ -95,6 +123,7 @@ class CudaSteps:
                              device=dev)
         moe.moe_capacity_dispatch(self._sel_problem(n), K, e_v.view(n, 1), w_v.view(n, 1), slot,
                                   drop, counts, self.sel_ws, offsets, rowtok)
+        self._count()
         return slot.view(n), offsets, rowtok
 
     def expert_ffn(self, x_rows, offsets, rowtok, W1, b1, W2, b2):
@@ -103,6 +132,7 @@ class CudaSteps:
         if n > 0:
             moe.moe_expert_ffn(self._ffn_problem(n), x_rows, offsets, rowtok, W1, b1, W2, b2, Y,
                                self.ffn_ws)
+            self._count()
         return Y[:n]
 
     def combine(self, x, Y_back, w, slot_back):
@@ -117,6 +147,7 @@ class CudaSteps:
         Y = Y_back if m > 0 else torch.zeros((1, self.d_model), dtype=x.dtype, device=x.device)
         out = torch.empty_like(x)
         moe.moe_combine(p, x, Y, w, ids, slot_back, offsets, out, self.comb_ws)
+        self._count()
         return out
 
 
@@ -154,8 +185,7 @@ class ExpertParallelLayer:
         P = T * k
         ids_f = ids.reshape(P).to(torch.int64)
         dest = ids_f // El                                             # owner of each pair
-        order = torch.argsort(dest, stable=True)                       # grouped by owner
-        send_cnt = torch.bincount(dest, minlength=world)
+        order, send_cnt = _group_order(dest, world)                    # grouped by owner
         recv_cnt = _a2a_counts(send_cnt, g)
         sc, rc = send_cnt.tolist(), recv_cnt.tolist()
         # Candidates: (local expert, weight), in each source's pair (= token) order.
@@ -166,27 +196,31 @@ class ExpertParallelLayer:
         slot_sent = _a2a(slot_v, rc, sc, g)
         slot = torch.empty(P, dtype=torch.int32, device=dev)
         slot[order] = slot_sent
-        # x rows of the kept pairs to their owners.
+        # x rows of the kept pairs to their owners.  The only host synchronisations of the
+        # forward are the two count exchanges; every index below has a size known from them, so
+        # no boolean mask is materialised on the host's behalf (nonzero_static).
         kept_sent = slot_sent >= 0
-        kcnt_send = torch.bincount(dest[order][kept_sent], minlength=world)
+        kcnt_send = torch.zeros(world, dtype=torch.int64, device=dev).scatter_add_(
+            0, dest[order], kept_sent.to(torch.int64))
         kcnt_recv = _a2a_counts(kcnt_send, g)
         ks, kr = kcnt_send.tolist(), kcnt_recv.tolist()
-        tok_sent = torch.div(order[kept_sent], k, rounding_mode="floor")
+        n_sent, n_rows = sum(ks), sum(kr)                              # kept rows sent, received
+        at_sent = order[torch.nonzero_static(kept_sent, size=n_sent).view(-1)]
+        tok_sent = torch.div(at_sent, k, rounding_mode="floor")
         x_rows = _a2a(x[tok_sent], ks, kr, g)
         # The owner's expert-sorted rows: row offsets[e] + slot holds the kept candidate whose
         # rank among the kept candidates (in arrival order) is the index of its x row.
         kept_v = slot_v >= 0
         kept_rank = torch.cumsum(kept_v.to(torch.int32), 0, dtype=torch.int32) - 1
-        n_rows = int(kept_v.sum().item())
         rowtok = kept_rank[rowtok_v[:n_rows].to(torch.int64)]
         Y = self.steps.expert_ffn(x_rows, offsets, rowtok, W1, b1, W2, b2)
         # Expert rows back, in the order the x rows came.
-        e_kept = e_v[kept_v].to(torch.int64)
-        rows_back = offsets[:-1].to(torch.int64)[e_kept] + slot_v[kept_v].to(torch.int64)
+        at_v = torch.nonzero_static(kept_v, size=n_rows).view(-1)
+        rows_back = offsets[:-1].to(torch.int64)[e_v[at_v].to(torch.int64)] + \
+            slot_v[at_v].to(torch.int64)
         Y_back = _a2a(Y[rows_back], kr, ks, g)
         slot_back = torch.full((P,), -1, dtype=torch.int32, device=dev)
-        slot_back[order[kept_sent]] = torch.arange(int(kept_sent.sum().item()),
-                                                   dtype=torch.int32, device=dev)
+        slot_back[at_sent] = torch.arange(n_sent, dtype=torch.int32, device=dev)
         out = self.steps.combine(x, Y_back, w, slot_back.view(T, k))
         slot = slot.view(T, k)
         return out, dict(ids=ids, w=w, slot=slot, drop=(slot < 0).to(torch.uint8))

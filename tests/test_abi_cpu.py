@@ -141,3 +141,19 @@ def test_prepare_router_rejects_bad_arguments(moe):
     assert lib.moe_prepare_router(ctypes.byref(bad), fake, fake, 1 << 30, None) == 1
     assert lib.moe_prepare_router(ctypes.byref(p), None, fake, 1 << 30, None) == 1
     assert lib.moe_prepare_router(ctypes.byref(p), fake, None, 0, None) == 3
+
+
+def test_bench_flag_word_matches_library_and_oracle(moe):
+    """bench.py builds one flag word for the library and the oracle; the bits must mean the same
+    thing on both sides."""
+    import argparse
+    import dataclasses
+    import bench
+    spec = inputs.CONFIGS["skewed_e64_top6"]
+    ns = argparse.Namespace(renormalize=True, drop_policy="arrival")
+    f = bench.layer_flags(dataclasses.replace(spec, gated=True), ns)
+    assert f == moe.FLAG_RENORMALIZE | moe.FLAG_ARRIVAL_ORDER | moe.FLAG_GATED
+    assert f == oracle.RENORMALIZE | oracle.ARRIVAL_ORDER | oracle.GATED
+    assert bench.layer_flags(spec, argparse.Namespace(renormalize=False, drop_policy="weight")) == 0
+    desc = bench.workload_desc(spec, f)
+    assert "arrival-order capacity" in desc and "renormalised top-k weights" in desc

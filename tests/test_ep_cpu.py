@@ -38,3 +38,16 @@ def test_expert_parallel_four_ranks(cfg):
     mp.start_processes(ep_worker.cpu_rank, args=(4, port, cfg, out), nprocs=4,
                        start_method="spawn")
     assert all(out[r] == [] for r in range(4)), dict(out)
+
+
+def test_group_order_is_a_stable_sort_by_destination():
+    """The exchange groups pairs by owner with a counting sort; it must equal a stable sort."""
+    import torch
+    from expert_ffn_layer_router_b200 import ep
+    g = torch.Generator().manual_seed(1)
+    for world in (1, 2, 3, 8, 64):
+        for P in (0, 1, 31, 5000):
+            dest = torch.randint(0, world, (P,), generator=g)
+            order, counts = ep._group_order(dest, world)
+            assert torch.equal(order, torch.argsort(dest, stable=True))
+            assert torch.equal(counts, torch.bincount(dest, minlength=world))
