@@ -21,8 +21,9 @@
 //            tokens are marked in a bitmap over the batch, whose prefix popcounts give each kept
 //            pair its slot (its rank in token order), so the result does not depend on the list
 //            order.
-// The counters and histograms must be zero when the route kernel starts; the kernel before it
-// in the same call clears them (the router's weight split, the fp32 logits kernel, or a memset).
+// The counters and histograms must be zero when the route kernel starts; a launch before it in
+// the same call clears them (the router's weight split, the router GEMM itself when the split was
+// prepared beforehand, the fp32 logits kernel, or a memset).
 #include <atomic>
 #include <cfloat>
 #include <cstdint>
