@@ -1,0 +1,76 @@
+"""Random small layers (hypothesis, derandomised): moe_forward against the oracle.
+
+Each example draws a layer shape, a capacity factor and the flag word, and checks what holds
+for every layer: the routing (ids, weight bits, slots, drop mask, counts) equals the oracle's
+routing of the forward's own fp32 logits bit for bit, the expert offsets are the prefix sums
+of the kept counts, every output row is within the dtype's tolerance of the oracle's layer, and
+a token whose pairs were all dropped leaves bit for bit as it came in.  Shapes span the
+small-batch and large-batch router and dispatch paths (T*k on both sides of 1024, T on both
+sides of 1024 for the bf16 router).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+from hypothesis import HealthCheck, given, settings
+from hypothesis import strategies as st
+
+import oracle
+from expert_ffn_layer_router_b200 import inputs
+from tests.gpu_util import assert_close, to_dev, to_host
+
+pytestmark = pytest.mark.gpu
+
+
+@st.composite
+def layers(draw):
+    T = draw(st.one_of(st.integers(1, 700), st.integers(1025, 2600)))
+    E = draw(st.integers(1, 40))
+    k = draw(st.integers(1, min(E, 8)))
+    d = draw(st.sampled_from([64, 128, 192]))
+    F = draw(st.sampled_from([64, 128, 320]))
+    C = draw(st.sampled_from([0.0, 0.5, 1.0, 1.25, 2.0, math.inf]))
+    flags = draw(st.integers(0, 7))
+    dtype = draw(st.sampled_from(["bf16", "bf16", "f32"]))
+    seed = draw(st.integers(0, 2 ** 16))
+    spec = inputs.LayerSpec("h", T, d, F, E, k, C, dtype, router="normal", router_bias=0.5,
+                            bias_std=0.05, gated=bool(flags & 4))
+    return spec, flags, seed
+
+
+@settings(max_examples=100, deadline=None, derandomize=True, print_blob=True,
+          suppress_health_check=[HealthCheck.too_slow, HealthCheck.data_too_large])
+@given(layers())
+def test_forward_random_layers(case):
+    from expert_ffn_layer_router_b200 import moe
+    spec, flags, seed = case
+    L = inputs.make_layer(spec, seed=seed)
+    layer = moe.MoELayer(spec.T, spec.d_model, spec.d_ff, spec.E, spec.k, spec.C, spec.dtype,
+                         flags=flags)
+    args = [to_dev(L[n]) for n in ("x", "Wr", "br", "W1", "b1", "W2", "b2")]
+    if spec.dtype == "bf16" and spec.gated and spec.d_ff % 128:
+        # Gated bf16 tiles hold 128 gate and 128 up rows: the header's documented limit.
+        with pytest.raises(moe.MoeError) as exc:
+            layer.forward(*args)
+        assert exc.value.status == 2           # MOE_ERR_UNSUPPORTED
+        return
+    out, rt = layer.forward(*args, want_routing=True)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(layer.ws) == 0
+    g = {k_: to_host(v) for k_, v in rt.items()}
+    rg = oracle.route(g["logits_out"], spec.k, layer.K, flags & 3)
+    assert np.array_equal(g["ids_out"], rg["ids"]), "expert ids differ"
+    assert np.array_equal(g["w_out"].view(np.uint32), rg["w"].view(np.uint32)), "weights differ"
+    assert np.array_equal(g["slot_out"], rg["slot"]), "slots differ"
+    assert np.array_equal(g["drop_out"], rg["drop"]), "drop mask differs"
+    received = np.bincount(rg["ids"].ravel(), minlength=spec.E)
+    kept = np.bincount(rg["ids"][rg["slot"] >= 0], minlength=spec.E)
+    assert np.array_equal(g["counts_out"][:spec.E], received), "received counts differ"
+    assert np.array_equal(g["counts_out"][spec.E:], kept), "kept counts differ"
+    assert kept.max(initial=0) <= layer.K
+    _, ref = oracle.combine_tokens(L["x"], L["W1"], L["b1"], L["W2"], L["b2"], rg, flags=flags)
+    got = to_host(out)
+    assert_close(got, ref, spec.dtype, "layer output")
+    none_kept = ~(rg["slot"] >= 0).any(axis=1)
+    assert got[none_kept].tobytes() == L["x"][none_kept].tobytes()
