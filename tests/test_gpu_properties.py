@@ -74,3 +74,41 @@ def test_forward_random_layers(case):
     assert_close(got, ref, spec.dtype, "layer output")
     none_kept = ~(rg["slot"] >= 0).any(axis=1)
     assert got[none_kept].tobytes() == L["x"][none_kept].tobytes()
+
+
+@st.composite
+def tied_logits(draw):
+    T = draw(st.one_of(st.integers(1, 300), st.integers(1025, 5000)))
+    E = draw(st.integers(1, 64))
+    k = draw(st.integers(1, min(E, 8)))
+    C = draw(st.sampled_from([0.25, 0.5, 1.0, 1.5, math.inf]))
+    flags = draw(st.integers(0, 3))
+    levels = draw(st.integers(1, 4))           # how many distinct logit values: ties everywhere
+    seed = draw(st.integers(0, 2 ** 16))
+    rng = np.random.default_rng(seed)
+    vals = np.array([-1.0, 0.0, 0.5, 2.0], np.float32)[:levels]
+    L = vals[rng.integers(0, levels, size=(T, E))].astype(np.float32)
+    return L, T, E, k, C, flags
+
+
+@settings(max_examples=60, deadline=None, derandomize=True, print_blob=True,
+          suppress_health_check=[HealthCheck.too_slow, HealthCheck.data_too_large])
+@given(tied_logits())
+def test_route_heavy_ties(case):
+    """moe_route on logits drawn from at most four values: ties in the top-k (lower expert
+    wins) and at every capacity boundary (lower token wins, or the first K with arrival order)
+    must match the oracle bit for bit."""
+    from expert_ffn_layer_router_b200 import moe
+    L, T, E, k, C, flags = case
+    layer = moe.MoELayer(T, 64, 64, E, k, C, "bf16", flags=flags)
+    r = layer.route(to_dev(L))
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(layer.ws) == 0
+    g = {k_: to_host(v) for k_, v in r.items()}
+    ro = oracle.route(L, k, layer.K, flags)
+    assert np.array_equal(g["ids"], ro["ids"]), "expert ids differ"
+    assert np.array_equal(g["w"].view(np.uint32), ro["w"].view(np.uint32)), "weights differ"
+    assert np.array_equal(g["slot"], ro["slot"]), "slots differ"
+    assert np.array_equal(g["drop"], ro["drop"]), "drop mask differs"
+    kept = np.bincount(ro["ids"][ro["slot"] >= 0], minlength=E)
+    assert np.array_equal(g["counts"][E:], kept)
