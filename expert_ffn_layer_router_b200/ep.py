@@ -1,7 +1,7 @@
 """Expert parallelism: the layer's E experts split over the ranks of a process group.
 
-"Expert Networks > Worked Example: Expert Specialization" runs its four experts "at the same time
-on different hardware units"; the fused-MoE dataflow diagram sends each token's rows to its
+In "Expert Networks > Worked Example: Expert Specialization" the four experts run concurrently,
+each on its own piece of hardware; the fused-MoE dataflow diagram sends each token's rows to its
 experts and sums the k outputs back in token order.  Here every rank holds T_local tokens and
 E / world experts (rank r owns experts [r E_l, (r + 1) E_l)), and one forward gives, for the
 union of all ranks' tokens in rank order, exactly what the single-device layer gives for that

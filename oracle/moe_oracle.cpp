@@ -11,7 +11,7 @@
 //     than K tokens drops the ones with the lowest router confidence; a dropped token leaves the
 //     layer unchanged through the residual.
 //   * same page, the trace of token 0: h = W1 x + b1, a = SiLU(h), y = W2 a + b2, and the output
-//     is x + w * y with w the router's confidence weight for that expert.
+//     is x + w * y, w being how confident the router is in that expert.
 //   * same page, closing paragraph: each expert processes its kept tokens as one batch.
 //   * "Some Tokens Do Not Get In" (getbasislab.com), sections "Why there is a buffer" and "Past
 //     the edge": t*k token slots to fill, a fixed buffer per expert, overflow tokens take the

@@ -2,7 +2,7 @@
 expert outputs around the owner's capacity selection and FFN, with every compute step done by
 the oracle.  Each rank's outputs and routing must equal the single-batch oracle layer's on the
 union of both ranks' tokens, bit for bit ("Expert Networks > Worked Example: Expert
-Specialization": the experts run on different hardware units; the capacity, drop priority and
+Specialization": the experts run concurrently on separate hardware; the capacity, drop priority and
 slots are those of the whole batch)."""
 import math
 
