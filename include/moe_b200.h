@@ -218,7 +218,7 @@ moe_status moe_set_stage_events(void* const* events, int32_t n);
 /* moe_route without a workspace, for callers that cannot allocate device memory: plug-ins of an
  * inference engine that owns all device memory and gives its plug-ins no allocator, and serving
  * loops that may not call cudaMalloc/cudaFree on the request path (an allocation can
- * synchronise the device).  The paper has no counterpart; it is a deployment aid.
+ * synchronise the device).  The source pages describe no such call; it is a deployment aid.
  *   Same arguments, outputs and results as moe_route (bit for bit), minus ws/ws_bytes.  The
  *   router/capacity scratch lives in one fixed 8 MiB array of device memory per GPU, part of the
  *   library image and held by every GPU that loads the library until the process exits.  Needs
@@ -226,9 +226,8 @@ moe_status moe_set_stage_events(void* const* events, int32_t n);
  *   8*E*ceil(T/32) for the selection's token bitmaps); larger problems get MOE_ERR_WORKSPACE
  *   before anything is launched (T=16384 with E=64 fits; T=65536 with E=128 does not).
  *   The first call in a CUDA context (for runtime-API callers: the first call on a device) looks
- *   up the array's device address in that context and caches it; make that first call before
- *   any stream capture.  The cached address dies with its context: do not call it across a
- *   cudaDeviceReset of that device.
+ *   up the array's device address in that context and caches it.  The cached address dies with
+ *   its context: do not call it across a cudaDeviceReset of that device.
  *   The status word lives in the array too: each call clears it when it starts, and
  *   moe_get_device_status(NULL, 0, stream, &code) reads it (MOE_DEV_BAD_INDEX for an id out of
  *   range).
