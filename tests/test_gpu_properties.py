@@ -112,3 +112,52 @@ def test_route_heavy_ties(case):
     assert np.array_equal(g["drop"], ro["drop"]), "drop mask differs"
     kept = np.bincount(ro["ids"][ro["slot"] >= 0], minlength=E)
     assert np.array_equal(g["counts"][E:], kept)
+
+
+@st.composite
+def medium_layers(draw):
+    T = draw(st.integers(1, 20000))
+    E = draw(st.sampled_from([8, 16, 33, 64, 128]))
+    k = draw(st.integers(1, min(E, 8)))
+    d = 64 * draw(st.integers(1, 32))
+    flags = draw(st.integers(0, 7))
+    F = (128 if flags & 4 else 64) * draw(st.integers(1, 16 if flags & 4 else 32))
+    C = draw(st.sampled_from([0.5, 1.0, 1.25, math.inf]))
+    seed = draw(st.integers(0, 2 ** 16))
+    spec = inputs.LayerSpec("m", T, d, F, E, k, C, "bf16", router="normal", router_bias=0.5,
+                            bias_std=0.05, gated=bool(flags & 4))
+    return spec, flags, seed
+
+
+@settings(max_examples=12, deadline=None, derandomize=True, print_blob=True,
+          suppress_health_check=[HealthCheck.too_slow, HealthCheck.data_too_large])
+@given(medium_layers())
+def test_forward_random_medium_layers(case):
+    """Larger random bf16 layers (up to 20,000 tokens, d_model and d_ff up to 2048): several
+    m-tiles per expert, pair and single tiles, weight-streaming tiles and the tensor-core router
+    all occur.  Routing is checked on every token; outputs on 256 sampled tokens plus every
+    token whose pairs were all dropped."""
+    from expert_ffn_layer_router_b200 import moe
+    spec, flags, seed = case
+    L = inputs.make_layer(spec, seed=seed)
+    layer = moe.MoELayer(spec.T, spec.d_model, spec.d_ff, spec.E, spec.k, spec.C, spec.dtype,
+                         flags=flags)
+    args = [to_dev(L[n]) for n in ("x", "Wr", "br", "W1", "b1", "W2", "b2")]
+    out, rt = layer.forward(*args, want_routing=True)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(layer.ws) == 0
+    g = {k_: to_host(v) for k_, v in rt.items()}
+    rg = oracle.route(g["logits_out"], spec.k, layer.K, flags & 3)
+    assert np.array_equal(g["ids_out"], rg["ids"]), "expert ids differ"
+    assert np.array_equal(g["w_out"].view(np.uint32), rg["w"].view(np.uint32)), "weights differ"
+    assert np.array_equal(g["slot_out"], rg["slot"]), "slots differ"
+    assert np.array_equal(g["drop_out"], rg["drop"]), "drop mask differs"
+    rng = np.random.default_rng(seed)
+    none_kept = ~(rg["slot"] >= 0).any(axis=1)
+    tokens = np.unique(np.concatenate([rng.choice(spec.T, size=min(256, spec.T), replace=False),
+                                       np.nonzero(none_kept)[0][:64]])).astype(np.int32)
+    _, ref = oracle.combine_tokens(L["x"], L["W1"], L["b1"], L["W2"], L["b2"], rg, tokens,
+                                   flags=flags)
+    got = to_host(out)
+    assert_close(got[tokens], ref, spec.dtype, "layer output")
+    assert got[none_kept].tobytes() == L["x"][none_kept].tobytes()
