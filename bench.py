@@ -332,6 +332,22 @@ def run_cuda(args):
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
     # The clock sampler runs from the warm-up through the timed steps (same load); warm-up lasts
     # at least W steps and at least half a second so the sampler sees the part under load.
+    # Timed region: K steps, L2 flushed before each (outside the step's events).  The headline
+    # steps carry only a start and an end event; a second, instrumented run of K steps records
+    # an event between every stage (moe_set_stage_events) for the per-kernel durations.  Stage
+    # events cost the GPU about 2.5 us each, so the headline is taken without them.  All events
+    # are created before the warm-up (torch creates a CUDA event at its first record), so the GPU
+    # idles only for the synchronisation and barrier between the warm-up and the timed steps.
+    K = args.steps
+    ev_sets = {inst: [[torch.cuda.Event(enable_timing=True)
+                       for _ in range(moe.STAGE_EVENTS if inst else 2)] for _ in range(K)]
+               for inst in (False, True)}
+    for rows in ev_sets.values():
+        for row in rows:
+            for e in row:
+                e.record(stream)
+    torch.cuda.synchronize()
+
     sampler.start()
     t_end = time.perf_counter() + args.min_warmup_s
     n_warm = 0
@@ -341,23 +357,10 @@ def run_cuda(args):
         n_warm += 1
         if n_warm % 8 == 0:
             torch.cuda.synchronize()
-    torch.cuda.synchronize()
     launches_per_step = moe.moe_last_launch_count()
-    kept = int(counts[spec.E:].sum().item())
-    received = int(counts[:spec.E].sum().item())
-
-    # Timed region: K steps, L2 flushed before each (outside the step's events).  The headline
-    # steps carry only a start and an end event; a second, instrumented run of K steps records
-    # an event between every stage (moe_set_stage_events) for the per-kernel durations.  Stage
-    # events cost the GPU about 2.5 us each, so the headline is taken without them.
-    K = args.steps
 
     def timed_steps(instrumented):
-        n_ev = moe.STAGE_EVENTS if instrumented else 2
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(K)]
-        for row in evs:                   # torch creates the CUDA event at its first record
-            for e in row:
-                e.record(stream)
+        evs = ev_sets[instrumented]
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
@@ -381,6 +384,8 @@ def run_cuda(args):
     evs_plain = timed_steps(False)
     evs = timed_steps(True)
     clocks = sampler.stop()
+    kept = int(counts[spec.E:].sum().item())
+    received = int(counts[:spec.E].sum().item())
     stage_ms = np.zeros((K, moe.STAGE_EVENTS - 1))
     for i in range(K):
         for s in range(moe.STAGE_EVENTS - 1):
