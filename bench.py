@@ -612,16 +612,15 @@ def run_ep(args):
 
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    for row in evs:                       # created before the warm-up, as in the default mode
+        for e in row:
+            e.record(stream)
     sampler.start()
     for _ in range(max(args.warmup, 3)):
         flush.zero_()
         step()
-    torch.cuda.synchronize()
-    K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
-    for row in evs:
-        for e in row:
-            e.record(stream)
     torch.cuda.synchronize()
     dist.barrier()
     torch.cuda.synchronize()
