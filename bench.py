@@ -517,7 +517,9 @@ def run_cuda(args):
                    "l2": "flushed before every timed step (256 MiB write, outside the step's"
                          " events); per-step inputs %.0f MB" % (input_bytes / 1e6),
                    "timing": "value: K steps with start/end events only; kernels and roofline:"
-                             " a second run of K steps with an event between stages",
+                             " a second run of K steps with an event between stages; the timed"
+                             " steps follow the warm-up with no idle gap (sustained,"
+                             " power-capped state)",
                    "router_weights": "split into two bf16 terms once, before the timed steps"
                                      " (moe_prepare_router)",
                    "kept_pairs": kept, "received_pairs": received,
