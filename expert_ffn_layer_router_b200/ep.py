@@ -59,6 +59,12 @@ def _group_order(dest, world):
     P = dest.numel()
     if P == 0:
         return dest.clone(), torch.zeros(world, dtype=torch.int64, device=dest.device)
+    if world > 16:
+        # The one-hot prefix sums below take P * world words; with many ranks a stable sort is
+        # the smaller way to the same order.
+        counts = torch.zeros(world, dtype=torch.int64, device=dest.device).scatter_add_(
+            0, dest, torch.ones_like(dest))
+        return torch.argsort(dest, stable=True), counts
     csum = torch.cumsum(torch.nn.functional.one_hot(dest, world), dim=0)   # [P, world]
     counts = csum[-1]
     rank_in = csum.gather(1, dest.view(-1, 1)).view(-1) - 1
