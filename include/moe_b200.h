@@ -86,8 +86,9 @@ typedef struct {
  *     j = 0..k-1, one correctly rounded division each); the renormalised weights are the ones
  *     reported, used for drop priority and in the combine.
  *   MOE_FLAG_ARRIVAL_ORDER: an overflowing expert keeps the first K pairs in token order, the
- *     reading of "Some Tokens Do Not Get In", "Past the edge" (tokens are assigned in order and
- *     the next one does not get in once the buffer is full), instead of the highest weights. */
+ *     reading of "Some Tokens Do Not Get In", "Past the edge" (each expert's fixed buffer fills
+ *     first come, first served, and later tokens are turned away), instead of the highest
+ *     weights. */
 #define MOE_FLAG_RENORMALIZE 1u
 #define MOE_FLAG_ARRIVAL_ORDER 2u
 /* Expert variant: gated FFN, after the fused-MoE dataflow diagram (GEMM 1 writes gate and up
