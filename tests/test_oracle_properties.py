@@ -66,3 +66,37 @@ def test_route_against_exhaustive_reference(case):
                 assert r["drop"][tj] == 0 and r["slot"][tj] == kept_sorted.index(tj)
             else:
                 assert r["drop"][tj] == 1 and r["slot"][tj] == -1
+
+
+@st.composite
+def small_layers(draw):
+    from expert_ffn_layer_router_b200 import inputs
+    T = draw(st.integers(1, 24))
+    d = draw(st.sampled_from([4, 8, 16]))
+    F = draw(st.sampled_from([4, 8, 12]))
+    E = draw(st.integers(1, 5))
+    k = draw(st.integers(1, E))
+    C = draw(st.sampled_from([0.0, 0.5, 1.0, math.inf]))
+    flags = draw(st.integers(0, 7))
+    dtype = draw(st.sampled_from(["f32", "bf16"]))
+    seed = draw(st.integers(0, 2 ** 16))
+    spec = inputs.LayerSpec("p", T, d, F, E, k, C, dtype, router="normal", router_bias=0.3,
+                            bias_std=0.1, gated=bool(flags & 4))
+    return inputs.make_layer(spec, seed=seed), k, C, flags
+
+
+@settings(max_examples=150, deadline=None, derandomize=True)
+@given(small_layers())
+def test_forward_against_dense_reference(case):
+    """The oracle's layer output (float64, before rounding) equals every expert run on every
+    token in torch float64 and masked by the oracle's routing: x + sum over kept j of w * y
+    (plain or gated experts)."""
+    from tests.test_oracle_pins import dense_gated_reference, dense_reference
+    layer, k, C, flags = case
+    res = oracle.forward(layer["x"], layer["Wr"], layer["br"], layer["W1"], layer["b1"],
+                         layer["W2"], layer["b2"], k, C, flags=flags)
+    ref, _ = (dense_gated_reference if flags & oracle.GATED else dense_reference)(
+        layer, res["route"])
+    np.testing.assert_allclose(res["out_f64"], ref, rtol=0, atol=1e-12)
+    none_kept = ~(res["route"]["slot"] >= 0).any(axis=1)
+    assert res["out"][none_kept].tobytes() == layer["x"][none_kept].tobytes()
