@@ -100,3 +100,47 @@ def test_forward_against_dense_reference(case):
     np.testing.assert_allclose(res["out_f64"], ref, rtol=0, atol=1e-12)
     none_kept = ~(res["route"]["slot"] >= 0).any(axis=1)
     assert res["out"][none_kept].tobytes() == layer["x"][none_kept].tobytes()
+
+
+@st.composite
+def given_routings(draw):
+    T = draw(st.integers(1, 50))
+    E = draw(st.integers(1, 8))
+    k = draw(st.integers(1, E))
+    K = draw(st.integers(0, 2 * T))
+    flags = draw(st.sampled_from([0, 2]))
+    ties = draw(st.booleans())
+    seed = draw(st.integers(0, 2 ** 20))
+    rng = np.random.default_rng(seed)
+    ids = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    w = ((rng.integers(1, 4, size=(T, k)) * 0.25) if ties else rng.random((T, k))).astype(
+        np.float32)
+    return ids, w, E, K, flags
+
+
+@settings(max_examples=300, deadline=None, derandomize=True)
+@given(given_routings())
+def test_select_against_exhaustive_reference(case):
+    """Capacity selection of an arbitrary routing, and its expert-sorted layout: offsets are the
+    prefix sums of the kept counts and row offsets[e] + slot holds the kept token."""
+    ids, w, E, K, flags = case
+    T, k = ids.shape
+    r = oracle.select(ids, w, E, K, flags)
+    for e in range(E):
+        cand = [(t, j) for t in range(T) for j in range(k) if ids[t, j] == e]
+        ranked = sorted(cand) if flags & oracle.ARRIVAL_ORDER else \
+            sorted(cand, key=lambda tj: (-float(w[tj]), tj[0]))
+        keep = set(ranked[:K])
+        kept_sorted = sorted(keep)
+        assert r["kept"][e] == min(len(cand), K)
+        for tj in cand:
+            if tj in keep:
+                assert r["drop"][tj] == 0 and r["slot"][tj] == kept_sorted.index(tj)
+            else:
+                assert r["drop"][tj] == 1 and r["slot"][tj] == -1
+    offsets, rowtok = oracle.dispatch(ids, r["slot"], E)
+    assert offsets[0] == 0 and np.array_equal(np.diff(offsets), r["kept"])
+    for t in range(T):
+        for j in range(k):
+            if r["slot"][t, j] >= 0:
+                assert rowtok[offsets[ids[t, j]] + r["slot"][t, j]] == t
