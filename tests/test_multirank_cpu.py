@@ -3,6 +3,7 @@
 Each rank of ``bench.py --gpus N`` runs an independent batch (no collective on the data path);
 the only cross-rank steps are a barrier and the max over ranks of the device time.
 """
+import json
 import os
 import subprocess
 import sys
@@ -51,3 +52,21 @@ def test_reference_arm_under_torchrun_prints_once():
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1 and '"impl": "reference"' in lines[0]
+
+
+def test_reference_arm_line_has_the_contract_keys():
+    # One process, the worked example's shape: the reference arm's JSON line carries the keys the
+    # bench contract asks of it, with the variant options reflected in its workload.
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0",
+           "--config", "tiny_f32", "--drop-policy", "arrival"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads([l for l in r.stdout.splitlines() if l.startswith("{")][-1])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert "arrival-order capacity" in line["config"]["workload"]
